@@ -1,0 +1,334 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the oracle.
+
+Every check takes an ``oracle.Oracle`` (the committed build, or a deliberately
+altered one in test_oracle_mutants.py) and raises AssertionError when the
+oracle disagrees with:
+
+* the E2M1 bit-field definition (sign, 2 exponent bits with bias 1, 1 mantissa
+  bit, subnormal at exponent 0) and the table in golden/e2m1_values.txt;
+* brute-force nearest-value encoding over all 16 codes, with the tie rule
+  "exact midpoints go to the value whose mantissa bit is 0";
+* the rounding bound of a nearest-value quantiser and the storage layout
+  (two codes per byte, low nibble = even k; one scale per 32 along K);
+* the router's hand-worked cases (golden/router_cases.txt), numpy's stable
+  sort, the full softmax at k = E, and sum_j w = 1;
+* numpy's stable argsort for the grouping;
+* the closed form of a layer whose codes are all equal;
+* a dense, unpermuted brute-force layer written here with numpy.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# -- independent decoders ------------------------------------------------------
+
+def e2m1_from_bits(code: int) -> float:
+    """E2M1 value from its bit fields (OCP MX v1.0 FP4 element definition)."""
+    s, e, m = (code >> 3) & 1, (code >> 1) & 3, code & 1
+    mag = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0)
+    return -mag if s else mag
+
+
+E2M1_TABLE = np.array([e2m1_from_bits(c) for c in range(16)], dtype=np.float64)
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def dequant_dense(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """codes [..., K/2, N], scales [..., K/32, N] -> float64 [..., K, N]."""
+    lo = E2M1_TABLE[codes & 0x0F]
+    hi = E2M1_TABLE[codes >> 4]
+    K2, N = codes.shape[-2:]
+    vals = np.empty(codes.shape[:-2] + (2 * K2, N), dtype=np.float64)
+    vals[..., 0::2, :] = lo
+    vals[..., 1::2, :] = hi
+    s = np.repeat(bf16_to_f64(scales), 32, axis=-2)
+    return vals * s
+
+
+def brute_force_code(r: float) -> int:
+    """Nearest E2M1 code to r: minimum |r - value|; ties to mantissa bit 0; zero is code 0."""
+    best, best_d = None, None
+    for c in range(16):
+        d = abs(Fraction(float(r)) - Fraction(E2M1_TABLE[c]))
+        if best is None or d < best_d or (d == best_d and (best & 1) and not (c & 1)):
+            best, best_d = c, d
+    if E2M1_TABLE[best] == 0.0:
+        return 0
+    return best
+
+
+def nearest_bf16_bits(v: np.float32) -> int:
+    """bf16 pattern nearest to float32 v (ties to even), by enumerating neighbours."""
+    b = int(np.float32(v).view(np.uint32))
+    lo = b >> 16
+    cands = [lo, lo + 1]
+    fv = Fraction(float(v))
+
+    def val(p):
+        return Fraction(float(np.uint32(p << 16).view(np.float32)))
+    d0, d1 = abs(fv - val(cands[0])), abs(fv - val(cands[1]))
+    if d0 < d1:
+        return cands[0]
+    if d1 < d0:
+        return cands[1]
+    return cands[0] if cands[0] % 2 == 0 else cands[1]
+
+
+# -- checks ----------------------------------------------------------------------
+
+def check_e2m1_table(o):
+    rows = [ln.split() for ln in open(os.path.join(GOLDEN, "e2m1_values.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 16
+    for code_s, val_s in rows:
+        code = int(code_s)
+        assert float(val_s) == e2m1_from_bits(code)
+        assert o.e2m1_decode(code) == float(val_s), f"code {code}"
+
+
+def encode_probe_values(rng) -> np.ndarray:
+    grid = np.unique(np.abs(E2M1_TABLE))
+    mids = (grid[1:] + grid[:-1]) / 2
+    base = np.concatenate([grid, mids, [6.5, 7.0, 100.0, 1e-3, 0.0]])
+    near = np.concatenate([np.nextafter(base.astype(np.float32), np.float32(np.inf)),
+                           np.nextafter(base.astype(np.float32), np.float32(-np.inf))])
+    rnd = rng.uniform(-7.0, 7.0, 400).astype(np.float32)
+    v = np.concatenate([base.astype(np.float32), near, rnd])
+    return np.concatenate([v, -v]).astype(np.float32)
+
+
+def check_encode_bruteforce(o, rng):
+    for r in encode_probe_values(rng):
+        exp = brute_force_code(float(r))
+        got = o.e2m1_encode(float(r))
+        assert got == exp, f"encode({float(r)!r}) = {got}, brute force {exp}"
+
+
+def check_quantize_layout(o):
+    E, K, N = 2, 64, 3
+    for (e, k, n, v) in [(0, 0, 0, 0.3), (1, 37, 2, -1.7), (0, 63, 1, 5.0), (1, 32, 0, -0.02)]:
+        W = np.zeros((E, K, N), dtype=np.float32)
+        W[e, k, n] = v
+        codes, scales = o.quantize(W)
+        nz = np.argwhere(codes != 0)
+        assert nz.tolist() == [[e, k // 2, n]], nz
+        byte = int(codes[e, k // 2, n])
+        code = (byte & 0xF) if k % 2 == 0 else (byte >> 4)
+        other = (byte >> 4) if k % 2 == 0 else (byte & 0xF)
+        assert other == 0
+        # the one element is the group max: |v| / s is 6 up to bf16 rounding of s
+        assert code == (15 if v < 0 else 7), code
+        snz = np.argwhere(scales != 0)
+        assert snz.tolist() == [[e, k // 32, n]], snz
+        assert int(scales[e, k // 32, n]) == nearest_bf16_bits(np.float32(abs(np.float32(v))) / np.float32(6))
+
+
+def check_quantize_roundtrip(o, rng):
+    E, K, N = 3, 128, 40
+    W = (rng.standard_normal((E, K, N)) * 0.02).astype(np.float32)
+    W[0, 0:32, 0] = 0.0                        # an all-zero group
+    W[1, 32:64, 1] = np.float32(0.01)          # a constant group
+    codes, scales = o.quantize(W)
+    assert codes.shape == (E, K // 2, N) and scales.shape == (E, K // 32, N)
+    deq = dequant_dense(codes, scales)
+    s = np.repeat(bf16_to_f64(scales), 32, axis=1)
+    # scale = nearest bf16 to float32(max|w| / 6), per group and column
+    gmax = np.abs(W).reshape(E, K // 32, 32, N).max(axis=2)
+    for idx in [(0, 0, 0), (1, 1, 1), (2, 3, 39), (0, 2, 17)]:
+        q = np.float32(gmax[idx]) / np.float32(6)
+        assert int(scales[idx]) == nearest_bf16_bits(q)
+    assert np.all(scales[0, 0, 0] == 0) and np.all(deq[0, 0:32, 0] == 0)
+    # nearest-value rounding: |deq - w| <= s * (half the local grid gap), ratios within [-6, 6]
+    grid = np.unique(E2M1_TABLE)
+    r = W.astype(np.float64) / np.where(s == 0, 1, s)
+    inside = np.abs(r) <= 6
+    hi_idx = np.clip(np.searchsorted(grid, r, side="left"), 1, len(grid) - 1)
+    gap = grid[hi_idx] - grid[hi_idx - 1]
+    err = np.abs(deq - W.astype(np.float64))
+    bound = s * gap / 2 * (1 + 1e-6) + 1e-30
+    assert np.all(err[inside] <= bound[inside])
+    assert np.all(np.abs(r) <= 6.0 * (1 + 2.0 ** -7))   # bf16 rounding of s may push past 6
+    # spot-check codes against brute force
+    for (e, k, n) in [(0, 5, 3), (2, 77, 10), (1, 127, 39), (1, 40, 1)]:
+        byte = int(codes[e, k // 2, n])
+        code = (byte & 0xF) if k % 2 == 0 else (byte >> 4)
+        sv = float(bf16_to_f64(scales[e, k // 32, n]))
+        exp = 0 if sv == 0 else brute_force_code(float(np.float32(W[e, k, n]) / np.float32(sv)))
+        assert code == exp
+
+
+def check_router_golden(o):
+    for ln in open(os.path.join(GOLDEN, "router_cases.txt")):
+        if not ln.strip() or ln.startswith("#"):
+            continue
+        k_s, l_s, i_s, w_s = [p.strip() for p in ln.split("|")]
+        k = int(k_s)
+        logits = np.array([[float(v) for v in l_s.split()]], dtype=np.float32)
+        idx, w = o.route(logits, k)
+        assert idx[0].tolist() == [int(v) for v in i_s.split()], (ln, idx)
+        np.testing.assert_allclose(w[0], [float(v) for v in w_s.split()], rtol=2e-7, atol=0)
+
+
+def check_router_random(o, rng):
+    for (T, E, k) in [(7, 16, 3), (5, 128, 8), (3, 512, 10), (4, 9, 9), (6, 33, 1)]:
+        logits = rng.standard_normal((T, E)).astype(np.float32)
+        logits[0, 3] = logits[0, 5]                       # a deliberate tie
+        logits[1 % T, :] = np.round(logits[1 % T, :])     # many ties
+        idx, w = o.route(logits, k)
+        for t in range(T):
+            order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))
+            assert idx[t].tolist() == order[:k].tolist()
+            sel = logits[t, idx[t]].astype(np.float64)
+            ref = np.exp(sel - sel.max()) / np.exp(sel - sel.max()).sum()
+            np.testing.assert_allclose(w[t], ref, rtol=1e-6)
+            assert abs(float(w[t].astype(np.float64).sum()) - 1.0) <= 1e-6
+            assert np.all(np.diff(w[t].astype(np.float64)) <= 0)
+        if k == 1:
+            assert np.all(w == 1.0)
+        if k == E:   # full softmax of the row
+            for t in range(T):
+                full = np.exp(logits[t] - logits[t].max()) / np.exp(logits[t] - logits[t].max()).sum()
+                np.testing.assert_allclose(w[t], full[idx[t]], rtol=1e-6)
+
+
+def check_group(o, rng):
+    for (T, E, k) in [(1, 128, 8), (9, 16, 4), (64, 128, 8), (5, 4, 4)]:
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+        counts, offsets, sp, pr = o.group(idx, E)
+        flat = idx.reshape(-1)
+        assert counts.tolist() == np.bincount(flat, minlength=E).tolist()
+        assert offsets.tolist() == [0] + np.cumsum(np.bincount(flat, minlength=E)).tolist()
+        assert sp.tolist() == np.argsort(flat, kind="stable").tolist()
+        assert np.all(pr[sp] == np.arange(T * k))
+
+
+def _layer_inputs(rng, E, H, I, T, random_codes):
+    if random_codes:
+        gu_c = rng.integers(0, 256, (E, H // 2, 2 * I), dtype=np.uint8)
+        dn_c = rng.integers(0, 256, (E, I // 2, H), dtype=np.uint8)
+        # scales: bf16 patterns of magnitudes around 0.002..0.01
+        gu_s = (np.abs(rng.standard_normal((E, H // 32, 2 * I))) * 0.004 + 0.001).astype(np.float32)
+        dn_s = (np.abs(rng.standard_normal((E, I // 32, H))) * 0.004 + 0.001).astype(np.float32)
+        gu_s = (gu_s.view(np.uint32) >> 16).astype(np.uint16)
+        dn_s = (dn_s.view(np.uint32) >> 16).astype(np.uint16)
+    else:
+        Wgu = (rng.standard_normal((E, H, 2 * I)) * 0.02).astype(np.float32)
+        Wdn = (rng.standard_normal((E, I, H)) * 0.02).astype(np.float32)
+        return Wgu, Wdn
+    return gu_c, gu_s, dn_c, dn_s
+
+
+def _expert_weights(E, H, I, gu_c, gu_s, dn_c, dn_s):
+    import oracle as _oracle_pkg
+    ew = _oracle_pkg.ExpertWeights(E, H, I)
+    for e in range(E):
+        ew.set(e, gu_c[e], gu_s[e], dn_c[e], dn_s[e])
+    return ew
+
+
+def dense_layer_reference(x_bf16, logits, k, gu_c, gu_s, dn_c, dn_s):
+    """Unpermuted brute force: every token through every expert, weighted by the routing mask."""
+    T, H = x_bf16.shape
+    E = logits.shape[1]
+    I = dn_c.shape[1] * 2
+    x = bf16_to_f64(x_bf16)
+    Wgu = dequant_dense(gu_c, gu_s)       # [E, H, 2I]
+    Wdn = dequant_dense(dn_c, dn_s)       # [E, I, H]
+    y = np.zeros((T, H))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))
+        sel = order[:k]
+        ls = logits[t, sel].astype(np.float64)
+        wsel = (np.exp(ls - ls[0]) / np.exp(ls - ls[0]).sum()).astype(np.float32).astype(np.float64)
+        mask = np.zeros(E)
+        mask[sel] = wsel
+        for e in range(E):
+            h = x[t] @ Wgu[e]
+            g, u = h[:I], h[I:]
+            a = g / (1.0 + np.exp(-g)) * u
+            y[t] += mask[e] * (a @ Wdn[e])
+    return y
+
+
+def check_dense_bruteforce(o, rng):
+    for (E, H, I, T, k) in [(4, 64, 32, 3, 2), (6, 32, 64, 2, 6), (8, 256, 128, 4, 2)]:
+        gu_c, gu_s, dn_c, dn_s = _layer_inputs(rng, E, H, I, T, random_codes=True)
+        x = rng.standard_normal((T, H)).astype(np.float32)
+        x_bf16 = (x.view(np.uint32) >> 16).astype(np.uint16)
+        logits = rng.standard_normal((T, E)).astype(np.float32)
+        ew = _expert_weights(E, H, I, gu_c, gu_s, dn_c, dn_s)
+        y64, yb = o.moe_forward(ew, x_bf16, logits, k)
+        ref = dense_layer_reference(x_bf16, logits, k, gu_c, gu_s, dn_c, dn_s)
+        scale = np.abs(ref).max()
+        assert np.abs(y64 - ref).max() <= 1e-10 * scale, np.abs(y64 - ref).max() / scale
+
+
+def check_closed_form(o, rng):
+    E, H, I, T, k = 5, 96, 64, 3, 3
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    x_bf16 = (x.view(np.uint32) >> 16).astype(np.uint16)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    for c, cd, s_bits, sd_bits in [(2, 9, 0x3B80, 0x3C00), (7, 4, 0x3A00, 0x3B00), (13, 3, 0x3C80, 0x3A80)]:
+        gu_c = np.full((E, H // 2, 2 * I), c | (c << 4), dtype=np.uint8)
+        dn_c = np.full((E, I // 2, H), cd | (cd << 4), dtype=np.uint8)
+        gu_s = np.full((E, H // 32, 2 * I), s_bits, dtype=np.uint16)
+        dn_s = np.full((E, I // 32, H), sd_bits, dtype=np.uint16)
+        ew = _expert_weights(E, H, I, gu_c, gu_s, dn_c, dn_s)
+        y64, yb, act = o.moe_forward(ew, x_bf16, logits, k, want_act=True)
+        s = float(bf16_to_f64(s_bits))
+        sd = float(bf16_to_f64(sd_bits))
+        vc, vd = e2m1_from_bits(c), e2m1_from_bits(cd)
+        for t in range(T):
+            sx = math.fsum(bf16_to_f64(x_bf16[t]))
+            g = vc * s * sx
+            a = g / (1.0 + math.exp(-g)) * g
+            np.testing.assert_allclose(act[t * k:(t + 1) * k], a, rtol=1e-12, atol=1e-300)
+            np.testing.assert_allclose(y64[t], vd * sd * I * a, rtol=1e-6)
+
+
+def check_bf16_output_rounding(o, rng):
+    vals = [1.0, 1.0 + 2.0 ** -8, 1.0 + 2.0 ** -8 + 2.0 ** -40, 1.0 + 3 * 2.0 ** -8,
+            -(1.0 + 2.0 ** -8 - 2.0 ** -40), 3.14159, -2.5e-3, 1e-38, 0.0]
+    vals += list(rng.standard_normal(200) * 10.0)
+    for v in vals:
+        got = o.f64_to_bf16(v)
+        # exact: nearest bf16 (ties even) to the real number v
+        fv = Fraction(v)
+        f32 = np.float32(v)
+        b = int(f32.view(np.uint32)) >> 16
+        cands = {(b + d) & 0xFFFF for d in (-1, 0, 1, 2)}
+        best = None
+        for cnd in cands:
+            cf = float(np.uint32(cnd << 16).view(np.float32))
+            if not math.isfinite(cf):
+                continue
+            cv = Fraction(cf)
+            d = abs(fv - cv)
+            if best is None or d < best[0] or (d == best[0] and cnd % 2 == 0):
+                best = (d, cnd)
+        assert got == best[1], (v, hex(got), hex(best[1]))
+
+
+ALL_CHECKS = [
+    ("e2m1_table", lambda o, rng: check_e2m1_table(o)),
+    ("encode_bruteforce", check_encode_bruteforce),
+    ("quantize_layout", lambda o, rng: check_quantize_layout(o)),
+    ("quantize_roundtrip", check_quantize_roundtrip),
+    ("router_golden", lambda o, rng: check_router_golden(o)),
+    ("router_random", check_router_random),
+    ("group", check_group),
+    ("closed_form", check_closed_form),
+    ("dense_bruteforce", check_dense_bruteforce),
+    ("bf16_output_rounding", check_bf16_output_rounding),
+]

@@ -1,0 +1,50 @@
+"""The pins must reject plausible mistakes: each case below plants one mistake
+in a copy of oracle.c (on the CPU), builds it, and requires at least one pin of
+pins.py to fail on that build."""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import pins
+
+MUTANTS = [
+    ("nibble_order_swapped",
+     "int code = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
+     "int code = (k % 2 == 0) ? (byte >> 4) : (byte & 0x0F);"),
+    ("tie_rule_quarter", "if (a <= 0.25f) m = 0;", "if (a < 0.25f) m = 0;"),
+    ("tie_rule_five", "else if (a <= 5.0f) m = 6;", "else if (a < 5.0f) m = 6;"),
+    ("scale_divisor", "orc_f32_to_bf16_rne(mx / 6.0f)", "orc_f32_to_bf16_rne(mx / 4.0f)"),
+    ("encode_drops_sign", "return (r < 0.0f) ? (m | 8) : m;", "return m;"),
+    ("decode_table_entry", "{0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f}",
+     "{0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 5.0f}"),
+    ("gate_up_swapped", "double g = gu[i], u = gu[I + i];", "double g = gu[I + i], u = gu[i];"),
+    ("silu_sign", "act[i] = g / (1.0 + exp(-g)) * u;", "act[i] = g / (1.0 + exp(g)) * u;"),
+    ("router_ties_high", "return a < b;", "return a > b;"),
+    ("softmax_drops_term", "for (int j = 0; j < k; ++j) den +=", "for (int j = 1; j < k; ++j) den +="),
+    ("combine_unweighted", "y[h] += (double)w[j] * o[h];", "y[h] += o[h];"),
+    ("input_reversed", "gu[n] += x[kk] *", "gu[n] += x[H - 1 - kk] *"),
+    ("group_unstable", "for (int64_t p = 0; p < P; ++p)\n            if (idx[p] == e) {",
+     "for (int64_t p = P - 1; p >= 0; --p)\n            if (idx[p] == e) {"),
+    ("bf16_round_half_up", "u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0x8000u;"),
+    ("down_scale_group", "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[(k / 32) * N + n]);",
+     "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[((k / 32) / 2) * N + n]);"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_reject_mutant(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    path = tmp_path / "oracle_mut.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.build(force=True, src=str(path), out=str(tmp_path / f"liboracle_{name}.so"))
+    o = oracle.Oracle(lib)
+    failed = []
+    for cname, check in pins.ALL_CHECKS:
+        try:
+            check(o, np.random.default_rng(2024))
+        except (AssertionError, ValueError):
+            failed.append(cname)
+    assert failed, f"no pin rejects the planted mistake '{name}'"
