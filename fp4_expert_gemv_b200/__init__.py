@@ -1,0 +1,199 @@
+"""Python binding of the fe_moe C ABI (include/fe_moe.h): argument marshalling only.
+
+Every function named ``fe_moe_*`` here calls the C entry point of the same
+name in ``libfe_moe.so``; all computation runs in the library's CUDA kernels.
+The library must have been built (``python -m fp4_expert_gemv_b200.build``);
+importing this package without it raises ImportError: there is no fallback.
+
+``MoELayer`` is a convenience wrapper that takes torch tensors (device memory
+and streams only) and checks status codes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfe_moe.so")
+
+FE_OK = 0
+FE_ERR_INVALID_ARG = -1
+FE_ERR_UNSUPPORTED = -2
+FE_ERR_NOT_LOADED = -3
+FE_ERR_CAPACITY = -4
+FE_ERR_OOM = -5
+FE_ERR_CUDA = -6
+FE_ERR_DEVICE_STATUS = -7
+FE_DEVICE_BAD_EXPERT = 0x1
+FE_DEVICE_NAN_LOGIT = 0x2
+
+PATH_AUTO, PATH_GEMV, PATH_TCGEN05 = 0, 1, 2
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m fp4_expert_gemv_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_i32 = ctypes.c_int
+_i64 = ctypes.c_int64
+_st = ctypes.c_int
+
+_SIGS = {
+    "fe_moe_create": (_st, [_i32, _i32, _i32, _i32, ctypes.POINTER(_P)]),
+    "fe_moe_reserve": (_st, [_P, _i32, _i32]),
+    "fe_moe_load_packed": (_st, [_P, _P, _P, _P, _P, _i32, _P]),
+    "fe_moe_forward": (_st, [_P, _P, _P, _i32, _i32, _P, _P]),
+    "fe_moe_forward_host": (_st, [_P, _P, _P, _i32, _i32, _P, _P]),
+    "fe_moe_get_routing": (_st, [_P, _P, _P, _P, _P, _P]),
+    "fe_moe_get_status": (_st, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "fe_moe_set_path": (_st, [_P, _i32]),
+    "fe_moe_status_string": (ctypes.c_char_p, [_st]),
+    "fe_moe_destroy": (None, [_P]),
+    "fe_moe_pack_host": (_st, [_P, _i64, _i64, _i64, _P, _P]),
+    "fe_moe_pack_device": (_st, [_P, _i64, _i64, _i64, _P, _P, _P]),
+    "fe_moe_device_bytes": (ctypes.c_size_t, [_P]),
+}
+
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+    globals()[_name] = _f
+
+
+class FeMoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = fe_moe_status_string(status)
+        super().__init__(f"{what}: {msg.decode() if msg else status} ({status})")
+
+
+def check(status: int, what: str = "fe_moe") -> None:
+    if status != FE_OK:
+        raise FeMoeError(status, what)
+
+
+def _dptr(t) -> int:
+    """Device address of a torch tensor (or an int address)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class MoELayer:
+    """One fe_moe handle: create + reserve, load packed weights, forward."""
+
+    def __init__(self, E: int, H: int, I: int, max_T: int, max_top_k: int, group: int = 32):
+        h = _P()
+        check(fe_moe_create(E, H, I, group, ctypes.byref(h)), "fe_moe_create")
+        self.h = h
+        self.E, self.H, self.I = E, H, I
+        self.max_T, self.max_top_k = max_T, max_top_k
+        try:
+            check(fe_moe_reserve(self.h, max_T, max_top_k), "fe_moe_reserve")
+        except Exception:
+            fe_moe_destroy(self.h)
+            self.h = None
+            raise
+
+    def load_packed(self, gu_codes, gu_scales, dn_codes, dn_scales, stream=None):
+        """Device torch tensors (uint8 codes, int16/uint16/bfloat16 scales) or host numpy arrays."""
+        import numpy as np
+        if isinstance(gu_codes, np.ndarray):
+            arrs = [np.ascontiguousarray(a) for a in (gu_codes, gu_scales, dn_codes, dn_scales)]
+            check(fe_moe_load_packed(self.h, *[a.ctypes.data for a in arrs], 0, _stream_ptr(stream)),
+                  "fe_moe_load_packed")
+            import torch
+            torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+        else:
+            for t in (gu_codes, gu_scales, dn_codes, dn_scales):
+                assert t.is_cuda and t.is_contiguous()
+            check(fe_moe_load_packed(self.h, _dptr(gu_codes), _dptr(gu_scales), _dptr(dn_codes), _dptr(dn_scales),
+                                     1, _stream_ptr(stream)), "fe_moe_load_packed")
+
+    def forward(self, x_bf16, logits, top_k: int, y_bf16=None, stream=None):
+        import torch
+        T = x_bf16.shape[0]
+        if y_bf16 is None:
+            y_bf16 = torch.empty((T, self.H), dtype=torch.bfloat16, device=x_bf16.device)
+        check(fe_moe_forward(self.h, _dptr(x_bf16), _dptr(logits), T, top_k, _dptr(y_bf16), _stream_ptr(stream)),
+              "fe_moe_forward")
+        return y_bf16
+
+    def forward_host(self, x_bf16_host, logits_host, top_k: int, y_bf16_host, stream=None):
+        """Host (ideally pinned) numpy/torch CPU buffers in and out; synchronous."""
+        def hp(a):
+            return a.ctypes.data if hasattr(a, "ctypes") else a.data_ptr()
+        T = x_bf16_host.shape[0]
+        check(fe_moe_forward_host(self.h, hp(x_bf16_host), hp(logits_host), T, top_k, hp(y_bf16_host),
+                                  _stream_ptr(stream)), "fe_moe_forward_host")
+        return y_bf16_host
+
+    def routing(self, T: int, top_k: int, stream=None):
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        idx = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, top_k), dtype=torch.float32, device=dev)
+        offsets = torch.empty(self.E + 1, dtype=torch.int32, device=dev)
+        sp = torch.empty(T * top_k, dtype=torch.int32, device=dev)
+        check(fe_moe_get_routing(self.h, _dptr(idx), _dptr(w), _dptr(offsets), _dptr(sp), _stream_ptr(stream)),
+              "fe_moe_get_routing")
+        return idx, w, offsets, sp
+
+    def status(self):
+        bits = ctypes.c_uint32(0)
+        st = fe_moe_get_status(self.h, ctypes.byref(bits))
+        return st, bits.value
+
+    def set_path(self, path: int):
+        check(fe_moe_set_path(self.h, path), "fe_moe_set_path")
+
+    def device_bytes(self) -> int:
+        return fe_moe_device_bytes(self.h)
+
+    def close(self):
+        if getattr(self, "h", None):
+            fe_moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def pack_host(W):
+    """numpy float32 [E, K, N] -> (codes uint8 [E, K/2, N], scales uint16 [E, K/32, N]) via fe_moe_pack_host."""
+    import numpy as np
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    E, K, N = W.shape
+    codes = np.empty((E, K // 2, N), dtype=np.uint8)
+    scales = np.empty((E, K // 32, N), dtype=np.uint16)
+    check(fe_moe_pack_host(W.ctypes.data, E, K, N, codes.ctypes.data, scales.ctypes.data), "fe_moe_pack_host")
+    return codes, scales
+
+
+def pack_device(W, codes=None, scales=None, stream=None):
+    """torch float32 CUDA [E, K, N] -> (codes uint8, scales int16 bf16-bits) via fe_moe_pack_device."""
+    import torch
+    E, K, N = W.shape
+    if codes is None:
+        codes = torch.empty((E, K // 2, N), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty((E, K // 32, N), dtype=torch.int16, device=W.device)
+    check(fe_moe_pack_device(_dptr(W), E, K, N, _dptr(codes), _dptr(scales), _stream_ptr(stream)),
+          "fe_moe_pack_device")
+    return codes, scales

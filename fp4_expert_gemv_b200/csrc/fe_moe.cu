@@ -1,0 +1,462 @@
+// fe_moe C ABI: handle, workspace, weight loading and the forward enqueue.
+// The declarations and the contract of every entry point are in
+// include/fe_moe.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/fe_moe.h"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "pack.cuh"
+#include "route.cuh"
+
+namespace fe_host {
+void pack(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales);
+}
+
+struct fe_moe_s {
+    int E = 0, H = 0, I = 0;
+    int device = 0;
+    int path = 0;
+    // column tiles (gemv.cuh): gate_up tiles hold TN gate + TN up columns
+    int gu_TW = 64, gu_tiles = 0;
+    int dn_TW = 128, dn_tiles = 0;
+    uint8_t* gu_codes = nullptr;
+    uint16_t* gu_scales = nullptr;
+    uint8_t* dn_codes = nullptr;
+    uint16_t* dn_scales = nullptr;
+    bool loaded = false;
+    // workspace
+    int max_T = 0, max_k = 0;
+    int32_t* idx = nullptr;
+    float* w = nullptr;
+    int32_t* counts = nullptr;
+    int32_t* offsets = nullptr;
+    int32_t* sorted_pair = nullptr;
+    int32_t* pair_row = nullptr;
+    int32_t* active = nullptr;
+    int32_t* n_active = nullptr;
+    int32_t* max_count = nullptr;
+    float* act = nullptr;
+    float* o = nullptr;
+    uint32_t* status = nullptr;
+    uint16_t* x_stage = nullptr;
+    float* logits_stage = nullptr;
+    uint16_t* y_stage = nullptr;
+    size_t weight_bytes = 0, work_bytes = 0;
+    int last_T = 0, last_k = 0;
+};
+
+namespace {
+
+#define FE_CUDA_TRY(expr)                                \
+    do {                                                 \
+        cudaError_t err__ = (expr);                      \
+        if (err__ != cudaSuccess) {                      \
+            return err__ == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA; \
+        }                                                \
+    } while (0)
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev)
+    {
+        if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard()
+    {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
+template <typename T>
+cudaError_t dmalloc(T** p, size_t n, size_t* acc)
+{
+    *p = nullptr;
+    if (n == 0) n = 1;
+    cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T));
+    if (e == cudaSuccess && acc) *acc += n * sizeof(T);
+    return e;
+}
+
+void free_workspace(fe_moe_s* h)
+{
+    void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
+                    h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+    h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
+    h->pair_row = nullptr; h->active = nullptr; h->n_active = nullptr; h->max_count = nullptr; h->act = nullptr;
+    h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
+    h->max_T = h->max_k = 0;
+    h->work_bytes = 0;
+}
+
+// Tile width TW = 16 * C columns for a matrix with K rows of reduction and N
+// columns: one thread per (16-column chunk, 32-k group), at most 256 threads
+// per CTA, C a power of two up to 32 dividing the columns (for the fused
+// gate_up matrix the tile holds TW/2 gate and TW/2 up columns, so TW/2 must
+// divide I).  Returns 0 if no width fits.
+int pick_tile_width(int K, int cols, bool gate_up)
+{
+    const int G = K / 32;
+    for (int C = 32; C >= (gate_up ? 2 : 1); C >>= 1) {   // gate_up: 16-byte chunks never straddle gate and up
+        if (C * G > 256) continue;
+        if (gate_up ? (cols % (8 * C) == 0) : (cols % (16 * C) == 0)) return 16 * C;
+    }
+    return 0;
+}
+
+int roundup32(int v) { return (v + 31) / 32 * 32; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int NT, bool GU>
+cudaError_t launch_gemv(const fe::GemvParams& p, int grid, int threads, cudaStream_t s)
+{
+    const size_t smem = fe::gemv_smem_bytes<NT>(p.K, p.TW, threads);
+    fe::gemv_kernel<NT, GU><<<grid, threads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <int NT, bool GU>
+cudaError_t allow_gemv_smem(int K, int TW)
+{
+    const size_t smem = fe::gemv_smem_bytes<NT>(K, TW, roundup32((TW / 16) * (K / 32)));
+    return cudaFuncSetAttribute(fe::gemv_kernel<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+// Opt the kernels into the dynamic shared memory this layer shape needs
+// (once, outside any stream capture).
+cudaError_t configure_kernels(const fe_moe_s* h)
+{
+    cudaError_t e = cudaFuncSetAttribute(fe::route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)fe::route_smem_bytes(h->E, 1024));
+    if (e == cudaSuccess) e = allow_gemv_smem<1, true>(h->H, h->gu_TW);
+    if (e == cudaSuccess) e = allow_gemv_smem<4, true>(h->H, h->gu_TW);
+    if (e == cudaSuccess) e = allow_gemv_smem<1, false>(h->I, h->dn_TW);
+    if (e == cudaSuccess) e = allow_gemv_smem<4, false>(h->I, h->dn_TW);
+    return e;
+}
+
+fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s)
+{
+    const int P = T * k;
+    const int max_active = std::min(h->E, P);
+    fe::GemvParams gp{};
+    gp.offsets = h->offsets;
+    gp.active = h->active;
+    gp.n_active = h->n_active;
+    gp.sorted_pair = h->sorted_pair;
+    gp.top_k = k;
+    // gate_up + SwiGLU: K = H, tiles of 32 gate + 32 up columns
+    gp.codes = h->gu_codes;
+    gp.scales = h->gu_scales;
+    gp.K = h->H;
+    gp.TW = h->gu_TW;
+    gp.n_tiles = h->gu_tiles;
+    gp.N_out = h->I;
+    gp.x = x;
+    gp.act_in = nullptr;
+    gp.out = h->act;
+    int threads = roundup32((h->gu_TW / 16) * (h->H / 32));
+    cudaError_t e = (T == 1) ? launch_gemv<1, true>(gp, max_active * h->gu_tiles, threads, s)
+                             : launch_gemv<4, true>(gp, max_active * h->gu_tiles, threads, s);
+    if (e != cudaSuccess) return FE_ERR_CUDA;
+    // down: K = I
+    gp.codes = h->dn_codes;
+    gp.scales = h->dn_scales;
+    gp.K = h->I;
+    gp.TW = h->dn_TW;
+    gp.n_tiles = h->dn_tiles;
+    gp.N_out = h->H;
+    gp.x = nullptr;
+    gp.act_in = h->act;
+    gp.out = h->o;
+    threads = roundup32((h->dn_TW / 16) * (h->I / 32));
+    e = (T == 1) ? launch_gemv<1, false>(gp, max_active * h->dn_tiles, threads, s)
+                 : launch_gemv<4, false>(gp, max_active * h->dn_tiles, threads, s);
+    if (e != cudaSuccess) return FE_ERR_CUDA;
+    return FE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fe_moe_status_string(fe_status s)
+{
+    switch (s) {
+        case FE_OK: return "ok";
+        case FE_ERR_INVALID_ARG: return "invalid argument";
+        case FE_ERR_UNSUPPORTED: return "unsupported";
+        case FE_ERR_NOT_LOADED: return "weights not loaded";
+        case FE_ERR_CAPACITY: return "T or top_k above the reserved workspace";
+        case FE_ERR_OOM: return "device out of memory";
+        case FE_ERR_CUDA: return "CUDA error";
+        case FE_ERR_DEVICE_STATUS: return "a kernel flagged bad data";
+    }
+    return "unknown status";
+}
+
+fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out)
+{
+    if (!out) return FE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (group != 32) return FE_ERR_UNSUPPORTED;
+    if (E < 1 || E > 1024 || H <= 0 || I <= 0 || H % 32 || I % 32) return FE_ERR_INVALID_ARG;
+    // gate_up tiles: TW/2 gate + TW/2 up columns, so TW/2 must divide I
+    const int gu_TW = pick_tile_width(H, I, true);
+    const int dn_TW = pick_tile_width(I, H, false);
+    if (gu_TW == 0 || dn_TW == 0) return FE_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FE_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FE_ERR_CUDA;
+    if (prop.major != 10) return FE_ERR_UNSUPPORTED;
+    fe_moe_s* h = new (std::nothrow) fe_moe_s();
+    if (!h) return FE_ERR_OOM;
+    h->E = E; h->H = H; h->I = I; h->device = dev;
+    h->gu_TW = gu_TW;
+    h->gu_tiles = I / (gu_TW / 2);
+    h->dn_TW = dn_TW;
+    h->dn_tiles = H / dn_TW;
+    size_t acc = 0;
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = dmalloc(&h->gu_codes, (size_t)E * (H / 2) * (2 * (size_t)I), &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->gu_scales, (size_t)E * (H / 32) * (2 * (size_t)I), &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->dn_codes, (size_t)E * (I / 2) * (size_t)H, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->dn_scales, (size_t)E * (I / 32) * (size_t)H, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->status, 1, &acc);
+    if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) {
+        fe_moe_destroy(h);
+        return e == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA;
+    }
+    h->weight_bytes = acc;
+    *out = h;
+    return FE_OK;
+}
+
+fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
+{
+    if (!h || max_T < 1 || max_top_k < 1 || max_top_k > h->E) return FE_ERR_INVALID_ARG;
+    if ((int64_t)max_T * max_top_k > (int64_t)1 << 26) return FE_ERR_UNSUPPORTED;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FE_ERR_CUDA;
+    uint32_t* keep_status = h->status;
+    h->status = nullptr;
+    free_workspace(h);
+    h->status = keep_status;
+    const size_t P = (size_t)max_T * max_top_k;
+    size_t acc = 0;
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = dmalloc(&h->idx, P, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->w, P, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->counts, (size_t)h->E, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->offsets, (size_t)h->E + 1, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->sorted_pair, P, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->pair_row, P, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->active, (size_t)h->E, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->n_active, 1, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->max_count, 1, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->act, P * h->I, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->o, P * h->H, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->x_stage, (size_t)max_T * h->H, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->logits_stage, (size_t)max_T * h->E, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->y_stage, (size_t)max_T * h->H, &acc);
+    if (e != cudaSuccess) {
+        keep_status = h->status;
+        h->status = nullptr;
+        free_workspace(h);
+        h->status = keep_status;
+        return e == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA;
+    }
+    if (configure_kernels(h) != cudaSuccess) return FE_ERR_CUDA;
+    h->max_T = max_T;
+    h->max_k = max_top_k;
+    h->work_bytes = acc;
+    return FE_OK;
+}
+
+fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t* gu_scales, const uint8_t* dn_codes,
+                             const uint16_t* dn_scales, int src_on_device, fe_stream_t stream)
+{
+    if (!h || !gu_codes || !gu_scales || !dn_codes || !dn_scales) return FE_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t E = h->E, H = h->H, I = h->I;
+    const size_t gu_c = (size_t)E * (H / 2) * (2 * I), gu_s = (size_t)E * (H / 32) * (2 * I);
+    const size_t dn_c = (size_t)E * (I / 2) * H, dn_s = (size_t)E * (I / 32) * H;
+    const uint8_t* sgc = gu_codes;
+    const uint16_t* sgs = gu_scales;
+    const uint8_t* sdc = dn_codes;
+    const uint16_t* sds = dn_scales;
+    void* staging = nullptr;
+    if (!src_on_device) {
+        const size_t bytes = gu_c + 2 * gu_s + dn_c + 2 * dn_s;
+        FE_CUDA_TRY(cudaMallocAsync(&staging, bytes, s));
+        uint8_t* b = static_cast<uint8_t*>(staging);
+        FE_CUDA_TRY(cudaMemcpyAsync(b, gu_codes, gu_c, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c, gu_scales, 2 * gu_s, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c + 2 * gu_s, dn_codes, dn_c, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c + 2 * gu_s + dn_c, dn_scales, 2 * dn_s, cudaMemcpyHostToDevice, s));
+        sgc = b;
+        sgs = reinterpret_cast<const uint16_t*>(b + gu_c);
+        sdc = b + gu_c + 2 * gu_s;
+        sds = reinterpret_cast<const uint16_t*>(b + gu_c + 2 * gu_s + dn_c);
+    } else if (!aligned16(gu_codes) || !aligned16(gu_scales) || !aligned16(dn_codes) || !aligned16(dn_scales)) {
+        return FE_ERR_INVALID_ARG;
+    }
+    fe::RelayoutParams rp{};
+    rp.src_codes = sgc; rp.src_scales = sgs; rp.dst_codes = h->gu_codes; rp.dst_scales = h->gu_scales;
+    rp.E = E; rp.K = H; rp.N = 2 * I; rp.TW = h->gu_TW; rp.gate_up = 1;
+    fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
+    rp.src_codes = sdc; rp.src_scales = sds; rp.dst_codes = h->dn_codes; rp.dst_scales = h->dn_scales;
+    rp.K = I; rp.N = H; rp.TW = h->dn_TW; rp.gate_up = 0;
+    fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
+    FE_CUDA_TRY(cudaGetLastError());
+    if (staging) FE_CUDA_TRY(cudaFreeAsync(staging, s));
+    h->loaded = true;
+    return FE_OK;
+}
+
+fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k, void* y_bf16,
+                         fe_stream_t stream)
+{
+    if (!h || T < 0 || top_k < 1 || top_k > h->E) return FE_ERR_INVALID_ARG;
+    if (T == 0) return FE_OK;
+    if (!x_bf16 || !router_logits || !y_bf16 || x_bf16 == y_bf16) return FE_ERR_INVALID_ARG;
+    if (!h->loaded) return FE_ERR_NOT_LOADED;
+    if (T > h->max_T || top_k > h->max_k) return FE_ERR_CAPACITY;
+    if ((reinterpret_cast<uintptr_t>(x_bf16) & 3u) || (reinterpret_cast<uintptr_t>(y_bf16) & 3u) ||
+        (reinterpret_cast<uintptr_t>(router_logits) & 3u))
+        return FE_ERR_INVALID_ARG;
+    if (h->path == 2) return FE_ERR_UNSUPPORTED;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int P = T * top_k;
+
+    fe::RouteParams rp{};
+    rp.logits = router_logits; rp.T = T; rp.E = h->E; rp.k = top_k;
+    rp.idx = h->idx; rp.w = h->w; rp.counts = h->counts; rp.offsets = h->offsets;
+    rp.sorted_pair = h->sorted_pair; rp.pair_row = h->pair_row; rp.active = h->active;
+    rp.n_active = h->n_active; rp.max_count = h->max_count; rp.status = h->status;
+    const int rthreads = std::min(1024, std::max(32, roundup32(std::max(P, 32 * std::min(T, 32)))));
+    fe::route_group_kernel<<<1, rthreads, fe::route_smem_bytes(h->E, rthreads), s>>>(rp);
+    if (cudaGetLastError() != cudaSuccess) return FE_ERR_CUDA;
+
+    fe_status st = gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
+    if (st != FE_OK) return st;
+
+    dim3 cgrid((h->H / 2 + 255) / 256, T);
+    fe::combine_kernel<<<cgrid, 256, 0, s>>>(h->o, h->w, h->pair_row, h->H, top_k,
+                                              static_cast<__nv_bfloat16*>(y_bf16));
+    if (cudaGetLastError() != cudaSuccess) return FE_ERR_CUDA;
+    h->last_T = T;
+    h->last_k = top_k;
+    return FE_OK;
+}
+
+fe_status fe_moe_forward_host(fe_moe_t h, const uint16_t* x_host, const float* logits_host, int T, int top_k,
+                              uint16_t* y_host, fe_stream_t stream)
+{
+    if (!h || T < 0 || top_k < 1 || top_k > h->E) return FE_ERR_INVALID_ARG;
+    if (T == 0) return FE_OK;
+    if (!x_host || !logits_host || !y_host) return FE_ERR_INVALID_ARG;
+    if (!h->loaded) return FE_ERR_NOT_LOADED;
+    if (T > h->max_T || top_k > h->max_k) return FE_ERR_CAPACITY;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    FE_CUDA_TRY(cudaMemcpyAsync(h->x_stage, x_host, sizeof(uint16_t) * (size_t)T * h->H, cudaMemcpyHostToDevice, s));
+    FE_CUDA_TRY(cudaMemcpyAsync(h->logits_stage, logits_host, sizeof(float) * (size_t)T * h->E,
+                                cudaMemcpyHostToDevice, s));
+    fe_status st = fe_moe_forward(h, h->x_stage, h->logits_stage, T, top_k, h->y_stage, stream);
+    if (st != FE_OK) return st;
+    FE_CUDA_TRY(cudaMemcpyAsync(y_host, h->y_stage, sizeof(uint16_t) * (size_t)T * h->H, cudaMemcpyDeviceToHost, s));
+    FE_CUDA_TRY(cudaStreamSynchronize(s));
+    return FE_OK;
+}
+
+fe_status fe_moe_get_routing(fe_moe_t h, int32_t* idx, float* w, int32_t* offsets, int32_t* sorted_pair,
+                             fe_stream_t stream)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    if (!h->idx) return FE_ERR_CAPACITY;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t P = (size_t)h->last_T * h->last_k;
+    if (idx && P) FE_CUDA_TRY(cudaMemcpyAsync(idx, h->idx, sizeof(int32_t) * P, cudaMemcpyDeviceToDevice, s));
+    if (w && P) FE_CUDA_TRY(cudaMemcpyAsync(w, h->w, sizeof(float) * P, cudaMemcpyDeviceToDevice, s));
+    if (offsets)
+        FE_CUDA_TRY(cudaMemcpyAsync(offsets, h->offsets, sizeof(int32_t) * (h->E + 1), cudaMemcpyDeviceToDevice, s));
+    if (sorted_pair && P)
+        FE_CUDA_TRY(cudaMemcpyAsync(sorted_pair, h->sorted_pair, sizeof(int32_t) * P, cudaMemcpyDeviceToDevice, s));
+    return FE_OK;
+}
+
+fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    uint32_t v = 0;
+    FE_CUDA_TRY(cudaDeviceSynchronize());
+    FE_CUDA_TRY(cudaMemcpy(&v, h->status, sizeof(v), cudaMemcpyDeviceToHost));
+    FE_CUDA_TRY(cudaMemset(h->status, 0, sizeof(v)));
+    if (bits) *bits = v;
+    return v ? FE_ERR_DEVICE_STATUS : FE_OK;
+}
+
+fe_status fe_moe_set_path(fe_moe_t h, int path)
+{
+    if (!h || path < 0 || path > 2) return FE_ERR_INVALID_ARG;
+    h->path = path;
+    return FE_OK;
+}
+
+void fe_moe_destroy(fe_moe_t h)
+{
+    if (!h) return;
+    {
+        DeviceGuard g(h->device);
+        cudaDeviceSynchronize();
+        free_workspace(h);
+        void* ptrs[] = {h->gu_codes, h->gu_scales, h->dn_codes, h->dn_scales};
+        for (void* p : ptrs)
+            if (p) cudaFree(p);
+    }
+    delete h;
+}
+
+size_t fe_moe_device_bytes(fe_moe_t h) { return h ? h->weight_bytes + h->work_bytes : 0; }
+
+fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales)
+{
+    if (!W || !codes || !scales || E < 1 || K < 32 || N < 1 || K % 32) return FE_ERR_INVALID_ARG;
+    fe_host::pack(W, E, K, N, codes, scales);
+    return FE_OK;
+}
+
+fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,
+                             fe_stream_t stream)
+{
+    if (!W || !codes || !scales || E < 1 || K < 32 || N < 1 || K % 32) return FE_ERR_INVALID_ARG;
+    const int64_t total = E * (K / 32) * N;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, 148 * 32);
+    fe::pack_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(W, E, K, N, codes, scales);
+    return cudaGetLastError() == cudaSuccess ? FE_OK : FE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+/*
+ * fe_moe: one packed FP4 mixture-of-experts FFN layer on an NVIDIA B200 (sm_100a).
+ *
+ * The layer is the packed MoE decode layer of the "FireEcho Engine" page
+ * (sections "The Goliath Kernel: Why It's Fast" and "Speed Optimization
+ * History", steps 1-5: grouped dispatch, fused gate_up projection, single-token
+ * decode path, multi-expert kernel, all experts in one contiguous buffer whose
+ * expert IDs are read from GPU memory), with the SiLU(gate)*up product of the
+ * "FastInfer" page (section "Confirmed elementwise SwiGLU scheduling"):
+ *
+ *   router   per token t: the top_k experts by logit (ties to the lower expert
+ *            index) in descending order are slots j = 0..top_k-1; slot weights
+ *            w[t][j] = softmax over the top_k selected logits;
+ *   grouping pair p = t*top_k + j goes to expert idx[t][j]; pairs are grouped
+ *            by expert, ordered by pair id inside an expert;
+ *   gate_up  h = x[t] . W_gu[e] (K = H, N = 2I), gate = h[0:I], up = h[I:2I],
+ *            act = silu(gate) * up;
+ *   down     o = act . W_dn[e] (K = I, N = H);
+ *   combine  y[t] = sum_j w[t][j] * o_{t,j}, summed in slot order, rounded
+ *            once to bfloat16.
+ *
+ * Weight format (what fe_moe_load_packed accepts): each expert matrix W[K][N]
+ * is stored as 4-bit E2M1 codes (bit 3 sign, magnitudes 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6; code 8 decodes to zero), two per byte with the LOW nibble holding the
+ * even k, all experts in one contiguous [E][K/2][N] byte buffer, plus one
+ * bfloat16 scale per group of 32 consecutive k in a [E][K/32][N] buffer:
+ * W[e][k][n] = e2m1(code) * scale[e][k/32][n].  The fused gate_up matrix has
+ * N = 2I columns, the gate columns [0, I) first and the up columns [I, 2I)
+ * second.  Weights are dequantised in registers inside the kernels; no
+ * dequantised weight is ever written to memory.
+ *
+ * Conventions for every entry point:
+ *  - return FE_OK (0) or a negative fe_status; no exception crosses the ABI;
+ *  - "device" pointers are CUDA device (or managed) memory on the handle's
+ *    device, "host" pointers are ordinary host memory (pinned memory makes the
+ *    copies asynchronous);
+ *  - fe_stream_t is a cudaStream_t (NULL = the legacy default stream);
+ *  - the library owns its weight copies and workspace; the caller owns x,
+ *    logits, y and the stream; one handle must not be used on two streams at
+ *    the same time;
+ *  - arguments are validated on the host before anything is enqueued; an
+ *    argument error enqueues nothing.
+ */
+#ifndef FE_MOE_H
+#define FE_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct fe_moe_s* fe_moe_t;
+typedef struct CUstream_st* fe_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+    FE_OK = 0,
+    FE_ERR_INVALID_ARG = -1,   /* bad dimension, null pointer, top_k out of range, ... */
+    FE_ERR_UNSUPPORTED = -2,   /* valid but not supported here (group != 32, no sm_100 GPU) */
+    FE_ERR_NOT_LOADED = -3,    /* forward before fe_moe_load_packed */
+    FE_ERR_CAPACITY = -4,      /* T or top_k above what fe_moe_reserve reserved */
+    FE_ERR_OOM = -5,           /* a device allocation failed */
+    FE_ERR_CUDA = -6,          /* a CUDA runtime call failed */
+    FE_ERR_DEVICE_STATUS = -7  /* a kernel flagged bad data (see fe_moe_get_status) */
+} fe_status;
+
+/* Device-side problem bits, reported through fe_moe_get_status. */
+#define FE_DEVICE_BAD_EXPERT 0x1   /* an expert id outside [0, E) reached a kernel */
+#define FE_DEVICE_NAN_LOGIT 0x2    /* a NaN router logit (treated as -inf) */
+
+/* Create a handle for a layer of E experts, hidden size H and expert
+ * intermediate size I on the current CUDA device.  group must be 32; H and I
+ * must be positive multiples of 32; E in [1, 1024].  Allocates the weight
+ * buffers (E * (H*2I + I*H) * 9/16 bytes) but no workspace. */
+fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out);
+
+/* Allocate the forward workspace for up to max_T tokens and top_k <= max_top_k.
+ * Synchronous, allocating, not capturable; call it before capturing forward in
+ * a CUDA graph.  Calling it again with larger limits re-allocates. */
+fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k);
+
+/* Load packed weights in the format above (sizes follow from E, H, I):
+ *   gate_up_codes  uint8 [E][H/2][2I],  gate_up_scales bf16 [E][H/32][2I],
+ *   down_codes     uint8 [E][I/2][H],   down_scales    bf16 [E][I/32][H].
+ * src_on_device = 1: the four pointers are device memory; 0: host memory.
+ * The library re-lays the bytes out into its own device buffers (column tiles
+ * for the kernels); the caller's buffers may be freed after the stream has
+ * passed this call.  Enqueued on stream; returns after enqueueing. */
+fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
+                             const uint8_t* down_codes, const uint16_t* down_scales, int src_on_device,
+                             fe_stream_t stream);
+
+/* The layer: y = MoE(x).  x_bf16 device bf16 [T][H], router_logits device
+ * float [T][E], y_bf16 device bf16 [T][H] (must not alias x).  T = 0 is a
+ * no-op.  1 <= top_k <= min(E, max_top_k), T <= max_T.  Asynchronous on
+ * stream: no host synchronisation and no allocation, so it can be captured in
+ * a CUDA graph and replayed with new contents in the same buffers.  The
+ * routing (idx, w, grouping) stays in the workspace until the next call. */
+fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k,
+                         void* y_bf16, fe_stream_t stream);
+
+/* The layer on HOST buffers: copies x and the logits to the device, runs
+ * fe_moe_forward and copies y back, then waits for the stream.  Same argument
+ * rules as fe_moe_forward (T <= max_T).  Synchronous. */
+fe_status fe_moe_forward_host(fe_moe_t h, const uint16_t* x_bf16_host, const float* router_logits_host, int T,
+                              int top_k, uint16_t* y_bf16_host, fe_stream_t stream);
+
+/* Copy the routing of the last forward into caller device buffers (any may
+ * be NULL): idx int32 [T][top_k], w float [T][top_k], offsets int32 [E+1]
+ * (exclusive scan of the per-expert pair counts), sorted_pair int32
+ * [T*top_k] (pair ids ordered by (expert, pair id)).  Enqueued on stream. */
+fe_status fe_moe_get_routing(fe_moe_t h, int32_t* idx, float* w, int32_t* offsets, int32_t* sorted_pair,
+                             fe_stream_t stream);
+
+/* Wait for the device and return FE_ERR_DEVICE_STATUS if a kernel flagged a
+ * problem since the last call (the bits go to *bits if non-NULL), FE_OK
+ * otherwise; clears the flags. */
+fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
+
+/* Force a compute path for the gate_up / down projections: 0 = automatic
+ * (by tokens per expert), 1 = the CUDA-core GEMV kernels, 2 = the tcgen05
+ * tensor-core grouped GEMM.  For tests and measurements. */
+fe_status fe_moe_set_path(fe_moe_t h, int path);
+
+/* Human-readable text of a status code (static storage). */
+const char* fe_moe_status_string(fe_status s);
+
+/* Free every buffer of the handle.  Waits for the device first. */
+void fe_moe_destroy(fe_moe_t h);
+
+/* The load-time packer: float W [E][K][N] -> E2M1 codes [E][K/2][N] and bf16
+ * scales [E][K/32][N].  Per group of 32 along k and column n: scale =
+ * bf16_rne(max|w| / 6) (the division in float32); code = the E2M1 value
+ * nearest to w / scale (float32 division), exact midpoints to the value with
+ * an even mantissa bit, ratios beyond 6 clamped to 6, a zero magnitude stored
+ * as code 0, an all-zero group as scale 0 and codes 0.  K % 32 == 0.
+ * Host version: host pointers, multithreaded, synchronous. */
+fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales);
+
+/* The same packer on the GPU: device pointers, enqueued on stream.  Produces
+ * bytes identical to fe_moe_pack_host. */
+fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,
+                             fe_stream_t stream);
+
+/* Bytes of device memory the handle holds (weights + workspace). */
+size_t fe_moe_device_bytes(fe_moe_t h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FE_MOE_H */

@@ -157,3 +157,45 @@ WORKLOADS = {
 }
 STACK_LAYERS = 48
 STACK_SEED0 = 1000
+
+
+# -- device copy of the generator (synth.cu, built into libfe_synth.so) ----------
+
+_DEVICE_LIB = None
+
+
+def _device_lib():
+    global _DEVICE_LIB
+    if _DEVICE_LIB is None:
+        import ctypes
+        import os
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfe_synth.so")
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is not built; run `python -m fp4_expert_gemv_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, u64, i64 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64
+        lib.fe_synth_gate_up.argtypes = [P, u64, i64, i64, i64, P]
+        lib.fe_synth_down.argtypes = [P, u64, i64, i64, i64, P]
+        lib.fe_synth_normal.argtypes = [P, u64, u64, i64, ctypes.c_float, P]
+        for f in (lib.fe_synth_gate_up, lib.fe_synth_down, lib.fe_synth_normal):
+            f.restype = ctypes.c_int
+        _DEVICE_LIB = lib
+    return _DEVICE_LIB
+
+
+def device_gate_up(dst_ptr: int, seed: int, E: int, H: int, I: int, stream_ptr: int) -> None:
+    """Fill float32 device memory [E, H, 2I] with weights_gate_up(seed, E, H, I)."""
+    if _device_lib().fe_synth_gate_up(dst_ptr, seed, E, H, I, stream_ptr) != 0:
+        raise RuntimeError("fe_synth_gate_up launch failed")
+
+
+def device_down(dst_ptr: int, seed: int, E: int, I: int, H: int, stream_ptr: int) -> None:
+    """Fill float32 device memory [E, I, H] with weights_down(seed, E, I, H)."""
+    if _device_lib().fe_synth_down(dst_ptr, seed, E, I, H, stream_ptr) != 0:
+        raise RuntimeError("fe_synth_down launch failed")
+
+
+def device_normal(dst_ptr: int, seed: int, tid: int, count: int, scale: float, stream_ptr: int) -> None:
+    """Fill float32 device memory [count] with normal_f32(seed, tid, i) * float32(scale)."""
+    if _device_lib().fe_synth_normal(dst_ptr, seed, tid, count, scale, stream_ptr) != 0:
+        raise RuntimeError("fe_synth_normal launch failed")

@@ -1,0 +1,80 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+header declares, and its host packer reproduces the oracle's quantiser."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fe_moe.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?(fe_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ["fe_moe_create", "fe_moe_load_packed", "fe_moe_forward", "fe_moe_destroy",
+                     "fe_moe_reserve", "fe_moe_get_routing", "fe_moe_get_status", "fe_moe_pack_host"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    import fp4_expert_gemv_b200 as fe
+    lib = ctypes.CDLL(fe.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding wraps each of them under the same name
+    for n in declared_functions():
+        assert hasattr(fe, n), n
+
+
+def test_status_strings():
+    import fp4_expert_gemv_b200 as fe
+    for code in range(0, -8, -1):
+        assert fe.fe_moe_status_string(code)
+    assert fe.fe_moe_status_string(-4) == b"T or top_k above the reserved workspace"
+
+
+def test_pack_host_matches_oracle_quantiser():
+    import fp4_expert_gemv_b200 as fe
+    rng = np.random.default_rng(5)
+    cases = [(rng.standard_normal((2, 64, 40)) * 0.02).astype(np.float32),
+             (rng.standard_normal((1, 96, 8)) * 5).astype(np.float32)]
+    W = np.zeros((2, 64, 16), np.float32)
+    W[0, 0:8, 3] = [3.0, 0.125, 0.375, 0.625, 0.875, 1.25, 1.75, 2.5]   # exact midpoints
+    W[1, 0:8, 4] = [-3.0, -0.125, -0.375, -0.625, -0.875, -1.25, -1.75, -2.5]
+    W[1, 32:64, 9] = 1e-3
+    cases.append(W)
+    # every ratio the encoder can see, through a constant scale of 1 (group max 6)
+    r = pins.encode_probe_values(rng)
+    r = r[np.abs(r) <= 6.0]
+    n = (r.size + 30) // 31
+    V = np.zeros((1, 32, n), np.float32)
+    V[0, 0, :] = 6.0
+    V[0, 1:, :].reshape(-1)[: r.size] = r
+    V[0, 1:, :] = np.pad(r, (0, 31 * n - r.size)).reshape(31, n)
+    cases.append(V)
+    orc = oracle.default()
+    for W in cases:
+        c, s = fe.pack_host(W)
+        c_ref, s_ref = orc.quantize(W)
+        assert np.array_equal(s, s_ref)
+        assert np.array_equal(c, c_ref)
+
+
+def test_synth_device_library_is_built():
+    path = os.path.join(ROOT, "synth", "libfe_synth.so")
+    assert os.path.exists(path)
+    lib = ctypes.CDLL(path)
+    for n in ("fe_synth_gate_up", "fe_synth_down", "fe_synth_normal"):
+        assert hasattr(lib, n)
