@@ -32,6 +32,8 @@ METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of B200 peak) at T=
 WORKLOAD = "decode_e128_t1"
 LAYERS = 48
 NOMINAL_HBM_GBS = 8000.0
+KERNEL_NAMES = {1: "whole layer on the GEMV chain (route + gate_up + down + combine, 4 kernels)",
+                3: "decode_kernel (whole layer, one cooperative launch); per-launch time = step time / layers"}
 BYTES_PER_EXPERT = lambda H, I: (H // 2) * 2 * I + (H // 32) * 2 * I * 2 + (I // 2) * H + (I // 32) * H * 2  # noqa: E731
 
 
@@ -276,6 +278,7 @@ def run_gpu(args):
     for l, m in enumerate(stack):
         idx, _, _, _ = m.routing(T, k)
         distinct.append(len(set(idx.cpu().numpy().reshape(-1).tolist())))
+    path, kernels_per_layer = stack[0].last_forward_info()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         forward_all(s)
@@ -354,12 +357,12 @@ def run_gpu(args):
         "hbm_gbs_achieved": achieved,
         "hbm_frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "whole layer (route + gate_up + down + combine)",
+                     "traffic": None, "kernel": KERNEL_NAMES.get(path, str(path)),
                      "peak_kind": peak_kind, "algorithmic_bytes_per_layer": bytes_layer[0]},
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 4 * layers * args.steps,
+        "gpu_launches": kernels_per_layer * layers * args.steps,
         "setup_s": setup_s,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -27,10 +27,10 @@ FE_ERR_DEVICE_STATUS = -7
 FE_DEVICE_BAD_EXPERT = 0x1
 FE_DEVICE_NAN_LOGIT = 0x2
 
-PATH_AUTO, PATH_GEMV, PATH_TCGEN05 = 0, 1, 2
+PATH_AUTO, PATH_GEMV, PATH_TCGEN05, PATH_FUSED_DECODE = 0, 1, 2, 3
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m fp4_expert_gemv_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python fp4_expert_gemv_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -48,11 +48,14 @@ _SIGS = {
     "fe_moe_get_routing": (_st, [_P, _P, _P, _P, _P, _P]),
     "fe_moe_get_status": (_st, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "fe_moe_set_path": (_st, [_P, _i32]),
+    "fe_moe_last_forward_info": (_st, [_P, ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+    "fe_moe_set_trace": (_st, [_P, _P]),
     "fe_moe_status_string": (ctypes.c_char_p, [_st]),
     "fe_moe_destroy": (None, [_P]),
     "fe_moe_pack_host": (_st, [_P, _i64, _i64, _i64, _P, _P]),
     "fe_moe_pack_device": (_st, [_P, _i64, _i64, _i64, _P, _P, _P]),
     "fe_moe_device_bytes": (ctypes.c_size_t, [_P]),
+    "fe_moe_last_error": (ctypes.c_char_p, []),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -66,7 +69,10 @@ class FeMoeError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         msg = fe_moe_status_string(status)
-        super().__init__(f"{what}: {msg.decode() if msg else status} ({status})")
+        detail = ""
+        if status in (FE_ERR_CUDA, FE_ERR_OOM):
+            detail = " [" + (fe_moe_last_error() or b"").decode(errors="replace") + "]"
+        super().__init__(f"{what}: {msg.decode() if msg else status} ({status}){detail}")
 
 
 def check(status: int, what: str = "fe_moe") -> None:
@@ -159,6 +165,11 @@ class MoELayer:
 
     def set_path(self, path: int):
         check(fe_moe_set_path(self.h, path), "fe_moe_set_path")
+
+    def last_forward_info(self):
+        path, kernels = _i32(0), _i32(0)
+        check(fe_moe_last_forward_info(self.h, ctypes.byref(path), ctypes.byref(kernels)), "fe_moe_last_forward_info")
+        return path.value, kernels.value
 
     def device_bytes(self) -> int:
         return fe_moe_device_bytes(self.h)

@@ -3,7 +3,8 @@
   fp4_expert_gemv_b200/libfe_moe.so   the layer (C ABI of include/fe_moe.h)
   synth/libfe_synth.so                the seeded weight generator used by tests and the benchmark
 
-Run ``python -m fp4_expert_gemv_b200.build`` (or ``__graft_entry__.build()``).
+Run ``python fp4_expert_gemv_b200/build.py`` (or ``__graft_entry__.build()``); the package
+itself cannot be imported before the library exists.
 """
 from __future__ import annotations
 

@@ -7,9 +7,11 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "../../include/fe_moe.h"
 #include "common.cuh"
+#include "decode.cuh"
 #include "gemv.cuh"
 #include "pack.cuh"
 #include "route.cuh"
@@ -22,13 +24,13 @@ struct fe_moe_s {
     int E = 0, H = 0, I = 0;
     int device = 0;
     int path = 0;
+    int sm_count = 0;
+    int smem_optin = 0;
     // column tiles (gemv.cuh): gate_up tiles hold TN gate + TN up columns
     int gu_TW = 64, gu_tiles = 0;
     int dn_TW = 128, dn_tiles = 0;
-    uint8_t* gu_codes = nullptr;
-    uint16_t* gu_scales = nullptr;
-    uint8_t* dn_codes = nullptr;
-    uint16_t* dn_scales = nullptr;
+    uint8_t* gu_tiles_buf = nullptr;   // [E][gu_tiles] tiles: codes then scales
+    uint8_t* dn_tiles_buf = nullptr;   // [E][dn_tiles]
     bool loaded = false;
     // workspace
     int max_T = 0, max_k = 0;
@@ -43,22 +45,34 @@ struct fe_moe_s {
     int32_t* max_count = nullptr;
     float* act = nullptr;
     float* o = nullptr;
+    unsigned long long* act_ll = nullptr;   // fused decode: tagged act words
+    int32_t* plan_first = nullptr;          // fused decode: work split per nd
+    unsigned* dec_sync = nullptr;           // fused decode: finished CTAs, epoch
+    unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
     uint32_t* status = nullptr;
     uint16_t* x_stage = nullptr;
     float* logits_stage = nullptr;
     uint16_t* y_stage = nullptr;
     size_t weight_bytes = 0, work_bytes = 0;
     int last_T = 0, last_k = 0;
+    int last_path = 0, last_kernels = 0;
 };
 
 namespace {
 
-#define FE_CUDA_TRY(expr)                                \
-    do {                                                 \
-        cudaError_t err__ = (expr);                      \
-        if (err__ != cudaSuccess) {                      \
-            return err__ == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA; \
-        }                                                \
+// Text of the last CUDA failure seen by this thread (fe_moe_last_error).
+thread_local char g_last_error[256] = "";
+
+fe_status record_cuda(cudaError_t e, const char* where)
+{
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+    return e == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA;
+}
+
+#define FE_CUDA_TRY(expr)                                 \
+    do {                                                  \
+        cudaError_t err__ = (expr);                       \
+        if (err__ != cudaSuccess) return record_cuda(err__, #expr); \
     } while (0)
 
 struct DeviceGuard {
@@ -88,12 +102,16 @@ cudaError_t dmalloc(T** p, size_t n, size_t* acc)
 void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
-                    h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage};
+                    h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
+                    h->act_ll, h->dec_sync, h->plan_first};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
     h->pair_row = nullptr; h->active = nullptr; h->n_active = nullptr; h->max_count = nullptr; h->act = nullptr;
     h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
+    h->act_ll = nullptr;
+    h->dec_sync = nullptr;
+    h->plan_first = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -132,16 +150,115 @@ cudaError_t allow_gemv_smem(int K, int TW)
     return cudaFuncSetAttribute(fe::gemv_kernel<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
+using DecodeFn = void (*)(fe::DecodeParams);
+
+DecodeFn decode_kernel_for(int C)
+{
+    switch (C) {
+        case 2: return fe::decode_kernel<2>;
+        case 4: return fe::decode_kernel<4>;
+        case 8: return fe::decode_kernel<8>;
+        case 16: return fe::decode_kernel<16>;
+        default: return fe::decode_kernel<32>;
+    }
+}
+
+uint32_t gu_tile_bytes(const fe_moe_s* h) { return (uint32_t)((h->H / 2) * h->gu_TW + (h->H / 32) * h->gu_TW * 2); }
+uint32_t dn_tile_bytes(const fe_moe_s* h) { return (uint32_t)((h->I / 2) * 16 + (h->I / 32) * 32); }
+
+fe::DecodePlan plan_for(const fe_moe_s* h, int nd)
+{
+    return fe::decode_plan(nd, h->H, gu_tile_bytes(h), h->gu_tiles, dn_tile_bytes(h), h->sm_count);
+}
+
+// Largest per-CTA weight bytes of the fused decode split over every possible
+// number of distinct routed experts, or 0 if T, top_k or the shape exceed the
+// fused kernel.
+size_t decode_weight_bytes(const fe_moe_s* h, int T, int k)
+{
+    const int P = T * k;
+    if (P > fe::kDecMaxPairs || h->sm_count <= 0 || h->I > 1024 || h->E > 1024 || h->H > 8192) return 0;
+    size_t worst = 0;
+    const int nd_max = std::min(h->E, P);
+    for (int nd = 1; nd <= nd_max; ++nd) {
+        const fe::DecodePlan plan = plan_for(h, nd);
+        for (int c = 0; c < h->sm_count; ++c) {
+            const int a = fe::decode_first_unit(plan, c), b = fe::decode_first_unit(plan, c + 1);
+            if (b - a > fe::kDecMaxItems) return 0;
+            size_t bytes = 0;
+            for (int u = a; u < b; ++u) bytes += (size_t)fe::decode_unit_bytes(plan, u);
+            worst = std::max(worst, bytes);
+        }
+    }
+    return (worst + 127) / 128 * 128;
+}
+
+// Work-split table of the fused kernel: first unit of CTA c for nd distinct experts.
+cudaError_t build_plan_table(fe_moe_s* h)
+{
+    const int cols = h->sm_count + 1;
+    std::vector<int32_t> tab((size_t)(fe::kDecMaxPairs + 1) * cols, 0);
+    for (int nd = 1; nd <= fe::kDecMaxPairs; ++nd) {
+        const fe::DecodePlan plan = plan_for(h, nd);
+        for (int c = 0; c <= h->sm_count; ++c) tab[(size_t)nd * cols + c] = fe::decode_first_unit(plan, c);
+    }
+    cudaError_t e = cudaMalloc(&h->plan_first, tab.size() * sizeof(int32_t));
+    if (e != cudaSuccess) return e;
+    h->work_bytes += tab.size() * sizeof(int32_t);
+    return cudaMemcpy(h->plan_first, tab.data(), tab.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+}
+
+size_t decode_smem_total(const fe_moe_s* h, size_t wbytes, int T, int k)
+{
+    return fe::decode_smem_layout((uint32_t)wbytes, T, k, h->H, h->I, h->E, h->gu_TW).total;
+}
+
+fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, int k, void* y, size_t wbytes,
+                      cudaStream_t s)
+{
+    fe::DecodeParams dp{};
+    dp.x = static_cast<const uint16_t*>(x);
+    dp.logits = logits;
+    dp.y = static_cast<uint16_t*>(y);
+    dp.T = T; dp.E = h->E; dp.H = h->H; dp.I = h->I; dp.k = k;
+    dp.gu_tiles = h->gu_tiles_buf; dp.gu_ntiles = h->gu_tiles; dp.gu_tile_bytes = gu_tile_bytes(h);
+    dp.dn_tiles = h->dn_tiles_buf; dp.dn_tile_bytes = dn_tile_bytes(h);
+    dp.plan_first = h->plan_first;
+    dp.idx = h->idx; dp.w = h->w; dp.counts = h->counts; dp.offsets = h->offsets;
+    dp.sorted_pair = h->sorted_pair; dp.pair_row = h->pair_row;
+    dp.act = h->act_ll;
+    dp.sync = h->dec_sync;
+    dp.trace = h->trace;
+    dp.status = h->status;
+    dp.timeout_ns = 200ull * 1000 * 1000;
+    dp.weight_bytes = (uint32_t)wbytes;
+    dp.bulk_inputs = aligned16(x) && aligned16(logits) && ((size_t)T * h->E) % 4 == 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(h->sm_count);
+    cfg.blockDim = dim3(fe::kDecThreads);
+    cfg.dynamicSmemBytes = decode_smem_total(h, wbytes, T, k);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    FE_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel_for(h->gu_TW / 16), dp));
+    return FE_OK;
+}
+
 // Opt the kernels into the dynamic shared memory this layer shape needs
 // (once, outside any stream capture).
 cudaError_t configure_kernels(const fe_moe_s* h)
 {
     cudaError_t e = cudaFuncSetAttribute(fe::route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)fe::route_smem_bytes(h->E, 1024));
+                                         (int)fe::route_smem_bytes(h->E, fe::kRouteMaxThreads));
     if (e == cudaSuccess) e = allow_gemv_smem<1, true>(h->H, h->gu_TW);
     if (e == cudaSuccess) e = allow_gemv_smem<4, true>(h->H, h->gu_TW);
     if (e == cudaSuccess) e = allow_gemv_smem<1, false>(h->I, h->dn_TW);
     if (e == cudaSuccess) e = allow_gemv_smem<4, false>(h->I, h->dn_TW);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel_for(h->gu_TW / 16),
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_optin);
     return e;
 }
 
@@ -156,8 +273,7 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
     gp.sorted_pair = h->sorted_pair;
     gp.top_k = k;
     // gate_up + SwiGLU: K = H, tiles of 32 gate + 32 up columns
-    gp.codes = h->gu_codes;
-    gp.scales = h->gu_scales;
+    gp.tiles = h->gu_tiles_buf;
     gp.K = h->H;
     gp.TW = h->gu_TW;
     gp.n_tiles = h->gu_tiles;
@@ -168,10 +284,9 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
     int threads = roundup32((h->gu_TW / 16) * (h->H / 32));
     cudaError_t e = (T == 1) ? launch_gemv<1, true>(gp, max_active * h->gu_tiles, threads, s)
                              : launch_gemv<4, true>(gp, max_active * h->gu_tiles, threads, s);
-    if (e != cudaSuccess) return FE_ERR_CUDA;
+    if (e != cudaSuccess) return record_cuda(e, "gate_up gemv launch");
     // down: K = I
-    gp.codes = h->dn_codes;
-    gp.scales = h->dn_scales;
+    gp.tiles = h->dn_tiles_buf;
     gp.K = h->I;
     gp.TW = h->dn_TW;
     gp.n_tiles = h->dn_tiles;
@@ -182,7 +297,7 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
     threads = roundup32((h->dn_TW / 16) * (h->I / 32));
     e = (T == 1) ? launch_gemv<1, false>(gp, max_active * h->dn_tiles, threads, s)
                  : launch_gemv<4, false>(gp, max_active * h->dn_tiles, threads, s);
-    if (e != cudaSuccess) return FE_ERR_CUDA;
+    if (e != cudaSuccess) return record_cuda(e, "down gemv launch");
     return FE_OK;
 }
 
@@ -213,26 +328,31 @@ fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out)
     if (E < 1 || E > 1024 || H <= 0 || I <= 0 || H % 32 || I % 32) return FE_ERR_INVALID_ARG;
     // gate_up tiles: TW/2 gate + TW/2 up columns, so TW/2 must divide I
     const int gu_TW = pick_tile_width(H, I, true);
-    const int dn_TW = pick_tile_width(I, H, false);
+    // down tiles are 16 columns wide: the h-slice one CTA of the fused decode
+    // kernel owns for every routed expert (and a 1-chunk tile for the GEMV)
+    const int dn_TW = (I / 32 <= 256) ? 16 : 0;
     if (gu_TW == 0 || dn_TW == 0) return FE_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FE_ERR_CUDA;
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FE_ERR_CUDA;
     if (prop.major != 10) return FE_ERR_UNSUPPORTED;
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return FE_ERR_CUDA;
     fe_moe_s* h = new (std::nothrow) fe_moe_s();
     if (!h) return FE_ERR_OOM;
     h->E = E; h->H = H; h->I = I; h->device = dev;
+    h->sm_count = prop.multiProcessorCount;
+    h->smem_optin = optin;
     h->gu_TW = gu_TW;
     h->gu_tiles = I / (gu_TW / 2);
     h->dn_TW = dn_TW;
     h->dn_tiles = H / dn_TW;
     size_t acc = 0;
     cudaError_t e = cudaSuccess;
-    if (e == cudaSuccess) e = dmalloc(&h->gu_codes, (size_t)E * (H / 2) * (2 * (size_t)I), &acc);
-    if (e == cudaSuccess) e = dmalloc(&h->gu_scales, (size_t)E * (H / 32) * (2 * (size_t)I), &acc);
-    if (e == cudaSuccess) e = dmalloc(&h->dn_codes, (size_t)E * (I / 2) * (size_t)H, &acc);
-    if (e == cudaSuccess) e = dmalloc(&h->dn_scales, (size_t)E * (I / 32) * (size_t)H, &acc);
+    // codes (K/2 bytes per column) + scales (K/32 bf16 per column)
+    if (e == cudaSuccess) e = dmalloc(&h->gu_tiles_buf, (size_t)E * (2 * (size_t)I) * (H / 2 + H / 16), &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->dn_tiles_buf, (size_t)E * (size_t)H * (I / 2 + I / 16), &acc);
     if (e == cudaSuccess) e = dmalloc(&h->status, 1, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(uint32_t));
     if (e != cudaSuccess) {
@@ -272,6 +392,12 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = dmalloc(&h->x_stage, (size_t)max_T * h->H, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->logits_stage, (size_t)max_T * h->E, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->y_stage, (size_t)max_T * h->H, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->act_ll, (size_t)fe::kDecMaxPairs * h->I, &acc);
+    if (e == cudaSuccess) e = cudaMemset(h->act_ll, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
+    if (e == cudaSuccess) e = dmalloc(&h->dec_sync, 2, &acc);
+    if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, 2 * sizeof(unsigned));
+    h->work_bytes = 0;
+    if (e == cudaSuccess) e = build_plan_table(h);
     if (e != cudaSuccess) {
         keep_status = h->status;
         h->status = nullptr;
@@ -279,10 +405,10 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
         h->status = keep_status;
         return e == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA;
     }
-    if (configure_kernels(h) != cudaSuccess) return FE_ERR_CUDA;
+    FE_CUDA_TRY(configure_kernels(h));
     h->max_T = max_T;
     h->max_k = max_top_k;
-    h->work_bytes = acc;
+    h->work_bytes += acc;
     return FE_OK;
 }
 
@@ -317,10 +443,10 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
         return FE_ERR_INVALID_ARG;
     }
     fe::RelayoutParams rp{};
-    rp.src_codes = sgc; rp.src_scales = sgs; rp.dst_codes = h->gu_codes; rp.dst_scales = h->gu_scales;
+    rp.src_codes = sgc; rp.src_scales = sgs; rp.dst = h->gu_tiles_buf;
     rp.E = E; rp.K = H; rp.N = 2 * I; rp.TW = h->gu_TW; rp.gate_up = 1;
     fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
-    rp.src_codes = sdc; rp.src_scales = sds; rp.dst_codes = h->dn_codes; rp.dst_scales = h->dn_scales;
+    rp.src_codes = sdc; rp.src_scales = sds; rp.dst = h->dn_tiles_buf;
     rp.K = I; rp.N = H; rp.TW = h->dn_TW; rp.gate_up = 0;
     fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
     FE_CUDA_TRY(cudaGetLastError());
@@ -340,20 +466,35 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     if ((reinterpret_cast<uintptr_t>(x_bf16) & 3u) || (reinterpret_cast<uintptr_t>(y_bf16) & 3u) ||
         (reinterpret_cast<uintptr_t>(router_logits) & 3u))
         return FE_ERR_INVALID_ARG;
-    if (h->path == 2) return FE_ERR_UNSUPPORTED;
+    if (h->path == FE_PATH_TCGEN05) return FE_ERR_UNSUPPORTED;
     DeviceGuard g(h->device);
     if (!g.ok) return FE_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     const int P = T * top_k;
+
+    if (h->path == FE_PATH_AUTO || h->path == FE_PATH_FUSED_DECODE) {
+        const size_t wbytes = decode_weight_bytes(h, T, top_k);
+        if (wbytes > 0 && decode_smem_total(h, wbytes, T, top_k) <= (size_t)h->smem_optin) {
+            fe_status st = decode_path(h, x_bf16, router_logits, T, top_k, y_bf16, wbytes, s);
+            if (st == FE_OK) {
+                h->last_T = T;
+                h->last_k = top_k;
+                h->last_path = FE_PATH_FUSED_DECODE;
+                h->last_kernels = 1;
+            }
+            return st;
+        }
+        if (h->path == FE_PATH_FUSED_DECODE) return FE_ERR_UNSUPPORTED;
+    }
 
     fe::RouteParams rp{};
     rp.logits = router_logits; rp.T = T; rp.E = h->E; rp.k = top_k;
     rp.idx = h->idx; rp.w = h->w; rp.counts = h->counts; rp.offsets = h->offsets;
     rp.sorted_pair = h->sorted_pair; rp.pair_row = h->pair_row; rp.active = h->active;
     rp.n_active = h->n_active; rp.max_count = h->max_count; rp.status = h->status;
-    const int rthreads = std::min(1024, std::max(32, roundup32(std::max(P, 32 * std::min(T, 32)))));
+    const int rthreads = std::min(fe::kRouteMaxThreads, std::max(32, roundup32(std::max(P, 32 * T))));
     fe::route_group_kernel<<<1, rthreads, fe::route_smem_bytes(h->E, rthreads), s>>>(rp);
-    if (cudaGetLastError() != cudaSuccess) return FE_ERR_CUDA;
+    FE_CUDA_TRY(cudaGetLastError());
 
     fe_status st = gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
     if (st != FE_OK) return st;
@@ -361,9 +502,11 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     dim3 cgrid((h->H / 2 + 255) / 256, T);
     fe::combine_kernel<<<cgrid, 256, 0, s>>>(h->o, h->w, h->pair_row, h->H, top_k,
                                               static_cast<__nv_bfloat16*>(y_bf16));
-    if (cudaGetLastError() != cudaSuccess) return FE_ERR_CUDA;
+    FE_CUDA_TRY(cudaGetLastError());
     h->last_T = T;
     h->last_k = top_k;
+    h->last_path = FE_PATH_GEMV;
+    h->last_kernels = 4;
     return FE_OK;
 }
 
@@ -421,8 +564,23 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits)
 
 fe_status fe_moe_set_path(fe_moe_t h, int path)
 {
-    if (!h || path < 0 || path > 2) return FE_ERR_INVALID_ARG;
+    if (!h || path < FE_PATH_AUTO || path > FE_PATH_FUSED_DECODE) return FE_ERR_INVALID_ARG;
     h->path = path;
+    return FE_OK;
+}
+
+fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    h->trace = device_buf;
+    return FE_OK;
+}
+
+fe_status fe_moe_last_forward_info(fe_moe_t h, int* path, int* kernels)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    if (path) *path = h->last_path;
+    if (kernels) *kernels = h->last_kernels;
     return FE_OK;
 }
 
@@ -433,7 +591,7 @@ void fe_moe_destroy(fe_moe_t h)
         DeviceGuard g(h->device);
         cudaDeviceSynchronize();
         free_workspace(h);
-        void* ptrs[] = {h->gu_codes, h->gu_scales, h->dn_codes, h->dn_scales};
+        void* ptrs[] = {h->gu_tiles_buf, h->dn_tiles_buf};
         for (void* p : ptrs)
             if (p) cudaFree(p);
     }
@@ -441,6 +599,8 @@ void fe_moe_destroy(fe_moe_t h)
 }
 
 size_t fe_moe_device_bytes(fe_moe_t h) { return h ? h->weight_bytes + h->work_bytes : 0; }
+
+const char* fe_moe_last_error(void) { return g_last_error; }
 
 fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales)
 {

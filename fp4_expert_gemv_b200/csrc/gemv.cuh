@@ -11,9 +11,13 @@
 //
 // Weight layout inside the library (re-laid out at load time from the
 // [E][K/2][N] byte / [E][K/32][N] scale format): every expert matrix is cut
-// into column tiles of TW columns; a tile is one contiguous block of K/2 rows
-// of TW bytes (row r holds k = 2r in the low nibbles, k = 2r + 1 in the high
-// nibbles), followed in a separate buffer by its K/32 rows of TW bf16 scales.
+// into column tiles of TW columns; a tile is one contiguous block of K/2 byte
+// rows of TW bytes, byte row r holding k = 2r in the low nibbles and k = 2r+1
+// in the high nibbles, stored group-interleaved: [16][K/32][TW], entry
+// (i, g) = byte row 16g + i.  A thread owning group g reads its 16 rows with a
+// stride of (K/32) * TW bytes, and neighbouring threads (neighbouring groups)
+// read neighbouring 16-byte vectors.  The K/32 rows of TW bf16 scales of the
+// tile follow its codes, so one tile is one contiguous block.
 // For gate_up a tile holds TN gate columns then the TN matching up columns,
 // so the SwiGLU epilogue of a tile needs nothing from another tile.
 //
@@ -31,8 +35,7 @@
 namespace fe {
 
 struct GemvParams {
-    const uint8_t* codes;     // tiles [E][n_tiles][K/2][TW]
-    const uint16_t* scales;   // tiles [E][n_tiles][K/32][TW] (bf16 bits)
+    const uint8_t* tiles;     // [E][n_tiles] x {codes [16][K/32][TW], scales bf16 [K/32][TW]}
     int K;                    // reduction length
     int TW;                   // tile width in columns (bytes per row)
     int n_tiles;              // tiles per expert
@@ -140,13 +143,13 @@ __global__ void __launch_bounds__(256) gemv_kernel(GemvParams p)
 
     // this thread's weights: 16 rows x 16 bytes and 16 scales
     const size_t tile_id = (size_t)e * p.n_tiles + tile;
-    const uint8_t* wt = p.codes + tile_id * (size_t)(K / 2) * TW;
-    const uint16_t* st = p.scales + tile_id * (size_t)G * TW;
+    const uint8_t* wt = p.tiles + tile_id * ((size_t)(K / 2) * TW + (size_t)G * TW * 2);
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(wt + (size_t)(K / 2) * TW);
     uint4 q[16];
     float sc[16];
     if (valid) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = ldg_stream(wt + (size_t)(16 * g + i) * TW + 16 * c);
+        for (int i = 0; i < 16; ++i) q[i] = ldg_stream(wt + ((size_t)i * G + g) * TW + 16 * c);
         const uint4 s0 = *reinterpret_cast<const uint4*>(st + (size_t)g * TW + 16 * c);
         const uint4 s1 = *reinterpret_cast<const uint4*>(st + (size_t)g * TW + 16 * c + 8);
         const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};

@@ -62,15 +62,18 @@ __global__ void pack_kernel(const float* __restrict__ W, int64_t E, int64_t K, i
 
 // Re-layout of one matrix family into column tiles (see gemv.cuh):
 //   src codes  [E][K/2][N], src scales [E][K/32][N]
-//   dst codes  [E][n_tiles][K/2][TW], dst scales [E][n_tiles][K/32][TW]
+//   dst        [E][n_tiles] tiles of tile_bytes = (K/2)*TW + (K/32)*TW*2:
+//              codes [16][K/32][TW] -- entry (i, g, j) is source byte row
+//              16*g + i (k = 32g + 2i, 32g + 2i + 1) of tile column j, so the
+//              16 rows of one 32-k group are (K/32) * TW bytes apart and
+//              consecutive groups are adjacent -- then the scales [K/32][TW]
 // Tile column j maps to source column col(tile, j): for the fused gate_up
 // matrix (TN = TW/2, I = N/2) j < TN -> tile*TN + j (gate), j >= TN ->
 // I + tile*TN + j - TN (up); otherwise tile*TW + j.
 struct RelayoutParams {
     const uint8_t* src_codes;
     const uint16_t* src_scales;
-    uint8_t* dst_codes;
-    uint16_t* dst_scales;
+    uint8_t* dst;
     int64_t E, K, N;
     int TW;
     int gate_up;
@@ -90,6 +93,7 @@ __global__ void relayout_kernel(RelayoutParams p)
 {
     const int64_t n_tiles = p.N / p.TW;
     const int64_t rows = p.K / 2, G = p.K / 32;
+    const int64_t tile_bytes = rows * p.TW + G * p.TW * 2;
     const int64_t cchunks = p.E * n_tiles * rows * (p.TW / 16);
     const int64_t schunks = p.E * n_tiles * G * (p.TW / 8);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -97,12 +101,14 @@ __global__ void relayout_kernel(RelayoutParams p)
         if (i < cchunks) {
             const int64_t jc = i % (p.TW / 16);
             int64_t rest = i / (p.TW / 16);
-            const int64_t r = rest % rows;
+            const int64_t dr = rest % rows;           // destination row = ii * G + g
             rest /= rows;
             const int64_t tile = rest % n_tiles, e = rest / n_tiles;
+            const int64_t ii = dr / G, g = dr % G;
+            const int64_t r = 16 * g + ii;            // source byte row
             const int64_t col = relayout_src_col(p, tile, 16 * jc);   // 16 consecutive source columns
             const uint4 v = *reinterpret_cast<const uint4*>(p.src_codes + (e * rows + r) * p.N + col);
-            *reinterpret_cast<uint4*>(p.dst_codes + ((e * n_tiles + tile) * rows + r) * p.TW + 16 * jc) = v;
+            *reinterpret_cast<uint4*>(p.dst + (e * n_tiles + tile) * tile_bytes + dr * p.TW + 16 * jc) = v;
         } else {
             const int64_t i2 = i - cchunks;
             const int64_t jc = i2 % (p.TW / 8);
@@ -112,7 +118,7 @@ __global__ void relayout_kernel(RelayoutParams p)
             const int64_t tile = rest % n_tiles, e = rest / n_tiles;
             const int64_t col = relayout_src_col(p, tile, 8 * jc);
             const uint4 v = *reinterpret_cast<const uint4*>(p.src_scales + (e * G + g) * p.N + col);
-            *reinterpret_cast<uint4*>(p.dst_scales + ((e * n_tiles + tile) * G + g) * p.TW + 8 * jc) = v;
+            *reinterpret_cast<uint4*>(p.dst + (e * n_tiles + tile) * tile_bytes + rows * p.TW + (g * p.TW + 8 * jc) * 2) = v;
         }
     }
 }

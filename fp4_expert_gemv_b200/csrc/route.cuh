@@ -36,8 +36,10 @@ FE_DEV bool route_better(float va, int ia, float vb, int ib)
 
 constexpr int kRouteMaxPerLane = 32;  // E <= 1024
 
+constexpr int kRouteMaxThreads = 512;
+
 // Dynamic shared memory: cnt[E] | cursor[E] | wcnt[nwarps][E]
-__global__ void route_group_kernel(RouteParams p)
+__global__ void __launch_bounds__(kRouteMaxThreads) route_group_kernel(RouteParams p)
 {
     extern __shared__ int32_t sm[];
     const int E = p.E, k = p.k, T = p.T;

@@ -118,10 +118,26 @@ fe_status fe_moe_get_routing(fe_moe_t h, int32_t* idx, float* w, int32_t* offset
  * otherwise; clears the flags. */
 fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
 
-/* Force a compute path for the gate_up / down projections: 0 = automatic
- * (by tokens per expert), 1 = the CUDA-core GEMV kernels, 2 = the tcgen05
- * tensor-core grouped GEMM.  For tests and measurements. */
+/* Compute paths of fe_moe_forward. */
+#define FE_PATH_AUTO 0          /* chosen per call from T, top_k and the shape */
+#define FE_PATH_GEMV 1          /* route kernel + grouped GEMV gate_up + GEMV down + combine (any T) */
+#define FE_PATH_TCGEN05 2       /* tcgen05 tensor-core grouped GEMM (large T) */
+#define FE_PATH_FUSED_DECODE 3  /* one cooperative kernel for the whole layer (T * top_k <= 16) */
+
+/* Force a compute path (FE_PATH_*); FE_ERR_UNSUPPORTED from forward if the
+ * forced path cannot run the call.  For tests and measurements. */
 fe_status fe_moe_set_path(fe_moe_t h, int path);
+
+/* Which path the last successful forward took and how many kernels it
+ * enqueued. */
+fe_status fe_moe_last_forward_info(fe_moe_t h, int* path, int* kernels);
+
+/* Diagnostics: when device_buf (device memory, [number of SMs][16] uint64)
+ * is set, the fused decode kernel writes %globaltimer stamps of its phases
+ * there (0 start, 8 logits loaded, 9 routed, 10 routing shared, 11 work split,
+ * 12 barriers initialised, 1 loads issued, 2 x staged, 3 gate_up done, 4 act
+ * read back, 5 down done, 6 end).  NULL switches it off. */
+fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf);
 
 /* Human-readable text of a status code (static storage). */
 const char* fe_moe_status_string(fe_status s);
@@ -142,6 +158,10 @@ fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint
  * bytes identical to fe_moe_pack_host. */
 fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,
                              fe_stream_t stream);
+
+/* Text of the last CUDA failure behind an FE_ERR_CUDA / FE_ERR_OOM returned to
+ * this thread ("" if none); static thread-local storage. */
+const char* fe_moe_last_error(void);
 
 /* Bytes of device memory the handle holds (weights + workspace). */
 size_t fe_moe_device_bytes(fe_moe_t h);

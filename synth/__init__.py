@@ -171,7 +171,7 @@ def _device_lib():
         import os
         path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfe_synth.so")
         if not os.path.exists(path):
-            raise ImportError(f"{path} is not built; run `python -m fp4_expert_gemv_b200.build`")
+            raise ImportError(f"{path} is not built; run `python fp4_expert_gemv_b200/build.py`")
         lib = ctypes.CDLL(path)
         P, u64, i64 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64
         lib.fe_synth_gate_up.argtypes = [P, u64, i64, i64, i64, P]

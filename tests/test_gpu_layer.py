@@ -85,10 +85,11 @@ def test_pack_device_matches_oracle(torch_cuda):
         assert np.array_equal(c.cpu().numpy(), c_ref)
 
 
-def test_tiny_layer_host_packed(torch_cuda):
+@pytest.mark.parametrize("path", ["auto", "gemv"])
+def test_tiny_layer_host_packed(torch_cuda, path):
     cfg, seed, x, lg = harness.workload_inputs("tiny")
     E, H, I, k = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"]
-    gl = harness.GpuLayer(E, H, I, seed, max_T=64, max_k=8, source="host")
+    gl = harness.GpuLayer(E, H, I, seed, max_T=64, max_k=8, source="host", path=PATHS[path])
     osd = harness.OracleSide(E, H, I, seed)
     run_and_check(gl, osd, x, lg, k, what="tiny")
     # a second batch of other sizes through the same handle: ragged token counts
@@ -111,13 +112,21 @@ def test_tiny_layer_device_packed_equals_host_packed(torch_cuda):
     assert np.array_equal(ya, yb)
 
 
+PATHS = {"auto": 0, "gemv": 1}
+
+
+@pytest.mark.parametrize("path", ["auto", "gemv"])
 @pytest.mark.parametrize("seed", [1, 2, 3])
-def test_decode_e128_t1(torch_cuda, seed):
+def test_decode_e128_t1(torch_cuda, seed, path):
     cfg, seed, x, lg = harness.workload_inputs("decode_e128_t1", seed=seed)
     E, H, I, k = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"]
-    gl = harness.GpuLayer(E, H, I, seed, max_T=64, max_k=16, source="device", keep_packed=True)
+    gl = harness.GpuLayer(E, H, I, seed, max_T=64, max_k=16, source="device", keep_packed=True,
+                          path=PATHS[path])
     osd = harness.OracleSide(E, H, I, seed)
-    run_and_check(gl, osd, x, lg, k, what=f"decode_e128_t1 seed {seed}")
+    run_and_check(gl, osd, x, lg, k, what=f"decode_e128_t1 seed {seed} path {path}")
+    import fp4_expert_gemv_b200 as fe
+    taken, kernels = gl.layer.last_forward_info()
+    assert taken == (fe.PATH_FUSED_DECODE if path == "auto" else fe.PATH_GEMV), taken
     # the device-generated, device-packed bytes of the touched experts equal the oracle's
     idx, _ = oracle.default().route(lg, k)
     for e in np.unique(idx)[:3]:
@@ -150,7 +159,10 @@ def test_decode_e512(torch_cuda, seed, T):
     E, H, I, k = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"]
     gl = _cached_layer(E, H, I, seed)
     osd = _cached_oracle(E, H, I, seed)
-    run_and_check(gl, osd, x, lg, k, what=f"e512 seed {seed} T={T}")
+    for path in ("auto", "gemv"):
+        gl.layer.set_path(PATHS[path])
+        run_and_check(gl, osd, x, lg, k, what=f"e512 seed {seed} T={T} path {path}")
+    gl.layer.set_path(0)
 
 
 _LAYERS, _ORACLES = {}, {}
@@ -180,11 +192,12 @@ def test_prefill_t4096_sampled(torch_cuda):
     _LAYERS.clear()
 
 
-def test_edge_cases(torch_cuda):
+@pytest.mark.parametrize("path", ["auto", "gemv"])
+def test_edge_cases(torch_cuda, path):
     torch = torch_cuda
     import fp4_expert_gemv_b200 as fe
     E, H, I, seed = 8, 256, 128, 0
-    gl = harness.GpuLayer(E, H, I, seed, max_T=40, max_k=8, source="host")
+    gl = harness.GpuLayer(E, H, I, seed, max_T=40, max_k=8, source="host", path=PATHS[path])
     osd = harness.OracleSide(E, H, I, seed)
     x = synth.activations_bf16(50, 40, H)
     # k = 1 and k = E
@@ -240,12 +253,17 @@ def test_deterministic(torch_cuda):
     a = gl.forward(x, lg, k)[0]
     b = gl.forward(x, lg, k)[0]
     assert np.array_equal(a, b)
+    # the fused single-token kernel too (its combine is ordered, no atomics)
+    a1 = gl.forward(x[:1], lg[:1], k)[0]
+    for _ in range(3):
+        assert np.array_equal(gl.forward(x[:1], lg[:1], k)[0], a1)
 
 
-def test_graph_replay_with_changing_inputs(torch_cuda):
+@pytest.mark.parametrize("path", ["auto", "gemv"])
+def test_graph_replay_with_changing_inputs(torch_cuda, path):
     torch = torch_cuda
     E, H, I, seed, T, k = 8, 256, 128, 0, 4, 2
-    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=k, source="host")
+    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=k, source="host", path=PATHS[path])
     osd = harness.OracleSide(E, H, I, seed)
     xs = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
     ls = torch.empty((T, E), dtype=torch.float32, device="cuda")
@@ -306,7 +324,10 @@ def test_argument_errors(torch_cuda):
         assert fe.fe_moe_forward(h, None, 16, 1, 2, 32, None) == fe.FE_ERR_INVALID_ARG
         assert fe.fe_moe_forward(h, 16, 16, 1, 2, 16, None) == fe.FE_ERR_INVALID_ARG   # y aliases x
         assert fe.fe_moe_forward(h, 16, 16, -1, 2, 32, None) == fe.FE_ERR_INVALID_ARG
-        assert fe.fe_moe_set_path(h, 3) == fe.FE_ERR_INVALID_ARG
+        assert fe.fe_moe_set_path(h, 4) == fe.FE_ERR_INVALID_ARG
+        assert fe.fe_moe_set_path(h, fe.PATH_TCGEN05) == fe.FE_OK
+        assert fe.fe_moe_forward(h, 16, 16, 1, 2, 32, None) == fe.FE_ERR_UNSUPPORTED
+        assert fe.fe_moe_set_path(h, fe.PATH_AUTO) == fe.FE_OK
         st, = [fe.fe_moe_get_status(h, None)]
         assert st == fe.FE_OK
     finally:
