@@ -143,11 +143,13 @@ cudaError_t launch_gemv(const fe::GemvParams& p, int grid, int threads, cudaStre
     return cudaGetLastError();
 }
 
+// Function attributes are process-wide, so every kernel is opted into the
+// device's largest dynamic shared memory once: a handle of another shape must
+// never lower the limit below what this handle's launches request.
 template <int NT, bool GU>
-cudaError_t allow_gemv_smem(int K, int TW)
+cudaError_t allow_gemv_smem(int optin)
 {
-    const size_t smem = fe::gemv_smem_bytes<NT>(K, TW, roundup32((TW / 16) * (K / 32)));
-    return cudaFuncSetAttribute(fe::gemv_kernel<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    return cudaFuncSetAttribute(fe::gemv_kernel<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
 }
 
 using DecodeFn = void (*)(fe::DecodeParams);
@@ -247,18 +249,18 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     return FE_OK;
 }
 
-// Opt the kernels into the dynamic shared memory this layer shape needs
-// (once, outside any stream capture).
+// Opt the kernels into the device's largest dynamic shared memory (once,
+// outside any stream capture).
 cudaError_t configure_kernels(const fe_moe_s* h)
 {
-    cudaError_t e = cudaFuncSetAttribute(fe::route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)fe::route_smem_bytes(h->E, fe::kRouteMaxThreads));
-    if (e == cudaSuccess) e = allow_gemv_smem<1, true>(h->H, h->gu_TW);
-    if (e == cudaSuccess) e = allow_gemv_smem<4, true>(h->H, h->gu_TW);
-    if (e == cudaSuccess) e = allow_gemv_smem<1, false>(h->I, h->dn_TW);
-    if (e == cudaSuccess) e = allow_gemv_smem<4, false>(h->I, h->dn_TW);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel_for(h->gu_TW / 16),
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_optin);
+    const int optin = h->smem_optin;
+    cudaError_t e = cudaFuncSetAttribute(fe::route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess) e = allow_gemv_smem<1, true>(optin);
+    if (e == cudaSuccess) e = allow_gemv_smem<4, true>(optin);
+    if (e == cudaSuccess) e = allow_gemv_smem<1, false>(optin);
+    if (e == cudaSuccess) e = allow_gemv_smem<4, false>(optin);
+    for (int C = 2; C <= 32 && e == cudaSuccess; C *= 2)
+        e = cudaFuncSetAttribute(decode_kernel_for(C), cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     return e;
 }
 
@@ -618,5 +620,6 @@ fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, ui
     fe::pack_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(W, E, K, N, codes, scales);
     return cudaGetLastError() == cudaSuccess ? FE_OK : FE_ERR_CUDA;
 }
+
 
 }  // extern "C"
