@@ -56,6 +56,7 @@ _SIGS = {
     "fe_moe_pack_device": (_st, [_P, _i64, _i64, _i64, _P, _P, _P]),
     "fe_moe_device_bytes": (ctypes.c_size_t, [_P]),
     "fe_moe_last_error": (ctypes.c_char_p, []),
+    "fe_moe_forward_noalloc": (_st, [_i32, _i32, _i32, _P, _P, _P, _P, _P, _P, _i32, _i32, _P, _P]),
 }
 
 for _name, (_res, _args) in _SIGS.items():

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -13,6 +14,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "gemv.cuh"
+#include "gemv_canonical.cuh"
 #include "pack.cuh"
 #include "route.cuh"
 
@@ -621,5 +623,171 @@ fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, ui
     return cudaGetLastError() == cudaSuccess ? FE_OK : FE_ERR_CUDA;
 }
 
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward (fe_moe_forward_noalloc).
+//
+// For callers that may not allocate device memory at all -- no cudaMalloc,
+// no stream-ordered pool, no library that allocates on their behalf -- for
+// instance code that runs under an external memory manager that owns every
+// device byte, or inside a region where an allocation could stall or fail.
+// Such a caller passes the packed weights, x, the logits and y in its own
+// buffers; the routing lists, act and the per-pair down outputs live in one
+// file-scope device array instead of a reserved workspace.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+    bool ready = false;
+    unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+};
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[64];
+
+// Once per device, with that device current: the device address of the
+// scratch array (its name in host code is only a stand-in) and the kernels'
+// shared-memory opt-in.  Neither allocates.
+fe_status noalloc_setup(int dev, unsigned char** scratch)
+{
+    if (dev < 0 || dev >= 64) return FE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoAllocDevice& d = g_noalloc_dev[dev];
+    if (!d.ready) {
+        void* ptr = nullptr;
+        FE_CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+        int optin = 0;
+        FE_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        FE_CUDA_TRY(cudaFuncSetAttribute(fe::route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin));
+        FE_CUDA_TRY(cudaFuncSetAttribute(fe::gemv_canonical_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin));
+        FE_CUDA_TRY(cudaFuncSetAttribute(fe::gemv_canonical_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin));
+        FE_CUDA_TRY(cudaFuncSetAttribute(fe::gemv_canonical_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin));
+        FE_CUDA_TRY(cudaFuncSetAttribute(fe::gemv_canonical_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin));
+        d.scratch = static_cast<unsigned char*>(ptr);
+        d.ready = true;
+    }
+    *scratch = d.scratch;
+    return FE_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Carve the scratch array; returns the bytes needed (0 = does not fit).
+struct NoAllocLayout {
+    size_t status, idx, w, sorted_pair, pair_row, counts, offsets, active, n_active, max_count, act, o, total;
+};
+
+NoAllocLayout noalloc_layout(int E, int H, int I, int T, int k)
+{
+    NoAllocLayout L;
+    const size_t P = (size_t)T * k;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off = align256(off + bytes); return at; };
+    L.status = take(4);
+    L.idx = take(4 * P);
+    L.w = take(4 * P);
+    L.sorted_pair = take(4 * P);
+    L.pair_row = take(4 * P);
+    L.counts = take(4 * (size_t)E);
+    L.offsets = take(4 * ((size_t)E + 1));
+    L.active = take(4 * (size_t)E);
+    L.n_active = take(4);
+    L.max_count = take(4);
+    L.act = take(4 * P * I);
+    L.o = take(4 * P * H);
+    L.total = off;
+    return L;
+}
+
+template <int NT, bool GU>
+cudaError_t launch_canonical(const fe::CanonParams& p, int grid, int threads, cudaStream_t s)
+{
+    const size_t smem = fe::gemv_smem_bytes<NT>(p.K, p.TW, threads);
+    fe::gemv_canonical_kernel<NT, GU><<<grid, threads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+fe_status fe_moe_forward_noalloc(int E, int H, int I, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
+                                 const uint8_t* down_codes, const uint16_t* down_scales, const void* x_bf16,
+                                 const float* router_logits, int T, int top_k, void* y_bf16, fe_stream_t stream)
+{
+    if (E < 1 || E > 1024 || H <= 0 || I <= 0 || H % 32 || I % 32 || T < 0 || top_k < 1 || top_k > E)
+        return FE_ERR_INVALID_ARG;
+    if (T == 0) return FE_OK;
+    if (!gate_up_codes || !gate_up_scales || !down_codes || !down_scales || !x_bf16 || !router_logits || !y_bf16 ||
+        x_bf16 == y_bf16)
+        return FE_ERR_INVALID_ARG;
+    if (!aligned16(gate_up_codes) || !aligned16(gate_up_scales) || !aligned16(down_codes) || !aligned16(down_scales) ||
+        (reinterpret_cast<uintptr_t>(x_bf16) & 3u) || (reinterpret_cast<uintptr_t>(y_bf16) & 3u) ||
+        (reinterpret_cast<uintptr_t>(router_logits) & 3u))
+        return FE_ERR_INVALID_ARG;
+    const int gu_TW = pick_tile_width(H, I, true);
+    const int dn_TW = pick_tile_width(I, H, false);
+    if (gu_TW == 0 || dn_TW == 0) return FE_ERR_UNSUPPORTED;
+    const NoAllocLayout L = noalloc_layout(E, H, I, T, top_k);
+    if (L.total > kNoAllocScratchBytes) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "fe_moe_forward_noalloc: T*top_k = %d pairs need %zu bytes of scratch, above the %zu-byte static "
+                 "array (pairs * (I + H) * 4 bytes must stay below it)",
+                 T * top_k, L.total, kNoAllocScratchBytes);
+        return FE_ERR_CAPACITY;
+    }
+    int dev = 0;
+    FE_CUDA_TRY(cudaGetDevice(&dev));
+    unsigned char* scr = nullptr;
+    const fe_status st0 = noalloc_setup(dev, &scr);
+    if (st0 != FE_OK) return st0;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int P = T * top_k;
+
+    fe::RouteParams rp{};
+    rp.logits = router_logits; rp.T = T; rp.E = E; rp.k = top_k;
+    rp.idx = reinterpret_cast<int32_t*>(scr + L.idx);
+    rp.w = reinterpret_cast<float*>(scr + L.w);
+    rp.counts = reinterpret_cast<int32_t*>(scr + L.counts);
+    rp.offsets = reinterpret_cast<int32_t*>(scr + L.offsets);
+    rp.sorted_pair = reinterpret_cast<int32_t*>(scr + L.sorted_pair);
+    rp.pair_row = reinterpret_cast<int32_t*>(scr + L.pair_row);
+    rp.active = reinterpret_cast<int32_t*>(scr + L.active);
+    rp.n_active = reinterpret_cast<int32_t*>(scr + L.n_active);
+    rp.max_count = reinterpret_cast<int32_t*>(scr + L.max_count);
+    rp.status = reinterpret_cast<uint32_t*>(scr + L.status);
+    const int rthreads = std::min(fe::kRouteMaxThreads, std::max(32, roundup32(std::max(P, 32 * T))));
+    fe::route_group_kernel<<<1, rthreads, fe::route_smem_bytes(E, rthreads), s>>>(rp);
+    FE_CUDA_TRY(cudaGetLastError());
+
+    const int max_active = std::min(E, P);
+    fe::CanonParams cp{};
+    cp.offsets = rp.offsets; cp.active = rp.active; cp.n_active = rp.n_active; cp.sorted_pair = rp.sorted_pair;
+    cp.top_k = top_k;
+    cp.codes = gate_up_codes; cp.scales = gate_up_scales; cp.K = H; cp.N = 2 * I; cp.TW = gu_TW;
+    cp.n_tiles = I / (gu_TW / 2); cp.N_out = I; cp.x = static_cast<const uint16_t*>(x_bf16); cp.act_in = nullptr;
+    cp.out = reinterpret_cast<float*>(scr + L.act);
+    int threads = roundup32((gu_TW / 16) * (H / 32));
+    cudaError_t e = (T == 1) ? launch_canonical<1, true>(cp, max_active * cp.n_tiles, threads, s)
+                             : launch_canonical<4, true>(cp, max_active * cp.n_tiles, threads, s);
+    if (e != cudaSuccess) return record_cuda(e, "noalloc gate_up launch");
+    cp.codes = down_codes; cp.scales = down_scales; cp.K = I; cp.N = H; cp.TW = dn_TW; cp.n_tiles = H / dn_TW;
+    cp.N_out = H; cp.x = nullptr; cp.act_in = reinterpret_cast<const float*>(scr + L.act);
+    cp.out = reinterpret_cast<float*>(scr + L.o);
+    threads = roundup32((dn_TW / 16) * (I / 32));
+    e = (T == 1) ? launch_canonical<1, false>(cp, max_active * cp.n_tiles, threads, s)
+                 : launch_canonical<4, false>(cp, max_active * cp.n_tiles, threads, s);
+    if (e != cudaSuccess) return record_cuda(e, "noalloc down launch");
+
+    dim3 cgrid((H / 2 + 255) / 256, T);
+    fe::combine_kernel<<<cgrid, 256, 0, s>>>(reinterpret_cast<const float*>(scr + L.o), rp.w, rp.pair_row, H, top_k,
+                                              static_cast<__nv_bfloat16*>(y_bf16));
+    FE_CUDA_TRY(cudaGetLastError());
+    return FE_OK;
+}
 
 }  // extern "C"

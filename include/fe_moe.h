@@ -159,6 +159,30 @@ fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint
 fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,
                              fe_stream_t stream);
 
+/* Allocation-free forward.  No counterpart on the source pages: an addition for
+ * callers that must not allocate device memory -- for instance code running
+ * under an external memory manager that owns every device byte, or code that
+ * may not call cudaMalloc, a stream-ordered pool or any allocating library
+ * routine at the point where it runs the layer.  It needs no handle and no
+ * workspace: the caller passes the packed weights in the format of
+ * fe_moe_load_packed (device memory, 16-byte aligned, read in place), x, the
+ * logits and y; the routing lists and intermediate activations live in one
+ * static device array of 4 MiB that every GPU which loads the library holds
+ * until the process exits.  Calls whose T * top_k * (I + H) * 4 bytes plus a
+ * few KiB of routing lists exceed that array return FE_ERR_CAPACITY with the
+ * reason in fe_moe_last_error(); nothing is enqueued then.  The first call on
+ * each device, with that device current, looks up the array's device address
+ * and sets kernel attributes (neither allocates); make that first call before
+ * any stream capture.  Every call shares the array and leaves its contents
+ * behind; each call writes every scratch word it reads, so nothing has to be
+ * cleared between calls, but calls whose kernels overlap on the GPU (other
+ * streams, other threads) race on the array and must be serialised by the
+ * caller.  Same sizes and layouts as fe_moe_create + fe_moe_forward; no
+ * allocation, no host synchronisation; argument errors as fe_moe_forward. */
+fe_status fe_moe_forward_noalloc(int E, int H, int I, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
+                                 const uint8_t* down_codes, const uint16_t* down_scales, const void* x_bf16,
+                                 const float* router_logits, int T, int top_k, void* y_bf16, fe_stream_t stream);
+
 /* Text of the last CUDA failure behind an FE_ERR_CUDA / FE_ERR_OOM returned to
  * this thread ("" if none); static thread-local storage. */
 const char* fe_moe_last_error(void);
