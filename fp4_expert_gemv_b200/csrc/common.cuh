@@ -77,6 +77,13 @@ FE_DEV float silu_mul(float g, float u)
     return g / (1.0f + expf(-g)) * u;
 }
 
+FE_DEV unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // ld.global.nc with L1 no-allocate: weights are streamed once per launch.
 FE_DEV uint4 ldg_stream(const void* p)
 {

@@ -3,42 +3,46 @@
 // "FireEcho Engine", sections "Speed Optimization History" (single-token
 // decode fast path, multi-expert kernel, packed contiguous expert buffer,
 // CUDA-graph decode) and "The Goliath Kernel: Why It's Fast" (expert IDs read
-// on the GPU, FP4 dequantised in registers, nothing dequantised written to
-// memory).  The pages' kernel runs one Triton launch per projection; here the
-// whole layer is one launch, so that the HBM stream of the down weights
-// overlaps the gate_up work and no launch boundary sits inside the layer:
+// on the GPU, FP4 dequantised in registers, tensor-core accumulation, nothing
+// dequantised written to memory).  The pages' kernel runs one Triton launch
+// per projection; here the whole layer is one launch, so that the HBM stream
+// of the down weights overlaps the gate_up work and no launch boundary sits
+// inside the layer:
 //
 //   1. one bulk copy brings the T router-logit rows and the T x rows into
 //      shared memory; every CTA routes the T tokens itself (the rank of each
 //      logit among the E logits of its token, counted by all threads in
 //      parallel: rank < k selects it as slot rank, ties to the lower index)
 //      and groups the T*k pairs by expert; CTA 0 also publishes the routing;
-//   2. from the routed experts every CTA looks up its contiguous range of
-//      units in a work-split table computed at reserve time: the gate_up units
-//      (expert, column tile) and the down units (16-column h-slice over all
-//      routed experts), cut into per-CTA ranges of equal bytes;
+//   2. from the number of distinct routed experts every CTA reads, in a
+//      table built at reserve time, its range of gate_up units (16 gate + 16
+//      up columns of one routed expert) and its range of down units (16
+//      output columns over all routed experts), balanced in bytes;
 //   3. one thread issues cp.async.bulk copies of ALL the CTA's weight bytes
 //      (both phases) into shared memory at once, one mbarrier per unit;
-//   4. gate_up units are reduced over K as soon as their bytes land, SwiGLU
-//      applied, act written to global memory (L2) as 64-bit words holding
-//      the fp32 value and the launch's epoch tag;
+//   4. gate_up units: mma.m16n8k16 with the tokens of the unit's expert as
+//      the N columns (mma.cuh), SiLU(gate)*up, act written to global memory
+//      (L2) as 64-bit words holding the fp32 value and the launch's epoch tag;
 //   5. each CTA that owns down units reads act back, polling (bounded) until
 //      every word carries this launch's tag -- the data is its own ready
 //      flag, so no grid-wide barrier round trip is needed;
-//   6. each CTA computes the 16 output columns of its h-slices for every
-//      pair from the down bytes already in shared memory and combines them in
-//      slot order: y is written once, without atomics.
+//   6. down units: one warp per routed expert, its pairs as the N columns;
+//      the 16 outputs of every pair are combined in slot order, so y is
+//      written once, without atomics.
 //
 // The kernel is launched with programmatic dependent launch: its CTAs load
 // only static data before griddepcontrol.wait, so the next layer's CTAs can
 // be resident and waiting while this layer finishes.
 #pragma once
 
+#include <vector>
+
 #include "common.cuh"
+#include "mma.cuh"
 
 namespace fe {
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecMaxPairs = 16;   // T * top_k handled by the fused kernel
 constexpr int kDecMaxItems = 48;   // weight units (mbarriers) per CTA
@@ -50,12 +54,9 @@ struct DecodeParams {
     const float* logits;      // [T][E]
     uint16_t* y;              // bf16 [T][H]
     int T, E, H, I, k;
-    const uint8_t* gu_tiles;  // [E][gu_ntiles] tiles of gu_tile_bytes
-    int gu_ntiles;
-    uint32_t gu_tile_bytes;
-    const uint8_t* dn_tiles;  // [E][H/16] tiles of dn_tile_bytes
-    uint32_t dn_tile_bytes;
-    const int32_t* plan_first;  // [kDecMaxPairs + 1][grid + 1] first unit of each CTA, per nd
+    const uint8_t* gu_blocks; // [E][I/16] gate_up units of 2 blocks (18H bytes)
+    const uint8_t* dn_blocks; // [E][H/16] down blocks (9I bytes)
+    const int32_t* plan;      // [kDecMaxPairs + 1][2][grid + 1]: first gate_up / down unit of each CTA, per nd
     int32_t* idx;
     float* w;
     int32_t* counts;
@@ -71,52 +72,38 @@ struct DecodeParams {
     unsigned long long* trace;  // optional [grid][16] %globaltimer stamps of the phases
 };
 
-// ---- work split (host: table construction; the kernel only reads the table) ----
-struct DecodePlan {
-    int64_t gu_bytes, dn_bytes, total;
-    int n_gu, n_dn, grid;
-};
-
-inline DecodePlan decode_plan(int nd, int H, uint32_t gu_tile_bytes, int gu_ntiles, uint32_t dn_tile_bytes, int grid)
+// ---- work split (host only: the kernel reads the table) ---------------------------
+// gate_up units: nd * I/16 of 18H bytes; down units: H/16 of nd * 9I bytes.
+// gate_up units are spread evenly over the CTAs; then each down unit goes to
+// the CTA with the fewest bytes so far (lowest index on ties).  Returns, for
+// c = 0..grid, the first gate_up and the first down unit of CTA c.
+inline void decode_split(int nd, int H, int I, int grid, std::vector<int>& gu_first, std::vector<int>& dn_first)
 {
-    DecodePlan p;
-    p.gu_bytes = gu_tile_bytes;
-    p.dn_bytes = (int64_t)nd * dn_tile_bytes;
-    p.n_gu = nd * gu_ntiles;
-    p.n_dn = H / 16;
-    p.total = p.n_gu * p.gu_bytes + p.n_dn * p.dn_bytes;
-    p.grid = grid;
-    return p;
-}
-
-inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
-// First unit of CTA c: units are laid end to end in byte order (gate_up units,
-// then down units) and CTA c takes those whose first byte falls in
-// [c * total / grid, (c + 1) * total / grid).
-inline int decode_first_unit(const DecodePlan& p, int c)
-{
-    const int64_t t0 = (int64_t)c * p.total;
-    const int64_t gu_end = (int64_t)p.n_gu * p.gu_bytes;
-    if (t0 <= gu_end * p.grid) {
-        const int64_t i = ceil_div64(t0, (int64_t)p.grid * p.gu_bytes);
-        return (int)(i < p.n_gu ? i : p.n_gu);
+    const int n_gu = nd * (I / 16), n_dn = H / 16;
+    const int64_t gu_bytes = 18ll * H, dn_bytes = (int64_t)nd * 9 * I;
+    std::vector<int> cgu(grid), cdn(grid, 0);
+    std::vector<int64_t> load(grid);
+    for (int c = 0; c < grid; ++c) {
+        cgu[c] = (int)((int64_t)(c + 1) * n_gu / grid - (int64_t)c * n_gu / grid);
+        load[c] = cgu[c] * gu_bytes;
     }
-    const int64_t j = ceil_div64(t0 - gu_end * p.grid, (int64_t)p.grid * p.dn_bytes);
-    return p.n_gu + (int)(j < p.n_dn ? j : p.n_dn);
+    for (int j = 0; j < n_dn; ++j) {
+        int best = 0;
+        for (int c = 1; c < grid; ++c)
+            if (load[c] < load[best]) best = c;
+        cdn[best] += 1;
+        load[best] += dn_bytes;
+    }
+    gu_first.assign(grid + 1, 0);
+    dn_first.assign(grid + 1, 0);
+    for (int c = 0; c < grid; ++c) {
+        gu_first[c + 1] = gu_first[c] + cgu[c];
+        dn_first[c + 1] = dn_first[c] + cdn[c];
+    }
 }
-
-inline int64_t decode_unit_bytes(const DecodePlan& p, int u) { return u < p.n_gu ? p.gu_bytes : p.dn_bytes; }
 
 // ---- PTX wrappers --------------------------------------------------------------
 FE_DEV uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-FE_DEV unsigned long long globaltimer()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 
 FE_DEV void mbar_init(uint32_t bar, uint32_t count)
 {
@@ -145,10 +132,10 @@ FE_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity)
 FE_DEV bool mbar_wait0(uint32_t bar, unsigned long long timeout_ns)
 {
     if (mbar_try_wait(bar, 0)) return true;
-    const unsigned long long t0 = globaltimer();
+    const unsigned long long t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, 0)) return true;
-        if (globaltimer() - t0 > timeout_ns) return false;
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
 }
 
@@ -181,56 +168,6 @@ FE_DEV void ld_volatile_2u64(const unsigned long long* p, unsigned long long& a,
     asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
 
-// Reduce 16 per-lane values over the 32/C lanes that share lane % C
-// (butterfly reduce-scatter): afterwards this lane holds NOUT = max(1, 16C/32)
-// finished sums, for columns col0 .. col0 + NOUT - 1 of its chunk.
-template <int C>
-struct Butterfly {
-    static constexpr int L = 32 / C;
-    static constexpr int NOUT = (16 / L) > 0 ? (16 / L) : 1;
-};
-
-template <int C>
-FE_DEV int butterfly16(float (&v)[16], int lane)
-{
-    int col0 = 0;
-    int n = 16;
-#pragma unroll
-    for (int m = 16; m >= C; m >>= 1) {
-        if (n > 1) {
-            const int half = n >> 1;
-            const bool up = (lane & m) != 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (j < half) {
-                    const float send = up ? v[j] : v[j + half];
-                    const float keep = up ? v[j + half] : v[j];
-                    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
-            }
-            if (up) col0 += half;
-            n = half;
-        } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
-        }
-    }
-    return col0;
-}
-
-// Padded f16x2 row index: one spare word per 16 rows (bank spread).
-FE_DEV int padrow(int r) { return r + (r >> 4); }
-__host__ __device__ inline int padded_rows(int rows) { return rows + rows / 16 + 1; }
-
-// Power-of-two shift s >= 0 with m * 2^-s < 2^15 (m = max |v| of a row).
-FE_DEV int fp16_shift(float m)
-{
-    int s = 0;
-    if (m >= 32768.0f && m <= 3.0e38f) s = (int)((__float_as_uint(m) >> 23) & 0xff) - 127 - 14;
-    return s;
-}
-
-FE_DEV float pow2f(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
-
 FE_DEV float logit_key(float v) { return v != v ? -INFINITY : v; }
 
 struct DecodeShared {
@@ -240,92 +177,96 @@ struct DecodeShared {
     int pdi[kDecMaxPairs];        // pair -> distinct-expert index
     int dex[kDecMaxPairs];        // distinct experts, ascending
     int dstart[kDecMaxPairs + 1]; // first sorted position of each distinct expert
-    int pf0[kDecMaxPairs + 1];    // this CTA's first unit, per nd
-    int pf1[kDecMaxPairs + 1];    // the next CTA's first unit, per nd
+    int plan[kDecMaxPairs + 1][4];  // per nd: gate_up first/end, down first/end of this CTA
     int xshift[kDecMaxPairs];
     int ashift[kDecMaxPairs];
+    int item_d[kDecMaxPairs + 1];   // down items: (distinct expert, first sorted pair, pairs <= 8)
+    int item_r[kDecMaxPairs + 1];
+    int item_n[kDecMaxPairs + 1];
+    int n_items;
     int nd;
     int abort;
     unsigned tag;
     float wmax[kDecWarps];
+    int rank_part[kDecThreads];
     float ob[kDecMaxPairs * 16];  // down: [pair][16] outputs
 };
 
 // Byte offsets of the dynamic shared memory regions.
 struct DecodeSmem {
-    uint32_t mbar, shared, red, xs, as, lg, xr, total;
+    uint32_t mbar, shared, red, dred, xs, as, lg, xr, total;
 };
 
 __host__ __device__ inline uint32_t align16(uint32_t v) { return (v + 15u) & ~15u; }
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(uint32_t weight_bytes, int T, int k, int H, int I, int E, int TW)
+// xs: T x rows + 1 zero row; as: T*k act rows + 1 zero row (brow_words each).
+__host__ __device__ inline DecodeSmem decode_smem_layout(uint32_t weight_bytes, int T, int k, int H, int I, int E)
 {
     DecodeSmem L;
     L.mbar = weight_bytes;
     L.shared = L.mbar + 8 * (kDecMaxItems + 1);
     L.red = align16(L.shared + (uint32_t)sizeof(DecodeShared));
-    L.xs = L.red + 4u * kDecWarps * TW;
-    L.as = L.xs + 4u * T * padded_rows(H / 2);
-    L.lg = align16(L.as + 4u * T * k * padded_rows(I / 2));
+    L.dred = L.red;   // gate_up partials and down partials are never live together
+    L.xs = L.red + 4u * (kDecWarps * 32 * 8 > 8 * 4 * 32 * 4 ? kDecWarps * 32 * 8 : 8 * 4 * 32 * 4);
+    L.as = L.xs + 4u * (T + 1) * brow_words(H);
+    L.lg = align16(L.as + 4u * (T * k + 1) * brow_words(I));
     L.xr = align16(L.lg + 4u * T * E);
     L.total = align16(L.xr + 2u * T * H);
     return L;
 }
 
-template <int C>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
 {
     extern __shared__ __align__(128) uint8_t dsm[];
-    constexpr int TW = 16 * C;
-    constexpr int TN = TW / 2;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2;
     const int T = p.T, E = p.E, H = p.H, I = p.I, k = p.k, P = T * k;
-    const int G = H / 32, Gd = I / 32;
-    const DecodeSmem L = decode_smem_layout(p.weight_bytes, T, k, H, I, E, TW);
+    const DecodeSmem L = decode_smem_layout(p.weight_bytes, T, k, H, I, E);
+    const uint32_t gu_unit = 2u * block_bytes(H), dn_blk = block_bytes(I);
+    const int xrw = brow_words(H), arw = brow_words(I);
 
     uint8_t* wbuf = dsm;
     DecodeShared& S = *reinterpret_cast<DecodeShared*>(dsm + L.shared);
     float* red = reinterpret_cast<float*>(dsm + L.red);
+    float* dred = reinterpret_cast<float*>(dsm + L.dred);   // down partials [8 items][4 quarters][lane][4]
     uint32_t* xs = reinterpret_cast<uint32_t*>(dsm + L.xs);
     uint32_t* as = reinterpret_cast<uint32_t*>(dsm + L.as);
     float* lg = reinterpret_cast<float*>(dsm + L.lg);
     uint16_t* xr = reinterpret_cast<uint16_t*>(dsm + L.xr);
-    const int xrow = padded_rows(H / 2), arow = padded_rows(I / 2);
     const uint32_t mbar0 = smem_addr(dsm + L.mbar);
     const uint32_t in_bar = mbar0 + 8 * kDecMaxItems;
     const bool tracing = p.trace != nullptr;
     unsigned long long* trace = tracing ? p.trace + (size_t)blockIdx.x * 16 : nullptr;
-    if (tracing && tid == 0) trace[0] = globaltimer();
+    if (tracing && tid == 0) trace[0] = globaltimer_ns();
 
     // ---- 0. static data only, then wait for the previous grid ---------------------
-    if (tid <= kDecMaxPairs) {
-        S.pf0[tid] = p.plan_first[tid * (gridDim.x + 1) + blockIdx.x];
-        S.pf1[tid] = p.plan_first[tid * (gridDim.x + 1) + blockIdx.x + 1];
+    if (tid < 4 * (kDecMaxPairs + 1)) {
+        const int nd = tid >> 2, which = tid & 3;   // 0: gate_up first, 1: end, 2: down first, 3: end
+        const int32_t* row = p.plan + ((size_t)nd * 2 + (which >> 1)) * (gridDim.x + 1);
+        S.plan[nd][which] = row[blockIdx.x + (which & 1)];
     }
     if (tid == 0) {
-        mbar_init(in_bar, 1);
+        for (int u = 0; u <= kDecMaxItems; ++u) mbar_init(mbar0 + 8 * u, 1);   // the weight units' and in_bar
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         S.abort = 0;
     }
+    for (int i = tid; i < xrw; i += kDecThreads) xs[T * xrw + i] = 0u;       // zero B rows
+    for (int i = tid; i < arw; i += kDecThreads) as[P * arw + i] = 0u;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (tid == 0) {
-        // this launch's epoch tag; the last CTA to read it advances it
-        const unsigned e0 = ld_acquire_gpu(p.sync + 1);
-        const unsigned arrived = atomicAdd(p.sync, 1u);
-        const unsigned tag = (e0 + 1u) ? (e0 + 1u) : 1u;
-        S.tag = tag;
-        if (arrived == gridDim.x - 1) {
-            // every CTA has read the epoch: advance it for the next launch
-            atomicExch(p.sync, 0u);
-            st_release_gpu(p.sync + 1, tag);
-        }
-        if (p.bulk_inputs) {
-            const uint32_t lb = 4u * T * E, xb = 2u * T * H;
-            mbar_expect_tx(in_bar, lb + xb);
-            bulk_g2s(smem_addr(lg), p.logits, lb, in_bar);
-            bulk_g2s(smem_addr(xr), p.x, xb, in_bar);
-        }
+    if (tid == 0 && p.bulk_inputs) {
+        const uint32_t lb = 4u * T * E, xb = 2u * T * H;
+        mbar_expect_tx(in_bar, lb + xb);
+        bulk_g2s(smem_addr(lg), p.logits, lb, in_bar);
+        bulk_g2s(smem_addr(xr), p.x, xb, in_bar);
+    }
+    // this launch's epoch (the previous launch's update is visible after
+    // griddepcontrol.wait); both requests are in flight while the CTA routes and
+    // their results are consumed only when act is about to be written
+    unsigned ep_e0 = 0, ep_arrived = 0;
+    if (tid == kDecThreads - 1) {
+        ep_e0 = *reinterpret_cast<volatile unsigned*>(p.sync + 1);
+        ep_arrived = atomicAdd(p.sync, 1u);
     }
     if (!p.bulk_inputs) {
         for (int i = tid; i < T * E; i += kDecThreads) lg[i] = p.logits[i];
@@ -334,37 +275,60 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     __syncthreads();
     if (p.bulk_inputs && !mbar_wait0(in_bar, p.timeout_ns)) {
         if (tid == 0) atomicOr(p.status, kDevLoadTimeout);
-        return;   // the copies never completed: nothing can be in flight any more
+        return;
     }
-    if (tracing && tid == 0) trace[8] = globaltimer();
+    if (tracing && tid == 0) trace[8] = globaltimer_ns();
 
     // ---- 1. routing: rank of every logit among its token's E logits ------------------
+    // nsplit threads share the comparisons of one logit (E <= 128: 2 or more)
     bool nan_seen = false;
-    for (int t = 0; t < T; ++t) {
-        const float* row = lg + t * E;
-        for (int e = tid; e < E; e += kDecThreads) {
-            const float v = logit_key(row[e]);
-            nan_seen |= row[e] != row[e];
-            int rank = 0;
-            int e2 = 0;
-            if ((E & 3) == 0) for (; e2 + 4 <= E; e2 += 4) {
-                const float4 o = *reinterpret_cast<const float4*>(row + e2);
-                const float o0 = logit_key(o.x), o1 = logit_key(o.y), o2 = logit_key(o.z), o3 = logit_key(o.w);
-                rank += (o0 > v) || (o0 == v && e2 < e);
-                rank += (o1 > v) || (o1 == v && e2 + 1 < e);
-                rank += (o2 > v) || (o2 == v && e2 + 2 < e);
-                rank += (o3 > v) || (o3 == v && e2 + 3 < e);
-            }
-            for (; e2 < E; ++e2) {
-                const float o = logit_key(row[e2]);
-                rank += (o > v) || (o == v && e2 < e);
-            }
-            if (rank < k) {
-                S.sel_e[t * k + rank] = e;
-                S.sel_w[t * k + rank] = v;
+    {
+        const int epad = (E + 31) & ~31;
+        const int nsplit = epad >= kDecThreads ? 1 : kDecThreads / epad;
+        const int chunk = ((E + nsplit - 1) / nsplit + 3) & ~3;
+        int* rk = S.rank_part;
+        for (int t = 0; t < T; ++t) {
+            const float* row = lg + t * E;
+            for (int base = 0; base < E; base += kDecThreads / nsplit) {
+                const int e = base + tid % epad, part = tid / epad;
+                int rank = 0;
+                if (e < E && part < nsplit) {
+                    const float v = logit_key(row[e]);
+                    nan_seen |= row[e] != row[e];
+                    const int lo = part * chunk, hi = min(E, lo + chunk);
+                    int e2 = lo;
+                    if ((E & 3) == 0) {
+#pragma unroll 4
+                        for (; e2 + 4 <= hi; e2 += 4) {
+                            const float4 o = *reinterpret_cast<const float4*>(row + e2);
+                            const float o0 = logit_key(o.x), o1 = logit_key(o.y), o2 = logit_key(o.z), o3 = logit_key(o.w);
+                            rank += (o0 > v) || (o0 == v && e2 < e);
+                            rank += (o1 > v) || (o1 == v && e2 + 1 < e);
+                            rank += (o2 > v) || (o2 == v && e2 + 2 < e);
+                            rank += (o3 > v) || (o3 == v && e2 + 3 < e);
+                        }
+                    }
+                    for (; e2 < hi; ++e2) {
+                        const float o = logit_key(row[e2]);
+                        rank += (o > v) || (o == v && e2 < e);
+                    }
+                }
+                if (nsplit > 1) {
+                    rk[tid] = rank;
+                    __syncthreads();
+                    if (part == 0 && e < E) {
+                        for (int q = 1; q < nsplit; ++q) rank += rk[tid + q * epad];
+                    }
+                    __syncthreads();
+                }
+                if (part == 0 && e < E && rank < k) {
+                    S.sel_e[t * k + rank] = e;
+                    S.sel_w[t * k + rank] = logit_key(row[e]);
+                }
             }
         }
     }
+    if (tracing && tid == 0) trace[10] = globaltimer_ns();
     if (__syncthreads_or(nan_seen) && tid == 0 && blockIdx.x == 0) atomicOr(p.status, kDevNanLogit);
     for (int t = warp; t < T; t += kDecWarps) {
         const float l0 = S.sel_w[t * k];
@@ -382,29 +346,48 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     }
     __syncthreads();
 
+    if (tracing && tid == 0) trace[12] = globaltimer_ns();
     // ---- 2. grouping (warp 0): stable order by expert --------------------------
     if (warp == 0) {
-        const int ep = lane < P ? S.sel_e[lane] : 0x7fffffff;
-        int rank = 0;
-        for (int q = 0; q < P; ++q) {
-            const int eq = __shfl_sync(0xffffffffu, ep, q);
-            rank += (eq < ep) || (eq == ep && q < lane);
+        int ep = 0x7fffffff, rank = 0;
+        if (lane < P) {
+            ep = S.sel_e[lane];
+            for (int q = 0; q < P; ++q) {
+                const int eq = S.sel_e[q];
+                rank += (eq < ep) || (eq == ep && q < lane);
+            }
+            S.sp[rank] = lane;
         }
-        if (lane < P) S.sp[rank] = lane;
-        __syncwarp();
-        const int er = lane < P ? S.sel_e[S.sp[lane]] : -1;
-        const int eprev = __shfl_up_sync(0xffffffffu, er, 1);
-        const bool start = lane < P && (lane == 0 || eprev != er);
-        const uint32_t starts = __ballot_sync(0xffffffffu, start);
-        const int d = __popc(starts & ((2u << lane) - 1u)) - 1;
-        if (start) {
-            S.dex[d] = er;
-            S.dstart[d] = lane;
+        // rank r is the first pair of its expert iff no pair of the same expert has
+        // a lower rank, i.e. no q < lane has the same expert
+        bool first = lane < P;
+        if (lane < P)
+            for (int q = 0; q < lane; ++q) first &= S.sel_e[q] != ep;
+        const uint32_t firsts = __ballot_sync(0xffffffffu, first);
+        // distinct index of this pair's expert = distinct experts below it
+        int dless = 0;
+        if (lane < P)
+            for (int q = 0; q < P; ++q) dless += ((firsts >> q) & 1u) && S.sel_e[q] < ep;
+        if (first) {
+            S.dex[dless] = ep;
+            S.dstart[dless] = rank;
         }
-        if (lane < P) S.pdi[S.sp[lane]] = d;
+        if (lane < P) S.pdi[lane] = dless;
         if (lane == 0) {
-            S.nd = __popc(starts);
-            S.dstart[__popc(starts)] = P;
+            S.nd = __popc(firsts);
+            S.dstart[__popc(firsts)] = P;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            int ni = 0;
+            for (int dd = 0; dd < S.nd; ++dd)
+                for (int r = S.dstart[dd]; r < S.dstart[dd + 1]; r += 8) {
+                    S.item_d[ni] = dd;
+                    S.item_r[ni] = r;
+                    S.item_n[ni] = min(8, S.dstart[dd + 1] - r);
+                    ++ni;
+                }
+            S.n_items = ni;
         }
         if (blockIdx.x == 0 && lane < P) {
             p.sorted_pair[lane] = S.sp[lane];
@@ -413,38 +396,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     }
     __syncthreads();
     const int nd = S.nd;
-    const unsigned tag = S.tag;
-    const int n_gu = nd * p.gu_ntiles;
-    const int u0 = S.pf0[nd], u1 = S.pf1[nd];
-    const uint32_t dn_unit = (uint32_t)nd * p.dn_tile_bytes;
-    if (tracing && tid == 0) trace[9] = globaltimer();
+    const int ntu = I / 16;   // gate_up units per expert
+    const int gu0 = S.plan[nd][0], gu1 = S.plan[nd][1], dn0 = S.plan[nd][2], dn1 = S.plan[nd][3];
+    const int ngu = gu1 - gu0, ndn = dn1 - dn0;
+    const uint32_t dn_unit = (uint32_t)nd * dn_blk;
+    if (tracing && tid == 0) trace[9] = globaltimer_ns();
 
-    // ---- 3. one thread issues every weight load of this CTA now -------------------
-    if (tid == 0) {
-        for (int u = u0; u < u1; ++u) mbar_init(mbar0 + 8 * (u - u0), 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        uint32_t off = 0;
-        const uint32_t wb = smem_addr(wbuf);
-        for (int u = u0; u < u1; ++u) {
-            const uint32_t bar = mbar0 + 8 * (u - u0);
-            if (u < n_gu) {
-                const int dd = u / p.gu_ntiles, tile = u - dd * p.gu_ntiles;
-                const size_t tile_id = (size_t)S.dex[dd] * p.gu_ntiles + tile;
-                mbar_expect_tx(bar, p.gu_tile_bytes);
-                bulk_g2s(wb + off, p.gu_tiles + tile_id * p.gu_tile_bytes, p.gu_tile_bytes, bar);
-                off += p.gu_tile_bytes;
-            } else {
-                const int j = u - n_gu;
-                mbar_expect_tx(bar, dn_unit);
-                for (int dd = 0; dd < nd; ++dd) {
-                    const size_t tile_id = (size_t)S.dex[dd] * (H / 16) + j;
-                    bulk_g2s(wb + off + dd * p.dn_tile_bytes, p.dn_tiles + tile_id * p.dn_tile_bytes, p.dn_tile_bytes,
-                             bar);
-                }
-                off += dn_unit;
-            }
+    // ---- 3. warp 0 issues every weight load of this CTA now -------------------------
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int u = 0; u < ngu; ++u) mbar_expect_tx(mbar0 + 8 * u, gu_unit);
+            for (int u = 0; u < ndn; ++u) mbar_expect_tx(mbar0 + 8 * (ngu + u), dn_unit);
         }
-        if (tracing) trace[1] = globaltimer();
+        __syncwarp();
+        const uint32_t wb = smem_addr(wbuf);
+        for (int u = lane; u < ngu; u += 32) {
+            const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
+            bulk_g2s(wb + u * gu_unit, p.gu_blocks + ((size_t)S.dex[dd] * ntu + j) * gu_unit, gu_unit, mbar0 + 8 * u);
+        }
+        for (int i = lane; i < ndn * nd; i += 32) {
+            const int u = i / nd, dd = i - u * nd, j = dn0 + u;
+            bulk_g2s(wb + ngu * gu_unit + u * dn_unit + dd * dn_blk,
+                     p.dn_blocks + ((size_t)S.dex[dd] * (H / 16) + j) * dn_blk, dn_blk, mbar0 + 8 * (ngu + u));
+        }
+        if (tracing && lane == 0) trace[1] = globaltimer_ns();
     }
     if (blockIdx.x == 0) {
         for (int e = tid; e <= E; e += kDecThreads) {
@@ -458,12 +433,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         }
     }
 
-    // ---- 4. x as f16x2 with a power-of-two shift per token --------------------------
+    // ---- 4. x rows as fp16 pairs with a power-of-two shift per token (whole CTA) -------
     for (int t = 0; t < T; ++t) {
-        const uint32_t* xrow32 = reinterpret_cast<const uint32_t*>(xr + t * H);
+        const uint32_t* xw = reinterpret_cast<const uint32_t*>(xr + (size_t)t * H);
         float m = 0.0f;
         for (int r = tid; r < H / 2; r += kDecThreads) {
-            const uint32_t two = xrow32[r];
+            const uint32_t two = xw[r];
             m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32((uint16_t)(two & 0xffff))),
                                fabsf(bf16_bits_to_f32((uint16_t)(two >> 16)))));
         }
@@ -478,89 +453,75 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         const float scl = pow2f(-sh);
         if (tid == 0) S.xshift[t] = sh;
         for (int r = tid; r < H / 2; r += kDecThreads) {
-            const uint32_t two = xrow32[r];
-            xs[t * xrow + padrow(r)] = f32x2_to_f16x2_rn(bf16_bits_to_f32((uint16_t)(two & 0xffff)) * scl,
-                                                        bf16_bits_to_f32((uint16_t)(two >> 16)) * scl);
+            const uint32_t two = xw[r];
+            xs[t * xrw + r] = f32x2_to_f16x2_rn(bf16_bits_to_f32((uint16_t)(two & 0xffff)) * scl,
+                                               bf16_bits_to_f32((uint16_t)(two >> 16)) * scl);
         }
         __syncthreads();
     }
-    if (tracing && tid == 0) trace[2] = globaltimer();
+    if (tracing && tid == 0) trace[2] = globaltimer_ns();
+
+    if (tid == kDecThreads - 1) {
+        const unsigned tg = (ep_e0 + 1u) ? (ep_e0 + 1u) : 1u;
+        S.tag = tg;
+        if (ep_arrived == gridDim.x - 1) {
+            // every CTA has read the epoch: advance it for the next launch
+            atomicExch(p.sync, 0u);
+            st_release_gpu(p.sync + 1, tg);
+        }
+    }
+    __syncthreads();
 
     // ---- 5. gate_up units -> tagged act ------------------------------------------------
-    const int c = tid % C, g = tid / C;
-    const bool gvalid = g < G;
     uint32_t off = 0;
-    int u = u0;
-    for (; u < u1 && u < n_gu; ++u) {
-        const uint32_t bar = mbar0 + 8 * (u - u0);
+    for (int u = 0; u < ngu; ++u) {
+        const uint32_t bar = mbar0 + 8 * u;
         if (!mbar_wait0(bar, p.timeout_ns)) {
             if (tid == 0) { atomicOr(p.status, kDevLoadTimeout); S.abort = 1; }
         }
         __syncthreads();
         if (S.abort) break;
-        const int dd = u / p.gu_ntiles, tile = u - dd * p.gu_ntiles;
-        const uint8_t* cbase = wbuf + off;
-        const uint16_t* sbase = reinterpret_cast<const uint16_t*>(wbuf + off + (H / 2) * TW);
-        uint4 q[16];
-        float sc[16];
-        if (gvalid) {
+        const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
+        const uint8_t* blk0 = wbuf + off;
+        const uint8_t* blk1 = blk0 + block_bytes(H);
+        const int r0 = S.dstart[dd], r1 = S.dstart[dd + 1];
+        for (int nb = r0; nb < r1; nb += 8) {
+            const int nvalid = min(8, r1 - nb);
+            const uint32_t* brow = xs + (g < nvalid ? S.sp[nb + g] / k : T) * xrw;
+            float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int q = warp; q < H / 64; q += kDecWarps) quad_mma2(blk0, blk1, H, brow, q, lane, t0, t1);
+            float* rl = red + (warp * 32 + lane) * 8;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) q[i] = *reinterpret_cast<const uint4*>(cbase + (i * G + g) * TW + 16 * c);
-            const uint4 s0 = *reinterpret_cast<const uint4*>(sbase + g * TW + 16 * c);
-            const uint4 s1 = *reinterpret_cast<const uint4*>(sbase + g * TW + 16 * c + 8);
-            const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                sc[2 * i] = bf16_bits_to_f32((uint16_t)(sw[i] & 0xffff));
-                sc[2 * i + 1] = bf16_bits_to_f32((uint16_t)(sw[i] >> 16));
+            for (int i = 0; i < 4; ++i) {
+                rl[i] = t0[i];
+                rl[4 + i] = t1[i];
             }
-        }
-        for (int r = S.dstart[dd]; r < S.dstart[dd + 1]; ++r) {
-            const int pid = S.sp[r], t = pid / k;
-            float acc[16];
+            __syncthreads();
+            if (tid < 128) {
+                const int n = tid & 15, jt = tid >> 4;
+                if (jt < nvalid) {
+                    const int ln = 4 * (n & 7) + (jt >> 1), idx = (n >> 3) * 2 + (jt & 1);
+                    float gs = 0.0f, us = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-            if (gvalid) {
-                const uint32_t* xrw = xs + t * xrow;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t x2 = xrw[padrow(16 * g + i)];
-                    const uint32_t words[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
-#pragma unroll
-                    for (int wd = 0; wd < 4; ++wd) {
-                        uint32_t h[4];
-                        e2m1x8_to_f16x2x4(words[wd], h);
-#pragma unroll
-                        for (int b = 0; b < 4; ++b) acc[4 * wd + b] = fma2_f16_f32(h[b], x2, acc[4 * wd + b]);
+                    for (int w2 = 0; w2 < kDecWarps; ++w2) {
+                        gs += red[(w2 * 32 + ln) * 8 + idx];
+                        us += red[(w2 * 32 + ln) * 8 + 4 + idx];
                     }
+                    const int pid = S.sp[nb + jt], t = pid / k;
+                    const float m = pow2f(S.xshift[t]);
+                    const float a = silu_mul(gs * m, us * m);
+                    st_volatile_u64(p.act + (size_t)pid * I + 16 * j + n, ((unsigned long long)S.tag << 32) | __float_as_uint(a));
                 }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) acc[j] *= sc[j];
-            }
-            const int col0 = butterfly16<C>(acc, lane);
-#pragma unroll
-            for (int j = 0; j < Butterfly<C>::NOUT; ++j) red[warp * TW + 16 * c + col0 + j] = acc[j];
-            __syncthreads();
-            if (tid < TN) {
-                float gs = 0.0f, us = 0.0f;
-#pragma unroll
-                for (int w2 = 0; w2 < kDecWarps; ++w2) {
-                    gs += red[w2 * TW + tid];
-                    us += red[w2 * TW + TN + tid];
-                }
-                const float m = pow2f(S.xshift[t]);
-                const float a = silu_mul(gs * m, us * m);
-                st_volatile_u64(p.act + (size_t)pid * I + tile * TN + tid,
-                                ((unsigned long long)tag << 32) | __float_as_uint(a));
             }
             __syncthreads();
         }
-        off += p.gu_tile_bytes;
+        off += gu_unit;
     }
-    if (tracing && tid == 0) trace[3] = globaltimer();
+    if (tracing && tid == 0) trace[3] = globaltimer_ns();
 
     // ---- 6. down units: read act back (tagged), compute, combine ------------------------
-    if (u < u1 && !S.abort) {
+    const unsigned tag = S.tag;
+    if (ndn > 0 && !S.abort) {
         // warp pp stages pair pp: up to 16 chunks of two tagged words per lane, all
         // requested at once, then only the late ones again
         for (int pp = warp; pp < P; pp += kDecWarps) {
@@ -577,9 +538,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 }
             }
             if (__any_sync(0xffffffffu, pending != 0)) {
-                const unsigned long long t0 = globaltimer();
+                const unsigned long long t0 = globaltimer_ns();
                 bool late = false;
                 while (__any_sync(0xffffffffu, pending != 0) && !late) {
+                    __nanosleep(100);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         if ((pending >> i) & 1u) {
@@ -587,7 +549,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                             if ((unsigned)(a0[i] >> 32) == tag && (unsigned)(a1[i] >> 32) == tag) pending &= ~(1u << i);
                         }
                     }
-                    late = __any_sync(0xffffffffu, globaltimer() - t0 > p.timeout_ns);
+                    late = __any_sync(0xffffffffu, globaltimer_ns() - t0 > p.timeout_ns);
                 }
                 if (late && lane == 0) {
                     atomicOr(p.status, kDevBarrierTimeout);
@@ -607,59 +569,78 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;
                 if (2 * r < I)
-                    as[pp * arow + padrow(r)] = f32x2_to_f16x2_rn(__uint_as_float((uint32_t)a0[i]) * scl,
-                                                                 __uint_as_float((uint32_t)a1[i]) * scl);
+                    as[pp * arw + r] = f32x2_to_f16x2_rn(__uint_as_float((uint32_t)a0[i]) * scl,
+                                                        __uint_as_float((uint32_t)a1[i]) * scl);
             }
         }
         __syncthreads();
     }
-    if (tracing && tid == 0) trace[4] = globaltimer();
-    for (; u < u1; ++u) {
-        const uint32_t bar = mbar0 + 8 * (u - u0);
+    if (tracing && tid == 0) trace[4] = globaltimer_ns();
+    for (int u = 0; u < ndn; ++u) {
+        const uint32_t bar = mbar0 + 8 * (ngu + u);
         if (!mbar_wait0(bar, p.timeout_ns)) {
             if (tid == 0) { atomicOr(p.status, kDevLoadTimeout); S.abort = 1; }
         }
         __syncthreads();
-        const int j = u - n_gu;
-        const uint32_t cb = (uint32_t)(I / 2) * 16;
+        const int j = dn0 + u;
         if (!S.abort) {
-            for (int pp = warp; pp < P; pp += kDecWarps) {
-                const int di = S.pdi[pp];
-                const uint8_t* cbase = wbuf + off + di * p.dn_tile_bytes;
-                const uint16_t* sbase = reinterpret_cast<const uint16_t*>(cbase + cb);
-                const uint32_t* ar = as + pp * arow;
-                float tot[16];
+            // every warp runs a strided share of the 64-k quads for every routed
+            // expert (independent accumulator chains); partial sums go to dred,
+            // then warp dd adds the 8 warps' partials of expert dd in warp order
+            const int nq = I / 64;
+            const int n_items = S.n_items;
+            for (int i0 = 0; i0 < n_items; i0 += 8) {
+                const int dn = min(8, n_items - i0);
+                // 32 tasks = 8 items x 4 quarters of K; warp w runs tasks w + W*m:
+                // items (w/4) + (W/4)*m, all in quarter w % 4 (independent chains)
+                constexpr int TPW = 32 / kDecWarps;   // tasks per warp
+                const int quarter = warp & 3;
+                const int qa = quarter * nq / 4, qb = (quarter + 1) * nq / 4;
+                float tot[TPW][4];
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) tot[jj] = 0.0f;
-                if (lane < Gd) {
-                    const int gg = lane;
-                    float acc[16];
+                for (int m = 0; m < TPW; ++m)
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
+                    for (int c2 = 0; c2 < 4; ++c2) tot[m][c2] = 0.0f;
+                for (int q = qa; q < qb; ++q) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint4 qq = *reinterpret_cast<const uint4*>(cbase + (i * Gd + gg) * 16);
-                        const uint32_t x2 = ar[padrow(16 * gg + i)];
-                        const uint32_t words[4] = {qq.x, qq.y, qq.z, qq.w};
-#pragma unroll
-                        for (int wd = 0; wd < 4; ++wd) {
-                            uint32_t h[4];
-                            e2m1x8_to_f16x2x4(words[wd], h);
-#pragma unroll
-                            for (int b = 0; b < 4; ++b) acc[4 * wd + b] = fma2_f16_f32(h[b], x2, acc[4 * wd + b]);
+                    for (int m = 0; m < TPW; ++m) {
+                        const int i = (warp >> 2) + (kDecWarps / 4) * m;
+                        if (i < dn) {
+                            const int it = i0 + i;
+                            const int r0 = S.item_r[it], nvalid = S.item_n[it];
+                            const uint32_t* brow = as + (g < nvalid ? S.sp[r0 + g] : P) * arw;
+                            quad_mma(wbuf + off + S.item_d[it] * dn_blk, I, brow, q, lane, tot[m]);
                         }
                     }
-                    const uint4 s0 = *reinterpret_cast<const uint4*>(sbase + gg * 16);
-                    const uint4 s1 = *reinterpret_cast<const uint4*>(sbase + gg * 16 + 8);
-                    const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                }
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        tot[2 * i] = acc[2 * i] * bf16_bits_to_f32((uint16_t)(sw[i] & 0xffff));
-                        tot[2 * i + 1] = acc[2 * i + 1] * bf16_bits_to_f32((uint16_t)(sw[i] >> 16));
+                for (int m = 0; m < TPW; ++m) {
+                    const int i = (warp >> 2) + (kDecWarps / 4) * m;
+                    if (i < dn)
+#pragma unroll
+                        for (int c2 = 0; c2 < 4; ++c2) dred[((i * 4 + quarter) * 32 + lane) * 4 + c2] = tot[m][c2];
+                }
+                __syncthreads();
+                if (warp < dn) {
+                    const int it = i0 + warp;
+                    float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+                        for (int c2 = 0; c2 < 4; ++c2) acc4[c2] += dred[((warp * 4 + qq) * 32 + lane) * 4 + c2];
+                    const int r0 = S.item_r[it], nvalid = S.item_n[it];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int jt = 2 * (lane & 3) + e2;
+                        if (jt < nvalid) {
+                            const int pid = S.sp[r0 + jt];
+                            const float m = pow2f(S.ashift[pid]);
+                            S.ob[pid * 16 + g] = acc4[e2] * m;
+                            S.ob[pid * 16 + g + 8] = acc4[2 + e2] * m;
+                        }
                     }
                 }
-                const int col0 = butterfly16<1>(tot, lane);
-                if ((lane & 1) == 0) S.ob[pp * 16 + col0] = tot[0] * pow2f(S.ashift[pp]);
+                __syncthreads();
             }
         }
         __syncthreads();
@@ -672,11 +653,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         __syncthreads();
         off += dn_unit;
     }
-    if (tracing && tid == 0) trace[5] = globaltimer();
+    if (tracing && tid == 0) trace[5] = globaltimer_ns();
 
     // ---- 7. never leave with copies in flight --------------------------------------------
     if (S.abort && tid == 0)
-        for (int uu = u0; uu < u1; ++uu) mbar_wait0(mbar0 + 8 * (uu - u0), p.timeout_ns);
+        for (int u = 0; u < ngu + ndn; ++u) mbar_wait0(mbar0 + 8 * u, p.timeout_ns);
 }
 
 }  // namespace fe

@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "gemv.cuh"
 #include "gemv_canonical.cuh"
+#include "gmma.cuh"
 #include "pack.cuh"
 #include "route.cuh"
 
@@ -28,11 +29,10 @@ struct fe_moe_s {
     int path = 0;
     int sm_count = 0;
     int smem_optin = 0;
-    // column tiles (gemv.cuh): gate_up tiles hold TN gate + TN up columns
-    int gu_TW = 64, gu_tiles = 0;
-    int dn_TW = 128, dn_tiles = 0;
-    uint8_t* gu_tiles_buf = nullptr;   // [E][gu_tiles] tiles: codes then scales
-    uint8_t* dn_tiles_buf = nullptr;   // [E][dn_tiles]
+    // fragment-ordered blocks of 16 columns (pack.cuh): gate_up units of a
+    // gate block and its up block, down blocks
+    uint8_t* gu_blocks = nullptr;   // [E][I/16] x 18H bytes
+    uint8_t* dn_blocks = nullptr;   // [E][H/16] x 9I bytes
     bool loaded = false;
     // workspace
     int max_T = 0, max_k = 0;
@@ -48,7 +48,7 @@ struct fe_moe_s {
     float* act = nullptr;
     float* o = nullptr;
     unsigned long long* act_ll = nullptr;   // fused decode: tagged act words
-    int32_t* plan_first = nullptr;          // fused decode: work split per nd
+    int32_t* plan = nullptr;                // fused decode: work split per nd
     unsigned* dec_sync = nullptr;           // fused decode: finished CTAs, epoch
     unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
     uint32_t* status = nullptr;
@@ -105,7 +105,7 @@ void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
-                    h->act_ll, h->dec_sync, h->plan_first};
+                    h->act_ll, h->dec_sync, h->plan};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
@@ -113,7 +113,7 @@ void free_workspace(fe_moe_s* h)
     h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
     h->act_ll = nullptr;
     h->dec_sync = nullptr;
-    h->plan_first = nullptr;
+    h->plan = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -137,84 +137,50 @@ int roundup32(int v) { return (v + 31) / 32 * 32; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int NT, bool GU>
-cudaError_t launch_gemv(const fe::GemvParams& p, int grid, int threads, cudaStream_t s)
-{
-    const size_t smem = fe::gemv_smem_bytes<NT>(p.K, p.TW, threads);
-    fe::gemv_kernel<NT, GU><<<grid, threads, smem, s>>>(p);
-    return cudaGetLastError();
-}
-
-// Function attributes are process-wide, so every kernel is opted into the
-// device's largest dynamic shared memory once: a handle of another shape must
-// never lower the limit below what this handle's launches request.
-template <int NT, bool GU>
-cudaError_t allow_gemv_smem(int optin)
-{
-    return cudaFuncSetAttribute(fe::gemv_kernel<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-}
-
-using DecodeFn = void (*)(fe::DecodeParams);
-
-DecodeFn decode_kernel_for(int C)
-{
-    switch (C) {
-        case 2: return fe::decode_kernel<2>;
-        case 4: return fe::decode_kernel<4>;
-        case 8: return fe::decode_kernel<8>;
-        case 16: return fe::decode_kernel<16>;
-        default: return fe::decode_kernel<32>;
-    }
-}
-
-uint32_t gu_tile_bytes(const fe_moe_s* h) { return (uint32_t)((h->H / 2) * h->gu_TW + (h->H / 32) * h->gu_TW * 2); }
-uint32_t dn_tile_bytes(const fe_moe_s* h) { return (uint32_t)((h->I / 2) * 16 + (h->I / 32) * 32); }
-
-fe::DecodePlan plan_for(const fe_moe_s* h, int nd)
-{
-    return fe::decode_plan(nd, h->H, gu_tile_bytes(h), h->gu_tiles, dn_tile_bytes(h), h->sm_count);
-}
-
 // Largest per-CTA weight bytes of the fused decode split over every possible
 // number of distinct routed experts, or 0 if T, top_k or the shape exceed the
 // fused kernel.
 size_t decode_weight_bytes(const fe_moe_s* h, int T, int k)
 {
     const int P = T * k;
-    if (P > fe::kDecMaxPairs || h->sm_count <= 0 || h->I > 1024 || h->E > 1024 || h->H > 8192) return 0;
+    if (P > fe::kDecMaxPairs || h->sm_count <= 0 || h->I > 1024 || h->E > 1024) return 0;
     size_t worst = 0;
     const int nd_max = std::min(h->E, P);
+    std::vector<int> gf, df;
     for (int nd = 1; nd <= nd_max; ++nd) {
-        const fe::DecodePlan plan = plan_for(h, nd);
+        fe::decode_split(nd, h->H, h->I, h->sm_count, gf, df);
         for (int c = 0; c < h->sm_count; ++c) {
-            const int a = fe::decode_first_unit(plan, c), b = fe::decode_first_unit(plan, c + 1);
-            if (b - a > fe::kDecMaxItems) return 0;
-            size_t bytes = 0;
-            for (int u = a; u < b; ++u) bytes += (size_t)fe::decode_unit_bytes(plan, u);
+            const int ngu = gf[c + 1] - gf[c], ndn = df[c + 1] - df[c];
+            if (ngu + ndn > fe::kDecMaxItems) return 0;
+            const size_t bytes = (size_t)ngu * 2 * fe::block_bytes(h->H) + (size_t)ndn * nd * fe::block_bytes(h->I);
             worst = std::max(worst, bytes);
         }
     }
     return (worst + 127) / 128 * 128;
 }
 
-// Work-split table of the fused kernel: first unit of CTA c for nd distinct experts.
+// Work-split table of the fused kernel: [nd][gate_up | down][CTA] first units.
 cudaError_t build_plan_table(fe_moe_s* h)
 {
     const int cols = h->sm_count + 1;
-    std::vector<int32_t> tab((size_t)(fe::kDecMaxPairs + 1) * cols, 0);
+    std::vector<int32_t> tab((size_t)(fe::kDecMaxPairs + 1) * 2 * cols, 0);
+    std::vector<int> gf, df;
     for (int nd = 1; nd <= fe::kDecMaxPairs; ++nd) {
-        const fe::DecodePlan plan = plan_for(h, nd);
-        for (int c = 0; c <= h->sm_count; ++c) tab[(size_t)nd * cols + c] = fe::decode_first_unit(plan, c);
+        fe::decode_split(nd, h->H, h->I, h->sm_count, gf, df);
+        for (int c = 0; c < cols; ++c) {
+            tab[((size_t)nd * 2 + 0) * cols + c] = gf[c];
+            tab[((size_t)nd * 2 + 1) * cols + c] = df[c];
+        }
     }
-    cudaError_t e = cudaMalloc(&h->plan_first, tab.size() * sizeof(int32_t));
+    cudaError_t e = cudaMalloc(&h->plan, tab.size() * sizeof(int32_t));
     if (e != cudaSuccess) return e;
     h->work_bytes += tab.size() * sizeof(int32_t);
-    return cudaMemcpy(h->plan_first, tab.data(), tab.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    return cudaMemcpy(h->plan, tab.data(), tab.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
 }
 
 size_t decode_smem_total(const fe_moe_s* h, size_t wbytes, int T, int k)
 {
-    return fe::decode_smem_layout((uint32_t)wbytes, T, k, h->H, h->I, h->E, h->gu_TW).total;
+    return fe::decode_smem_layout((uint32_t)wbytes, T, k, h->H, h->I, h->E).total;
 }
 
 fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, int k, void* y, size_t wbytes,
@@ -225,9 +191,8 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     dp.logits = logits;
     dp.y = static_cast<uint16_t*>(y);
     dp.T = T; dp.E = h->E; dp.H = h->H; dp.I = h->I; dp.k = k;
-    dp.gu_tiles = h->gu_tiles_buf; dp.gu_ntiles = h->gu_tiles; dp.gu_tile_bytes = gu_tile_bytes(h);
-    dp.dn_tiles = h->dn_tiles_buf; dp.dn_tile_bytes = dn_tile_bytes(h);
-    dp.plan_first = h->plan_first;
+    dp.gu_blocks = h->gu_blocks; dp.dn_blocks = h->dn_blocks;
+    dp.plan = h->plan;
     dp.idx = h->idx; dp.w = h->w; dp.counts = h->counts; dp.offsets = h->offsets;
     dp.sorted_pair = h->sorted_pair; dp.pair_row = h->pair_row;
     dp.act = h->act_ll;
@@ -247,22 +212,21 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    FE_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel_for(h->gu_TW / 16), dp));
+    FE_CUDA_TRY(cudaLaunchKernelEx(&cfg, fe::decode_kernel, dp));
     return FE_OK;
 }
 
 // Opt the kernels into the device's largest dynamic shared memory (once,
-// outside any stream capture).
+// outside any stream capture).  Function attributes are process-wide, so a
+// handle of another shape must never lower the limit below what this
+// handle's launches request.
 cudaError_t configure_kernels(const fe_moe_s* h)
 {
     const int optin = h->smem_optin;
     cudaError_t e = cudaFuncSetAttribute(fe::route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-    if (e == cudaSuccess) e = allow_gemv_smem<1, true>(optin);
-    if (e == cudaSuccess) e = allow_gemv_smem<4, true>(optin);
-    if (e == cudaSuccess) e = allow_gemv_smem<1, false>(optin);
-    if (e == cudaSuccess) e = allow_gemv_smem<4, false>(optin);
-    for (int C = 2; C <= 32 && e == cudaSuccess; C *= 2)
-        e = cudaFuncSetAttribute(decode_kernel_for(C), cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fe::gmma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fe::gmma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fe::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     return e;
 }
 
@@ -270,38 +234,34 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
 {
     const int P = T * k;
     const int max_active = std::min(h->E, P);
-    fe::GemvParams gp{};
+    fe::GmmaParams gp{};
     gp.offsets = h->offsets;
     gp.active = h->active;
     gp.n_active = h->n_active;
     gp.sorted_pair = h->sorted_pair;
     gp.top_k = k;
-    // gate_up + SwiGLU: K = H, tiles of 32 gate + 32 up columns
-    gp.tiles = h->gu_tiles_buf;
+    gp.status = h->status;
+    gp.timeout_ns = 200ull * 1000 * 1000;
+    // gate_up + SwiGLU: K = H, units of 16 gate + 16 up columns
+    gp.blocks = h->gu_blocks;
     gp.K = h->H;
-    gp.TW = h->gu_TW;
-    gp.n_tiles = h->gu_tiles;
+    gp.n_units = h->I / 16;
     gp.N_out = h->I;
     gp.x = x;
     gp.act_in = nullptr;
     gp.out = h->act;
-    int threads = roundup32((h->gu_TW / 16) * (h->H / 32));
-    cudaError_t e = (T == 1) ? launch_gemv<1, true>(gp, max_active * h->gu_tiles, threads, s)
-                             : launch_gemv<4, true>(gp, max_active * h->gu_tiles, threads, s);
-    if (e != cudaSuccess) return record_cuda(e, "gate_up gemv launch");
-    // down: K = I
-    gp.tiles = h->dn_tiles_buf;
+    fe::gmma_kernel<true><<<max_active * gp.n_units, fe::kGmmaThreads, fe::gmma_smem_bytes(true, h->H), s>>>(gp);
+    FE_CUDA_TRY(cudaGetLastError());
+    // down: K = I, units of 16 output columns
+    gp.blocks = h->dn_blocks;
     gp.K = h->I;
-    gp.TW = h->dn_TW;
-    gp.n_tiles = h->dn_tiles;
+    gp.n_units = h->H / 16;
     gp.N_out = h->H;
     gp.x = nullptr;
     gp.act_in = h->act;
     gp.out = h->o;
-    threads = roundup32((h->dn_TW / 16) * (h->I / 32));
-    e = (T == 1) ? launch_gemv<1, false>(gp, max_active * h->dn_tiles, threads, s)
-                 : launch_gemv<4, false>(gp, max_active * h->dn_tiles, threads, s);
-    if (e != cudaSuccess) return record_cuda(e, "down gemv launch");
+    fe::gmma_kernel<false><<<max_active * gp.n_units, fe::kGmmaThreads, fe::gmma_smem_bytes(false, h->I), s>>>(gp);
+    FE_CUDA_TRY(cudaGetLastError());
     return FE_OK;
 }
 
@@ -331,11 +291,9 @@ fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out)
     if (group != 32) return FE_ERR_UNSUPPORTED;
     if (E < 1 || E > 1024 || H <= 0 || I <= 0 || H % 32 || I % 32) return FE_ERR_INVALID_ARG;
     // gate_up tiles: TW/2 gate + TW/2 up columns, so TW/2 must divide I
-    const int gu_TW = pick_tile_width(H, I, true);
-    // down tiles are 16 columns wide: the h-slice one CTA of the fused decode
-    // kernel owns for every routed expert (and a 1-chunk tile for the GEMV)
-    const int dn_TW = (I / 32 <= 256) ? 16 : 0;
-    if (gu_TW == 0 || dn_TW == 0) return FE_ERR_UNSUPPORTED;
+    // fragment-ordered blocks: 64-k quads along K, 16-column blocks along N
+    if (H % 64 || I % 64) return FE_ERR_UNSUPPORTED;
+    if (fe::gmma_smem_bytes(true, H) > 227 * 1024 || fe::gmma_smem_bytes(false, I) > 227 * 1024) return FE_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FE_ERR_CUDA;
     cudaDeviceProp prop;
@@ -348,15 +306,11 @@ fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out)
     h->E = E; h->H = H; h->I = I; h->device = dev;
     h->sm_count = prop.multiProcessorCount;
     h->smem_optin = optin;
-    h->gu_TW = gu_TW;
-    h->gu_tiles = I / (gu_TW / 2);
-    h->dn_TW = dn_TW;
-    h->dn_tiles = H / dn_TW;
     size_t acc = 0;
     cudaError_t e = cudaSuccess;
-    // codes (K/2 bytes per column) + scales (K/32 bf16 per column)
-    if (e == cudaSuccess) e = dmalloc(&h->gu_tiles_buf, (size_t)E * (2 * (size_t)I) * (H / 2 + H / 16), &acc);
-    if (e == cudaSuccess) e = dmalloc(&h->dn_tiles_buf, (size_t)E * (size_t)H * (I / 2 + I / 16), &acc);
+    // codes (K/2 bytes per column) + scales (K/32 bf16 per column), same bytes as the packed format
+    if (e == cudaSuccess) e = dmalloc(&h->gu_blocks, (size_t)E * (I / 16) * 2 * fe::block_bytes(H), &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->dn_blocks, (size_t)E * (H / 16) * fe::block_bytes(I), &acc);
     if (e == cudaSuccess) e = dmalloc(&h->status, 1, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(uint32_t));
     if (e != cudaSuccess) {
@@ -447,11 +401,11 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
         return FE_ERR_INVALID_ARG;
     }
     fe::RelayoutParams rp{};
-    rp.src_codes = sgc; rp.src_scales = sgs; rp.dst = h->gu_tiles_buf;
-    rp.E = E; rp.K = H; rp.N = 2 * I; rp.TW = h->gu_TW; rp.gate_up = 1;
+    rp.src_codes = sgc; rp.src_scales = sgs; rp.dst = h->gu_blocks;
+    rp.E = E; rp.K = H; rp.N = 2 * I; rp.gate_up = 1;
     fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
-    rp.src_codes = sdc; rp.src_scales = sds; rp.dst = h->dn_tiles_buf;
-    rp.K = I; rp.N = H; rp.TW = h->dn_TW; rp.gate_up = 0;
+    rp.src_codes = sdc; rp.src_scales = sds; rp.dst = h->dn_blocks;
+    rp.K = I; rp.N = H; rp.gate_up = 0;
     fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
     FE_CUDA_TRY(cudaGetLastError());
     if (staging) FE_CUDA_TRY(cudaFreeAsync(staging, s));
@@ -595,7 +549,7 @@ void fe_moe_destroy(fe_moe_t h)
         DeviceGuard g(h->device);
         cudaDeviceSynchronize();
         free_workspace(h);
-        void* ptrs[] = {h->gu_tiles_buf, h->dn_tiles_buf};
+        void* ptrs[] = {h->gu_blocks, h->dn_blocks};
         for (void* p : ptrs)
             if (p) cudaFree(p);
     }

@@ -1,5 +1,6 @@
-// Grouped FP4 GEMV for small token counts: the gate_up projection with the
-// SwiGLU epilogue, and the down projection.
+// Shared pieces of the CUDA-core FP4 GEMV (used by the public-layout kernel of
+// the allocation-free entry point, gemv_canonical.cuh) and the ordered
+// combine of the per-pair down outputs.
 //
 // "FireEcho Engine", section "The Goliath Kernel: Why It's Fast": packed FP4
 // bytes are loaded, split into the low and high nibble, multiplied by the
@@ -35,7 +36,6 @@
 namespace fe {
 
 struct GemvParams {
-    const uint8_t* tiles;     // [E][n_tiles] x {codes [16][K/32][TW], scales bf16 [K/32][TW]}
     int K;                    // reduction length
     int TW;                   // tile width in columns (bytes per row)
     int n_tiles;              // tiles per expert
@@ -118,122 +118,6 @@ FE_DEV void stage_inputs(const GemvParams& p, int e_pos0, int nt, uint32_t* xs, 
         }
     }
     __syncthreads();
-}
-
-// blockDim.x = roundup32(C * G) <= 256; grid.x = max_active * n_tiles.
-// Dynamic shared memory: xs (f16x2 rows) | red [nwarps][NT][TW] floats | shift[NT]
-template <int NT, bool GATE_UP>
-__global__ void __launch_bounds__(256) gemv_kernel(GemvParams p)
-{
-    extern __shared__ __align__(16) uint32_t gsm[];
-    const int a = blockIdx.x / p.n_tiles;
-    const int tile = blockIdx.x - a * p.n_tiles;
-    if (a >= *p.n_active) return;
-    const int e = p.active[a];
-    const int pos0 = p.offsets[e], npos = p.offsets[e + 1] - pos0;
-
-    const int K = p.K, TW = p.TW, C = TW / 16, G = K / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    const int c = tid % C, g = tid / C;
-    const bool valid = g < G;
-
-    uint32_t* xs = gsm;
-    float* red = reinterpret_cast<float*>(gsm + xs_words<NT>(K));
-    int* shift = reinterpret_cast<int*>(red + nwarps * NT * TW);
-
-    // this thread's weights: 16 rows x 16 bytes and 16 scales
-    const size_t tile_id = (size_t)e * p.n_tiles + tile;
-    const uint8_t* wt = p.tiles + tile_id * ((size_t)(K / 2) * TW + (size_t)G * TW * 2);
-    const uint16_t* st = reinterpret_cast<const uint16_t*>(wt + (size_t)(K / 2) * TW);
-    uint4 q[16];
-    float sc[16];
-    if (valid) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = ldg_stream(wt + ((size_t)i * G + g) * TW + 16 * c);
-        const uint4 s0 = *reinterpret_cast<const uint4*>(st + (size_t)g * TW + 16 * c);
-        const uint4 s1 = *reinterpret_cast<const uint4*>(st + (size_t)g * TW + 16 * c + 8);
-        const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            sc[2 * i] = bf16_bits_to_f32((uint16_t)(sw[i] & 0xffff));
-            sc[2 * i + 1] = bf16_bits_to_f32((uint16_t)(sw[i] >> 16));
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sc[i] = 0.0f;
-    }
-
-    for (int c0 = 0; c0 < npos; c0 += NT) {
-        const int nt = min(NT, npos - c0);
-        stage_inputs<NT, GATE_UP>(p, pos0 + c0, nt, xs, shift, red);
-        // partial dot products of this thread's group for every token of the chunk
-        float acc[NT][16];
-#pragma unroll
-        for (int tok = 0; tok < NT; ++tok)
-#pragma unroll
-            for (int j = 0; j < 16; ++j) acc[tok][j] = 0.0f;
-        if (valid) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                uint32_t x2[NT];
-#pragma unroll
-                for (int tok = 0; tok < NT; ++tok) x2[tok] = xs[xs_index<NT>(16 * g + i, tok)];
-                const uint32_t words[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
-#pragma unroll
-                for (int wd = 0; wd < 4; ++wd) {
-                    uint32_t h[4];
-                    e2m1x8_to_f16x2x4(words[wd], h);
-#pragma unroll
-                    for (int b = 0; b < 4; ++b)
-#pragma unroll
-                        for (int tok = 0; tok < NT; ++tok)
-                            acc[tok][4 * wd + b] = fma2_f16_f32(h[b], x2[tok], acc[tok][4 * wd + b]);
-                }
-            }
-        }
-#pragma unroll
-        for (int tok = 0; tok < NT; ++tok) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float v = acc[tok][j] * sc[j];
-                // reduce over the lanes of this warp that hold the same chunk
-                for (int o = C; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                acc[tok][j] = v;
-            }
-            if (lane < C) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) red[(warp * NT + tok) * TW + 16 * lane + j] = acc[tok][j];
-            }
-        }
-        __syncthreads();
-        // finish the K reduction and write
-        if (GATE_UP) {
-            const int TN = TW / 2;
-            for (int i = tid; i < NT * TN; i += blockDim.x) {
-                const int tok = i / TN, n = i - tok * TN;
-                if (tok >= nt) continue;
-                float gsum = 0.0f, usum = 0.0f;
-                for (int w = 0; w < nwarps; ++w) {
-                    gsum += red[(w * NT + tok) * TW + n];
-                    usum += red[(w * NT + tok) * TW + TN + n];
-                }
-                const float m = __uint_as_float((uint32_t)(127 + shift[tok]) << 23);
-                p.out[(size_t)(pos0 + c0 + tok) * p.N_out + tile * TN + n] = silu_mul(gsum * m, usum * m);
-            }
-        } else {
-            for (int i = tid; i < NT * TW; i += blockDim.x) {
-                const int tok = i / TW, n = i - tok * TW;
-                if (tok >= nt) continue;
-                float s = 0.0f;
-                for (int w = 0; w < nwarps; ++w) s += red[(w * NT + tok) * TW + n];
-                const float m = __uint_as_float((uint32_t)(127 + shift[tok]) << 23);
-                p.out[(size_t)(pos0 + c0 + tok) * p.N_out + tile * TW + n] = s * m;
-            }
-        }
-        __syncthreads();
-    }
 }
 
 template <int NT>

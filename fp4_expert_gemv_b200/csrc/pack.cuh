@@ -60,65 +60,77 @@ __global__ void pack_kernel(const float* __restrict__ W, int64_t E, int64_t K, i
     }
 }
 
-// Re-layout of one matrix family into column tiles (see gemv.cuh):
-//   src codes  [E][K/2][N], src scales [E][K/32][N]
-//   dst        [E][n_tiles] tiles of tile_bytes = (K/2)*TW + (K/32)*TW*2:
-//              codes [16][K/32][TW] -- entry (i, g, j) is source byte row
-//              16*g + i (k = 32g + 2i, 32g + 2i + 1) of tile column j, so the
-//              16 rows of one 32-k group are (K/32) * TW bytes apart and
-//              consecutive groups are adjacent -- then the scales [K/32][TW]
-// Tile column j maps to source column col(tile, j): for the fused gate_up
-// matrix (TN = TW/2, I = N/2) j < TN -> tile*TN + j (gate), j >= TN ->
-// I + tile*TN + j - TN (up); otherwise tile*TW + j.
+// Re-layout of one expert matrix family into fragment-ordered column blocks.
+//
+// A block is 16 columns x K of one expert matrix (the A operand of a
+// tensor-core mma.m16n8k16 whose 16 rows are the block's columns and whose K
+// is the reduction), stored as one contiguous 9K-byte run:
+//   codes  K/64 quads of 512 bytes: byte 16*L + 4*s + j of quad q is the
+//          source byte (k-pair row 8*(4q+s) + t + 4*(j>>1), column g + 8*(j&1))
+//          with lane L = 4g + t; so lane L of a warp finds, in one 16-byte
+//          word, its four A-fragment registers for the four 16-k steps of the
+//          quad, each register one byte = (w[k even], w[k odd]) of one column;
+//   scales K/32 groups of 8 words: word g of group G holds the bf16 scales of
+//          columns g (low half) and g + 8 (high half), the two rows of the
+//          mma accumulator a lane owns.
+// For the fused gate_up matrix the block of gate columns [16j, 16j+16) is
+// followed by the block of up columns [I+16j, I+16j+16), so one gate_up unit
+// (both halves of 16 act columns) is one contiguous 18K-byte run.
 struct RelayoutParams {
-    const uint8_t* src_codes;
-    const uint16_t* src_scales;
-    uint8_t* dst;
+    const uint8_t* src_codes;   // [E][K/2][N]
+    const uint16_t* src_scales; // [E][K/32][N]
+    uint8_t* dst;               // [E][N/16] blocks of 9K bytes
     int64_t E, K, N;
-    int TW;
     int gate_up;
 };
 
-FE_DEV int64_t relayout_src_col(const RelayoutParams& p, int64_t tile, int64_t j)
+FE_DEV int64_t relayout_block_col0(const RelayoutParams& p, int64_t blk)
 {
     if (p.gate_up) {
-        const int64_t TN = p.TW / 2, I = p.N / 2;
-        return (j < TN) ? tile * TN + j : I + tile * TN + (j - TN);
+        const int64_t I = p.N / 2, j = blk >> 1;
+        return (blk & 1) ? I + 16 * j : 16 * j;
     }
-    return tile * p.TW + j;
+    return 16 * blk;
 }
 
-// One thread per 16 destination bytes (codes) / 8 destination scales.
+// One thread per destination 4-byte word (codes) or scale word.
 __global__ void relayout_kernel(RelayoutParams p)
 {
-    const int64_t n_tiles = p.N / p.TW;
-    const int64_t rows = p.K / 2, G = p.K / 32;
-    const int64_t tile_bytes = rows * p.TW + G * p.TW * 2;
-    const int64_t cchunks = p.E * n_tiles * rows * (p.TW / 16);
-    const int64_t schunks = p.E * n_tiles * G * (p.TW / 8);
+    const int64_t nblk = p.N / 16, K = p.K;
+    const int64_t blk_bytes = 9 * K;
+    const int64_t cwords = K / 8;     // 8K bytes of codes -> 2K words; per block: K/64 quads * 128 words
+    const int64_t code_words = (K / 64) * 128;
+    const int64_t scale_words = (K / 32) * 8;
+    const int64_t per_blk = code_words + scale_words;
+    (void)cwords;
+    const int64_t total = p.E * nblk * per_blk;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < cchunks + schunks; i += stride) {
-        if (i < cchunks) {
-            const int64_t jc = i % (p.TW / 16);
-            int64_t rest = i / (p.TW / 16);
-            const int64_t dr = rest % rows;           // destination row = ii * G + g
-            rest /= rows;
-            const int64_t tile = rest % n_tiles, e = rest / n_tiles;
-            const int64_t ii = dr / G, g = dr % G;
-            const int64_t r = 16 * g + ii;            // source byte row
-            const int64_t col = relayout_src_col(p, tile, 16 * jc);   // 16 consecutive source columns
-            const uint4 v = *reinterpret_cast<const uint4*>(p.src_codes + (e * rows + r) * p.N + col);
-            *reinterpret_cast<uint4*>(p.dst + (e * n_tiles + tile) * tile_bytes + dr * p.TW + 16 * jc) = v;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t w = i % per_blk;
+        const int64_t eb = i / per_blk;            // e * nblk + blk
+        const int64_t e = eb / nblk, blk = eb % nblk;
+        const int64_t col0 = relayout_block_col0(p, blk);
+        uint32_t v = 0;
+        uint8_t* dst = p.dst + eb * blk_bytes;
+        if (w < code_words) {
+            const int64_t q = w / 128, r = w % 128;
+            const int L = (int)(r / 4), s = (int)(r % 4);
+            const int g = L >> 2, t = L & 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t kp = 8 * (4 * q + s) + t + 4 * (j >> 1);
+                const int64_t col = col0 + g + 8 * (j & 1);
+                const uint32_t byte = p.src_codes[(e * (K / 2) + kp) * p.N + col];
+                v |= byte << (8 * j);
+            }
+            *reinterpret_cast<uint32_t*>(dst + 512 * q + 16 * L + 4 * s) = v;
         } else {
-            const int64_t i2 = i - cchunks;
-            const int64_t jc = i2 % (p.TW / 8);
-            int64_t rest = i2 / (p.TW / 8);
-            const int64_t g = rest % G;
-            rest /= G;
-            const int64_t tile = rest % n_tiles, e = rest / n_tiles;
-            const int64_t col = relayout_src_col(p, tile, 8 * jc);
-            const uint4 v = *reinterpret_cast<const uint4*>(p.src_scales + (e * G + g) * p.N + col);
-            *reinterpret_cast<uint4*>(p.dst + (e * n_tiles + tile) * tile_bytes + rows * p.TW + (g * p.TW + 8 * jc) * 2) = v;
+            const int64_t ws = w - code_words;
+            const int64_t G = ws / 8;
+            const int g = (int)(ws % 8);
+            const uint32_t lo = p.src_scales[(e * (K / 32) + G) * p.N + col0 + g];
+            const uint32_t hi = p.src_scales[(e * (K / 32) + G) * p.N + col0 + g + 8];
+            *reinterpret_cast<uint32_t*>(dst + 8 * K + 4 * ws) = lo | (hi << 16);
         }
     }
 }

@@ -209,6 +209,10 @@ def test_edge_cases(torch_cuda, path):
     lg_hot[:, 5] += 100.0
     run_and_check(gl, osd, x, lg_hot, 1, what="all tokens to one expert")
     run_and_check(gl, osd, x, lg_hot, 2, what="one hot expert, k=2")
+    # 12 tokens on one expert through the single-launch kernel: two 8-token blocks
+    run_and_check(gl, osd, x[:12], lg_hot[:12], 1, what="one hot expert, T=12, k=1")
+    if path == "auto":
+        assert gl.layer.last_forward_info()[0] == fe.PATH_FUSED_DECODE
     # ties: equal logits everywhere, and pairwise ties
     lg_tie = np.zeros((6, E), np.float32)
     lg_tie[1, :] = 1.0
