@@ -26,7 +26,7 @@ constexpr uint32_t kDevNanLogit = 0x2;
 // ---------------------------------------------------------------------------
 FE_DEV void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&h)[4])
 {
-    asm volatile("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
         "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
         "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"

@@ -46,6 +46,8 @@ constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecMaxPairs = 16;   // T * top_k handled by the fused kernel
 constexpr int kDecMaxItems = 48;   // weight units (mbarriers) per CTA
+constexpr int kDecMaxE = 512;      // experts routed by one warp: 16 logits per lane
+constexpr int kDecCandCap = 128;   // candidate keys per routing warp (in the gate_up partials' space)
 constexpr uint32_t kDevBarrierTimeout = 0x4;
 constexpr uint32_t kDevLoadTimeout = 0x8;
 
@@ -64,12 +66,12 @@ struct DecodeParams {
     int32_t* sorted_pair;
     int32_t* pair_row;
     unsigned long long* act;  // [kDecMaxPairs][I] by pair id: (epoch tag << 32) | fp32 bits
-    unsigned* sync;           // [2]: CTAs that read the epoch this launch, epoch
+    unsigned* epoch;          // [grid]: launches CTA c has run on this handle (the act tag of the last)
     uint32_t* status;
     unsigned long long timeout_ns;  // bound of every wait
     uint32_t weight_bytes;    // shared memory reserved for weight units
     int bulk_inputs;          // x and logits rows copied with cp.async.bulk (16-byte aligned)
-    unsigned long long* trace;  // optional [grid][16] %globaltimer stamps of the phases
+    unsigned long long* trace;  // optional [grid][64]: %globaltimer (0-31) and clock64 (32-63) stamps of the phases
 };
 
 // ---- work split (host only: the kernel reads the table) ---------------------------
@@ -146,16 +148,11 @@ FE_DEV void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar
                  : "memory");
 }
 
-FE_DEV unsigned ld_acquire_gpu(const unsigned* p)
+// Phase stamp i of the optional trace: %globaltimer and the SM's cycle counter.
+FE_DEV void stamp(unsigned long long* trace, int i)
 {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-FE_DEV void st_release_gpu(unsigned* p, unsigned v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    trace[i] = globaltimer_ns();
+    trace[32 + i] = (unsigned long long)clock64();
 }
 
 FE_DEV void st_volatile_u64(unsigned long long* p, unsigned long long v)
@@ -168,7 +165,136 @@ FE_DEV void ld_volatile_2u64(const unsigned long long* p, unsigned long long& a,
     asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
 
-FE_DEV float logit_key(float v) { return v != v ? -INFINITY : v; }
+// ---- routing ---------------------------------------------------------------------
+// Orderable key of logit v of expert e: a larger key ranks first.  NaN ranks
+// as -inf, -0 as +0, and among equal logits the lower expert index ranks
+// first, so keys are unique and the top-k order is the stable one.  A valid
+// key is never 0.
+FE_DEV unsigned long long route_key(float v, int e)
+{
+    uint32_t u = __float_as_uint(v != v ? -INFINITY : v);
+    if ((u << 1) == 0u) u = 0u;
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)ord << 32) | (0xffffffffu - (uint32_t)e);
+}
+
+FE_DEV float route_key_value(unsigned long long key)
+{
+    const uint32_t ord = (uint32_t)(key >> 32);
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+}
+
+FE_DEV int route_key_expert(unsigned long long key) { return (int)(0xffffffffu - (uint32_t)key); }
+
+// One warp selects the top-k (E <= 32 J) logits of one token row (global
+// memory), writing slot r = rank r: sel_e[r] expert, sel_w[r] logit.  Lane l
+// holds the keys of experts l, l+32, ...  A threshold theta such that k
+// lanes hold a key >= theta puts every key of the top k among the
+// candidates (keys >= theta), and since every key above a candidate is a
+// candidate too, a candidate's rank among the candidates is its rank among
+// all E.  theta is first the k-th largest lane maximum by value (one 32-bit
+// pass, ties counted); if that leaves more than 64 candidates (values tied
+// around it) it is refined to the k-th largest lane maximum key, which
+// leaves at most k J.  The candidates go to `cand` at slots counted from
+// ballots and each is ranked by counting.  cap >= max(64, k J) is the caller's
+// guarantee.  Returns whether the row holds a NaN (warp-uniform).
+template <int J>
+FE_DEV bool warp_topk(const float* row, int E, int k, int lane, unsigned long long* cand, int cap, int* sel_e,
+                      float* sel_w)
+{
+    constexpr unsigned FULL = 0xffffffffu;
+    unsigned long long key[J];
+    unsigned long long kmax = 0ull;
+    bool nan = false;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int e = lane + 32 * j;
+        key[j] = 0ull;
+        if (e < E) {
+            const float v = row[e];
+            nan |= v != v;
+            key[j] = route_key(v, e);
+        }
+        kmax = kmax > key[j] ? kmax : key[j];
+    }
+    // a lane whose maximum is below the k-th largest has >= k lanes strictly
+    // above it; lanes without a logit (E < 32) hold 0, below every valid key
+    const uint32_t omax = (uint32_t)(kmax >> 32);
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+#pragma unroll
+    for (int s = 0; s < 32; s += 4) {
+        r0 += __shfl_sync(FULL, omax, s) > omax;
+        r1 += __shfl_sync(FULL, omax, s + 1) > omax;
+        r2 += __shfl_sync(FULL, omax, s + 2) > omax;
+        r3 += __shfl_sync(FULL, omax, s + 3) > omax;
+    }
+    const uint32_t theta = __reduce_min_sync(FULL, (r0 + r1 + r2 + r3) < k ? omax : 0xffffffffu);
+    const unsigned long long theta_key = (unsigned long long)theta << 32;   // smallest key of value theta
+    int nc = 0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) nc += __popc(__ballot_sync(FULL, key[j] >= theta_key));
+    unsigned long long th = theta_key;
+    if (nc > 64) {
+        int q0 = 0, q1 = 0;
+#pragma unroll
+        for (int s = 0; s < 32; s += 2) {
+            q0 += __shfl_sync(FULL, kmax, s) > kmax;
+            q1 += __shfl_sync(FULL, kmax, s + 1) > kmax;
+        }
+        unsigned long long m = (q0 + q1) < k ? kmax : ~0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(FULL, m, o);
+            m = other < m ? other : m;
+        }
+        th = m;
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    nc = 0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const bool c = key[j] >= th;
+        const uint32_t bj = __ballot_sync(FULL, c);
+        const int pos = nc + __popc(bj & lt);
+        if (c && pos < cap) cand[pos] = key[j];
+        nc += __popc(bj);
+    }
+    nc = min(nc, cap);
+    __syncwarp();
+    for (int ci = lane; ci < nc; ci += 32) {
+        const unsigned long long mine = cand[ci];
+        int rank = 0;
+#pragma unroll 4
+        for (int q = 0; q < nc; ++q) rank += cand[q] > mine;
+        if (rank < k) {
+            sel_e[rank] = route_key_expert(mine);
+            sel_w[rank] = route_key_value(mine);
+        }
+    }
+    __syncwarp();
+    return __any_sync(FULL, nan);
+}
+
+FE_DEV bool warp_route(const float* row, int E, int k, int lane, unsigned long long* cand, int cap, int* sel_e,
+                       float* sel_w)
+{
+    if (E <= 32) return warp_topk<1>(row, E, k, lane, cand, cap, sel_e, sel_w);
+    if (E <= 64) return warp_topk<2>(row, E, k, lane, cand, cap, sel_e, sel_w);
+    if (E <= 128) return warp_topk<4>(row, E, k, lane, cand, cap, sel_e, sel_w);
+    if (E <= 256) return warp_topk<8>(row, E, k, lane, cand, cap, sel_e, sel_w);
+    return warp_topk<16>(row, E, k, lane, cand, cap, sel_e, sel_w);
+}
+
+// Softmax of one token's k selected logits (slot order) in place, by one warp.
+FE_DEV void warp_softmax(float* sel_w, int k, int lane)
+{
+    const float l0 = sel_w[0];
+    const float ej = lane < k ? expf(sel_w[lane] - l0) : 0.0f;
+    const float ssum = warp_sum(ej);
+    __syncwarp();
+    if (lane < k) sel_w[lane] = ej / ssum;
+    __syncwarp();
+}
 
 struct DecodeShared {
     int sel_e[kDecMaxPairs];
@@ -187,14 +313,39 @@ struct DecodeShared {
     int nd;
     int abort;
     unsigned tag;
-    float wmax[kDecWarps];
-    int rank_part[kDecThreads];
+    float wmax[2][kDecWarps];
     float ob[kDecMaxPairs * 16];  // down: [pair][16] outputs
 };
 
+
+// Single-token grouping: k distinct experts, the sorted position of slot
+// `lane` is the number of selected experts below its own.
+FE_DEV void group_single_token(DecodeShared& S, int k, int lane)
+{
+    if (lane < k) {
+        const int ep = S.sel_e[lane];
+        int pos = 0;
+#pragma unroll 4
+        for (int q = 0; q < k; ++q) pos += S.sel_e[q] < ep;
+        S.sp[pos] = lane;
+        S.pdi[lane] = pos;
+        S.dex[pos] = ep;
+        S.dstart[pos] = pos;
+        S.item_d[pos] = pos;
+        S.item_r[pos] = pos;
+        S.item_n[pos] = 1;
+    }
+    if (lane == 0) {
+        S.nd = k;
+        S.dstart[k] = k;
+        S.n_items = k;
+    }
+    __syncwarp();
+}
+
 // Byte offsets of the dynamic shared memory regions.
 struct DecodeSmem {
-    uint32_t mbar, shared, red, dred, xs, as, lg, xr, total;
+    uint32_t mbar, shared, red, dred, xs, as, xr, total;
 };
 
 __host__ __device__ inline uint32_t align16(uint32_t v) { return (v + 15u) & ~15u; }
@@ -209,8 +360,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(uint32_t weight_bytes, 
     L.dred = L.red;   // gate_up partials and down partials are never live together
     L.xs = L.red + 4u * (kDecWarps * 32 * 8 > 8 * 4 * 32 * 4 ? kDecWarps * 32 * 8 : 8 * 4 * 32 * 4);
     L.as = L.xs + 4u * (T + 1) * brow_words(H);
-    L.lg = align16(L.as + 4u * (T * k + 1) * brow_words(I));
-    L.xr = align16(L.lg + 4u * T * E);
+    L.xr = align16(L.as + 4u * (T * k + 1) * brow_words(I));
     L.total = align16(L.xr + 2u * T * H);
     return L;
 }
@@ -231,167 +381,202 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     float* dred = reinterpret_cast<float*>(dsm + L.dred);   // down partials [8 items][4 quarters][lane][4]
     uint32_t* xs = reinterpret_cast<uint32_t*>(dsm + L.xs);
     uint32_t* as = reinterpret_cast<uint32_t*>(dsm + L.as);
-    float* lg = reinterpret_cast<float*>(dsm + L.lg);
     uint16_t* xr = reinterpret_cast<uint16_t*>(dsm + L.xr);
     const uint32_t mbar0 = smem_addr(dsm + L.mbar);
     const uint32_t in_bar = mbar0 + 8 * kDecMaxItems;
     const bool tracing = p.trace != nullptr;
-    unsigned long long* trace = tracing ? p.trace + (size_t)blockIdx.x * 16 : nullptr;
-    if (tracing && tid == 0) trace[0] = globaltimer_ns();
+    unsigned long long* trace = tracing ? p.trace + (size_t)blockIdx.x * 64 : nullptr;
+    if (tracing && tid == 0) stamp(trace, 0);
 
     // ---- 0. static data only, then wait for the previous grid ---------------------
-    if (tid < 4 * (kDecMaxPairs + 1)) {
-        const int nd = tid >> 2, which = tid & 3;   // 0: gate_up first, 1: end, 2: down first, 3: end
+    if (tid >= 64 && tid < 64 + 4 * (kDecMaxPairs + 1)) {
+        // (warps 2-4: the routing warp goes straight to the logits)
+        const int nd = (tid - 64) >> 2, which = tid & 3;   // 0: gate_up first, 1: end, 2: down first, 3: end
         const int32_t* row = p.plan + ((size_t)nd * 2 + (which >> 1)) * (gridDim.x + 1);
         S.plan[nd][which] = row[blockIdx.x + (which & 1)];
     }
-    if (tid == 0) {
-        for (int u = 0; u <= kDecMaxItems; ++u) mbar_init(mbar0 + 8 * u, 1);   // the weight units' and in_bar
+    if (warp == 1) {
+        // lane 16 initialises in_bar (index kDecMaxItems) and issues the x copy below
+        for (int u = lane; u <= kDecMaxItems; u += 32) mbar_init(mbar0 + 8 * u, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        S.abort = 0;
+        if (lane == 0) S.abort = 0;
     }
     for (int i = tid; i < xrw; i += kDecThreads) xs[T * xrw + i] = 0u;       // zero B rows
     for (int i = tid; i < arw; i += kDecThreads) as[P * arw + i] = 0u;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (tid == 0 && p.bulk_inputs) {
-        const uint32_t lb = 4u * T * E, xb = 2u * T * H;
-        mbar_expect_tx(in_bar, lb + xb);
-        bulk_g2s(smem_addr(lg), p.logits, lb, in_bar);
+    if (tracing && tid == 0) stamp(trace, 8);
+    if (warp == 1 && lane == 16 && p.bulk_inputs) {
+        const uint32_t xb = 2u * T * H;
+        mbar_expect_tx(in_bar, xb);
         bulk_g2s(smem_addr(xr), p.x, xb, in_bar);
     }
-    // this launch's epoch (the previous launch's update is visible after
-    // griddepcontrol.wait); both requests are in flight while the CTA routes and
-    // their results are consumed only when act is about to be written
-    unsigned ep_e0 = 0, ep_arrived = 0;
-    if (tid == kDecThreads - 1) {
-        ep_e0 = *reinterpret_cast<volatile unsigned*>(p.sync + 1);
-        ep_arrived = atomicAdd(p.sync, 1u);
-    }
-    if (!p.bulk_inputs) {
-        for (int i = tid; i < T * E; i += kDecThreads) lg[i] = p.logits[i];
-        for (int i = tid; i < T * H; i += kDecThreads) xr[i] = p.x[i];
-    }
-    __syncthreads();
-    if (p.bulk_inputs && !mbar_wait0(in_bar, p.timeout_ns)) {
-        if (tid == 0) atomicOr(p.status, kDevLoadTimeout);
-        return;
-    }
-    if (tracing && tid == 0) trace[8] = globaltimer_ns();
+    // this launch's act tag: every launch runs every CTA once, so the per-CTA
+    // launch counts move in lockstep and all CTAs derive the same tag without
+    // talking to each other; the load is consumed only when act is about to be written
+    unsigned ep_e0 = 0;
+    if (tid == kDecThreads - 1) ep_e0 = *reinterpret_cast<volatile unsigned*>(p.epoch + blockIdx.x);
+    // candidate keys of the routing warps live in the gate_up partials' space
+    const int nroute = min(T, kDecWarps);
+    const int cap = (kDecWarps * kDecCandCap) / nroute;
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(red) + warp * cap;
 
-    // ---- 1. routing: rank of every logit among its token's E logits ------------------
-    // nsplit threads share the comparisons of one logit (E <= 128: 2 or more)
-    bool nan_seen = false;
-    {
-        const int epad = (E + 31) & ~31;
-        const int nsplit = epad >= kDecThreads ? 1 : kDecThreads / epad;
-        const int chunk = ((E + nsplit - 1) / nsplit + 3) & ~3;
-        int* rk = S.rank_part;
-        for (int t = 0; t < T; ++t) {
-            const float* row = lg + t * E;
-            for (int base = 0; base < E; base += kDecThreads / nsplit) {
-                const int e = base + tid % epad, part = tid / epad;
-                int rank = 0;
-                if (e < E && part < nsplit) {
-                    const float v = logit_key(row[e]);
-                    nan_seen |= row[e] != row[e];
-                    const int lo = part * chunk, hi = min(E, lo + chunk);
-                    int e2 = lo;
-                    if ((E & 3) == 0) {
-#pragma unroll 4
-                        for (; e2 + 4 <= hi; e2 += 4) {
-                            const float4 o = *reinterpret_cast<const float4*>(row + e2);
-                            const float o0 = logit_key(o.x), o1 = logit_key(o.y), o2 = logit_key(o.z), o3 = logit_key(o.w);
-                            rank += (o0 > v) || (o0 == v && e2 < e);
-                            rank += (o1 > v) || (o1 == v && e2 + 1 < e);
-                            rank += (o2 > v) || (o2 == v && e2 + 2 < e);
-                            rank += (o3 > v) || (o3 == v && e2 + 3 < e);
-                        }
-                    }
-                    for (; e2 < hi; ++e2) {
-                        const float o = logit_key(row[e2]);
-                        rank += (o > v) || (o == v && e2 < e);
-                    }
-                }
-                if (nsplit > 1) {
-                    rk[tid] = rank;
-                    __syncthreads();
-                    if (part == 0 && e < E) {
-                        for (int q = 1; q < nsplit; ++q) rank += rk[tid + q * epad];
-                    }
-                    __syncthreads();
-                }
-                if (part == 0 && e < E && rank < k) {
-                    S.sel_e[t * k + rank] = e;
-                    S.sel_w[t * k + rank] = logit_key(row[e]);
-                }
-            }
+    // ---- 1. routing: warp t selects the top-k logits of token t ----------------------
+    // With T = 1, warp 0 routes and goes straight on to the loads (the softmax
+    // and the published routing come after them); with T > 1 every token's
+    // warp also takes its softmax, then the CTA meets before the grouping.
+    if (warp < nroute) {
+        for (int t = warp; t < T; t += kDecWarps) {
+            const bool nan = warp_route(p.logits + (size_t)t * E, E, k, lane, cand, cap, S.sel_e + t * k, S.sel_w + t * k);
+            if (nan && lane == 0 && blockIdx.x == 0) atomicOr(p.status, kDevNanLogit);
+            if (T > 1) warp_softmax(S.sel_w + t * k, k, lane);
         }
     }
-    if (tracing && tid == 0) trace[10] = globaltimer_ns();
-    if (__syncthreads_or(nan_seen) && tid == 0 && blockIdx.x == 0) atomicOr(p.status, kDevNanLogit);
-    for (int t = warp; t < T; t += kDecWarps) {
-        const float l0 = S.sel_w[t * k];
-        const float ej = lane < k ? expf(S.sel_w[t * k + lane] - l0) : 0.0f;
-        const float ssum = warp_sum(ej);
-        __syncwarp();
-        if (lane < k) {
-            const float wj = ej / ssum;
-            S.sel_w[t * k + lane] = wj;
-            if (blockIdx.x == 0) {
-                p.idx[t * k + lane] = S.sel_e[t * k + lane];
-                p.w[t * k + lane] = wj;
-            }
-        }
-    }
-    __syncthreads();
+    if (tracing && tid == 0) stamp(trace, 10);
+    if (T > 1) __syncthreads();
+    if (tracing && tid == 0) stamp(trace, 12);
 
-    if (tracing && tid == 0) trace[12] = globaltimer_ns();
-    // ---- 2. grouping (warp 0): stable order by expert --------------------------
     if (warp == 0) {
-        int ep = 0x7fffffff, rank = 0;
-        if (lane < P) {
-            ep = S.sel_e[lane];
+        // ---- 2. grouping: stable order of the P pairs by expert --------------------------
+        if (T == 1) {
+            group_single_token(S, k, lane);
+        } else {
+            const int ep = lane < P ? S.sel_e[lane] : 0x7fffffff;
+            uint32_t less = 0, same = 0;
             for (int q = 0; q < P; ++q) {
-                const int eq = S.sel_e[q];
-                rank += (eq < ep) || (eq == ep && q < lane);
+                const int eq = __shfl_sync(0xffffffffu, ep, q);
+                less |= (uint32_t)(eq < ep) << q;
+                same |= (uint32_t)(eq == ep) << q;
             }
-            S.sp[rank] = lane;
-        }
-        // rank r is the first pair of its expert iff no pair of the same expert has
-        // a lower rank, i.e. no q < lane has the same expert
-        bool first = lane < P;
-        if (lane < P)
-            for (int q = 0; q < lane; ++q) first &= S.sel_e[q] != ep;
-        const uint32_t firsts = __ballot_sync(0xffffffffu, first);
-        // distinct index of this pair's expert = distinct experts below it
-        int dless = 0;
-        if (lane < P)
-            for (int q = 0; q < P; ++q) dless += ((firsts >> q) & 1u) && S.sel_e[q] < ep;
-        if (first) {
-            S.dex[dless] = ep;
-            S.dstart[dless] = rank;
-        }
-        if (lane < P) S.pdi[lane] = dless;
-        if (lane == 0) {
-            S.nd = __popc(firsts);
-            S.dstart[__popc(firsts)] = P;
+            const uint32_t below = (1u << lane) - 1u;
+            const int rank = __popc(less) + __popc(same & below);   // sorted position of pair `lane`
+            const bool first = lane < P && (same & below) == 0;     // lowest pair id of its expert
+            const uint32_t firsts = __ballot_sync(0xffffffffu, first);
+            const int dless = __popc(firsts & less);                // distinct index of its expert
+            const int nd = __popc(firsts);
+            const int cnt = __popc(same);                           // pairs of its expert
+            const int nit = first ? (cnt + 7) / 8 : 0;              // down items (<= 8 pairs each)
+            int ibase = 0, n_items = 0;
+            for (int q = 0; q < P; ++q) {
+                const int nq = __shfl_sync(0xffffffffu, nit, q);
+                ibase += ((less >> q) & 1u) ? nq : 0;
+                n_items += nq;
+            }
+            if (lane < P) {
+                S.sp[rank] = lane;
+                S.pdi[lane] = dless;
+            }
+            if (first) {
+                S.dex[dless] = ep;
+                S.dstart[dless] = rank;
+                for (int i = 0; i < nit; ++i) {
+                    S.item_d[ibase + i] = dless;
+                    S.item_r[ibase + i] = rank + 8 * i;
+                    S.item_n[ibase + i] = min(8, cnt - 8 * i);
+                }
+            }
+            if (lane == 0) {
+                S.nd = nd;
+                S.dstart[nd] = P;
+                S.n_items = n_items;
+            }
         }
         __syncwarp();
-        if (lane == 0) {
-            int ni = 0;
-            for (int dd = 0; dd < S.nd; ++dd)
-                for (int r = S.dstart[dd]; r < S.dstart[dd + 1]; r += 8) {
-                    S.item_d[ni] = dd;
-                    S.item_r[ni] = r;
-                    S.item_n[ni] = min(8, S.dstart[dd + 1] - r);
-                    ++ni;
-                }
-            S.n_items = ni;
+        if (tracing && lane == 0) stamp(trace, 9);
+        // the other warps were parked until now, so that the path to the loads had
+        // the SM to itself; the copy issue below is paced by the TMA unit
+        asm volatile("bar.arrive 2, %0;" ::"n"(kDecThreads) : "memory");
+
+        // ---- 3. every weight load of this CTA, issued now ------------------------------
+        {
+            const int nd = S.nd;
+            const int ntu = I / 16;   // gate_up units per expert
+            const int gu0 = S.plan[nd][0], ngu = S.plan[nd][1] - gu0;
+            const int dn0 = S.plan[nd][2], ndn = S.plan[nd][3] - dn0;
+            const uint32_t dn_unit = (uint32_t)nd * dn_blk;
+            for (int u = lane; u < ngu + ndn; u += 32) mbar_expect_tx(mbar0 + 8 * u, u < ngu ? gu_unit : dn_unit);
+            __syncwarp();
+            if (tracing && lane == 0) stamp(trace, 15);
+            const uint32_t wb = smem_addr(wbuf);
+            for (int u = lane; u < ngu; u += 32) {
+                const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
+                bulk_g2s(wb + u * gu_unit, p.gu_blocks + ((size_t)S.dex[dd] * ntu + j) * gu_unit, gu_unit,
+                         mbar0 + 8 * u);
+            }
+            for (int i = lane; i < ndn * nd; i += 32) {
+                const int u = i / nd, dd = i - u * nd, j = dn0 + u;
+                bulk_g2s(wb + ngu * gu_unit + u * dn_unit + dd * dn_blk,
+                         p.dn_blocks + ((size_t)S.dex[dd] * (H / 16) + j) * dn_blk, dn_blk, mbar0 + 8 * (ngu + u));
+            }
         }
-        if (blockIdx.x == 0 && lane < P) {
-            p.sorted_pair[lane] = S.sp[lane];
-            p.pair_row[S.sp[lane]] = lane;
+        if (tracing && lane == 0) stamp(trace, 1);
+
+        // ---- the routing's remaining outputs ------------------------------------------------
+        if (T == 1) warp_softmax(S.sel_w, k, lane);
+        if (blockIdx.x == 0) {
+            for (int q = lane; q < P; q += 32) {
+                p.idx[q] = S.sel_e[q];
+                p.w[q] = S.sel_w[q];
+            }
+        }
+    } else {
+        asm volatile("bar.sync 2, %0;" ::"n"(kDecThreads) : "memory");
+        // ---- 4. (warps 1..) x rows as fp16 pairs with a power-of-two shift per token -----
+        constexpr int XT = kDecThreads - 32;
+        const int xt = tid - 32;
+        if (blockIdx.x == 0) {
+            for (int e = xt; e <= E; e += XT) {
+                int below = 0, eq = 0;
+                for (int q = 0; q < P; ++q) {
+                    below += S.sel_e[q] < e;
+                    eq += S.sel_e[q] == e;
+                }
+                p.offsets[e] = below;
+                if (e < E) p.counts[e] = eq;
+            }
+            for (int r = xt; r < P; r += XT) {
+                p.sorted_pair[r] = S.sp[r];
+                p.pair_row[S.sp[r]] = r;
+            }
+        }
+        // every thread of the group waits (bounded) for x; the group agrees on the
+        // outcome before the named barriers of the staging loop
+        if (p.bulk_inputs && !mbar_wait0(in_bar, p.timeout_ns)) S.abort = 1;
+        asm volatile("bar.sync 1, %0;" ::"n"(XT) : "memory");
+        if (S.abort) {
+            if (xt == 0) atomicOr(p.status, kDevLoadTimeout);
+        } else {
+            for (int t = 0; t < T; ++t) {
+                const uint32_t* xw = p.bulk_inputs ? reinterpret_cast<const uint32_t*>(xr + (size_t)t * H)
+                                                   : reinterpret_cast<const uint32_t*>(p.x + (size_t)t * H);
+                float m = 0.0f;
+                for (int r = xt; r < H / 2; r += XT) {
+                    const uint32_t two = xw[r];
+                    m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32((uint16_t)(two & 0xffff))),
+                                       fabsf(bf16_bits_to_f32((uint16_t)(two >> 16)))));
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) S.wmax[t & 1][warp] = m;
+                asm volatile("bar.sync 1, %0;" ::"n"(XT) : "memory");
+                float mm = 0.0f;
+#pragma unroll
+                for (int w2 = 1; w2 < kDecWarps; ++w2) mm = fmaxf(mm, S.wmax[t & 1][w2]);
+                const int sh = fp16_shift(mm);
+                const float scl = pow2f(-sh);
+                if (xt == 0) S.xshift[t] = sh;
+                for (int r = xt; r < H / 2; r += XT) {
+                    const uint32_t two = xw[r];
+                    xs[t * xrw + r] = f32x2_to_f16x2_rn(bf16_bits_to_f32((uint16_t)(two & 0xffff)) * scl,
+                                                       bf16_bits_to_f32((uint16_t)(two >> 16)) * scl);
+                }
+            }
+        }
+        if (tracing && xt == 0) stamp(trace, 2);
+        if (tid == kDecThreads - 1) {
+            const unsigned tg = (ep_e0 + 1u) ? (ep_e0 + 1u) : 1u;   // 0 is the never-written value
+            S.tag = tg;
+            p.epoch[blockIdx.x] = tg;
         }
     }
     __syncthreads();
@@ -400,77 +585,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     const int gu0 = S.plan[nd][0], gu1 = S.plan[nd][1], dn0 = S.plan[nd][2], dn1 = S.plan[nd][3];
     const int ngu = gu1 - gu0, ndn = dn1 - dn0;
     const uint32_t dn_unit = (uint32_t)nd * dn_blk;
-    if (tracing && tid == 0) trace[9] = globaltimer_ns();
-
-    // ---- 3. warp 0 issues every weight load of this CTA now -------------------------
-    if (warp == 0) {
-        if (lane == 0) {
-            for (int u = 0; u < ngu; ++u) mbar_expect_tx(mbar0 + 8 * u, gu_unit);
-            for (int u = 0; u < ndn; ++u) mbar_expect_tx(mbar0 + 8 * (ngu + u), dn_unit);
-        }
-        __syncwarp();
-        const uint32_t wb = smem_addr(wbuf);
-        for (int u = lane; u < ngu; u += 32) {
-            const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
-            bulk_g2s(wb + u * gu_unit, p.gu_blocks + ((size_t)S.dex[dd] * ntu + j) * gu_unit, gu_unit, mbar0 + 8 * u);
-        }
-        for (int i = lane; i < ndn * nd; i += 32) {
-            const int u = i / nd, dd = i - u * nd, j = dn0 + u;
-            bulk_g2s(wb + ngu * gu_unit + u * dn_unit + dd * dn_blk,
-                     p.dn_blocks + ((size_t)S.dex[dd] * (H / 16) + j) * dn_blk, dn_blk, mbar0 + 8 * (ngu + u));
-        }
-        if (tracing && lane == 0) trace[1] = globaltimer_ns();
+    if (tracing && tid == 0) {
+        trace[32 + 28] = (unsigned long long)ngu;
+        trace[32 + 29] = (unsigned long long)ndn;
     }
-    if (blockIdx.x == 0) {
-        for (int e = tid; e <= E; e += kDecThreads) {
-            int below = 0, eq = 0;
-            for (int q = 0; q < P; ++q) {
-                below += S.sel_e[q] < e;
-                eq += S.sel_e[q] == e;
-            }
-            p.offsets[e] = below;
-            if (e < E) p.counts[e] = eq;
-        }
-    }
-
-    // ---- 4. x rows as fp16 pairs with a power-of-two shift per token (whole CTA) -------
-    for (int t = 0; t < T; ++t) {
-        const uint32_t* xw = reinterpret_cast<const uint32_t*>(xr + (size_t)t * H);
-        float m = 0.0f;
-        for (int r = tid; r < H / 2; r += kDecThreads) {
-            const uint32_t two = xw[r];
-            m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32((uint16_t)(two & 0xffff))),
-                               fabsf(bf16_bits_to_f32((uint16_t)(two >> 16)))));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) S.wmax[warp] = m;
-        __syncthreads();
-        float mm = 0.0f;
-#pragma unroll
-        for (int w2 = 0; w2 < kDecWarps; ++w2) mm = fmaxf(mm, S.wmax[w2]);
-        const int sh = fp16_shift(mm);
-        const float scl = pow2f(-sh);
-        if (tid == 0) S.xshift[t] = sh;
-        for (int r = tid; r < H / 2; r += kDecThreads) {
-            const uint32_t two = xw[r];
-            xs[t * xrw + r] = f32x2_to_f16x2_rn(bf16_bits_to_f32((uint16_t)(two & 0xffff)) * scl,
-                                               bf16_bits_to_f32((uint16_t)(two >> 16)) * scl);
-        }
-        __syncthreads();
-    }
-    if (tracing && tid == 0) trace[2] = globaltimer_ns();
-
-    if (tid == kDecThreads - 1) {
-        const unsigned tg = (ep_e0 + 1u) ? (ep_e0 + 1u) : 1u;
-        S.tag = tg;
-        if (ep_arrived == gridDim.x - 1) {
-            // every CTA has read the epoch: advance it for the next launch
-            atomicExch(p.sync, 0u);
-            st_release_gpu(p.sync + 1, tg);
-        }
-    }
-    __syncthreads();
 
     // ---- 5. gate_up units -> tagged act ------------------------------------------------
     uint32_t off = 0;
@@ -480,6 +598,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             if (tid == 0) { atomicOr(p.status, kDevLoadTimeout); S.abort = 1; }
         }
         __syncthreads();
+        if (tracing && tid == 0 && (u == 0 || u == ngu - 1)) stamp(trace, u == 0 ? 11 : 13);
         if (S.abort) break;
         const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
         const uint8_t* blk0 = wbuf + off;
@@ -489,35 +608,64 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             const int nvalid = min(8, r1 - nb);
             const uint32_t* brow = xs + (g < nvalid ? S.sp[nb + g] / k : T) * xrw;
             float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 2
             for (int q = warp; q < H / 64; q += kDecWarps) quad_mma2(blk0, blk1, H, brow, q, lane, t0, t1);
-            float* rl = red + (warp * 32 + lane) * 8;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                rl[i] = t0[i];
-                rl[4 + i] = t1[i];
+            if (tracing && tid == 0 && u == 0) stamp(trace, 16);
+            // partials of the valid token columns only: red[warp][column][gate 16 | up 16];
+            // lane (g, c) holds rows g, g+8 of columns 2c, 2c+1
+            {
+                const int c = lane & 3;
+                float* rw = red + warp * (8 * 32);
+                if (2 * c < nvalid) {
+                    rw[(2 * c) * 32 + g] = t0[0];
+                    rw[(2 * c) * 32 + g + 8] = t0[2];
+                    rw[(2 * c) * 32 + 16 + g] = t1[0];
+                    rw[(2 * c) * 32 + 24 + g] = t1[2];
+                }
+                if (2 * c + 1 < nvalid) {
+                    rw[(2 * c + 1) * 32 + g] = t0[1];
+                    rw[(2 * c + 1) * 32 + g + 8] = t0[3];
+                    rw[(2 * c + 1) * 32 + 16 + g] = t1[1];
+                    rw[(2 * c + 1) * 32 + 24 + g] = t1[3];
+                }
             }
             __syncthreads();
-            if (tid < 128) {
-                const int n = tid & 15, jt = tid >> 4;
+            if (tracing && tid == 0 && u == 0) stamp(trace, 17);
+            // 4 threads per (column, output): each adds 4 warps' partials, then 2 shuffles
+            {
+                const int qtr = tid & 3, n = (tid >> 2) & 15, jt = tid >> 6;   // jt < 8: all threads take part
+                float gs = 0.0f, us = 0.0f;
                 if (jt < nvalid) {
-                    const int ln = 4 * (n & 7) + (jt >> 1), idx = (n >> 3) * 2 + (jt & 1);
-                    float gs = 0.0f, us = 0.0f;
 #pragma unroll
-                    for (int w2 = 0; w2 < kDecWarps; ++w2) {
-                        gs += red[(w2 * 32 + ln) * 8 + idx];
-                        us += red[(w2 * 32 + ln) * 8 + 4 + idx];
+                    for (int w2 = 0; w2 < kDecWarps / 4; ++w2) {
+                        const float* rw = red + (qtr * (kDecWarps / 4) + w2) * (8 * 32) + jt * 32;
+                        gs += rw[n];
+                        us += rw[16 + n];
                     }
+                }
+                gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+                us += __shfl_xor_sync(0xffffffffu, us, 1);
+                gs += __shfl_xor_sync(0xffffffffu, gs, 2);
+                us += __shfl_xor_sync(0xffffffffu, us, 2);
+                if (jt < nvalid && qtr == 0) {
                     const int pid = S.sp[nb + jt], t = pid / k;
                     const float m = pow2f(S.xshift[t]);
                     const float a = silu_mul(gs * m, us * m);
                     st_volatile_u64(p.act + (size_t)pid * I + 16 * j + n, ((unsigned long long)S.tag << 32) | __float_as_uint(a));
                 }
             }
+            if (tracing && tid == 0 && u == 0) stamp(trace, 18);
             __syncthreads();
+            if (tracing && tid == 0 && u == 0) stamp(trace, 19);
         }
         off += gu_unit;
     }
-    if (tracing && tid == 0) trace[3] = globaltimer_ns();
+    if (tracing && tid == 0) stamp(trace, 3);
+    if (tracing) {
+        // diagnostics only: when the down weights have landed
+        for (int u = 0; u < ndn; ++u) mbar_wait0(mbar0 + 8 * (ngu + u), p.timeout_ns);
+        if (tid == 0) stamp(trace, 14);
+    }
 
     // ---- 6. down units: read act back (tagged), compute, combine ------------------------
     const unsigned tag = S.tag;
@@ -575,13 +723,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         }
         __syncthreads();
     }
-    if (tracing && tid == 0) trace[4] = globaltimer_ns();
+    if (tracing && tid == 0) stamp(trace, 4);
     for (int u = 0; u < ndn; ++u) {
         const uint32_t bar = mbar0 + 8 * (ngu + u);
         if (!mbar_wait0(bar, p.timeout_ns)) {
             if (tid == 0) { atomicOr(p.status, kDevLoadTimeout); S.abort = 1; }
         }
         __syncthreads();
+        if (tracing && tid == 0 && u == 0) stamp(trace, 6);
         const int j = dn0 + u;
         if (!S.abort) {
             // every warp runs a strided share of the 64-k quads for every routed
@@ -620,7 +769,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
 #pragma unroll
                         for (int c2 = 0; c2 < 4; ++c2) dred[((i * 4 + quarter) * 32 + lane) * 4 + c2] = tot[m][c2];
                 }
+                if (tracing && tid == 0 && u == 0 && i0 == 0) stamp(trace, 20);
                 __syncthreads();
+                if (tracing && tid == 0 && u == 0 && i0 == 0) stamp(trace, 7);
                 if (warp < dn) {
                     const int it = i0 + warp;
                     float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -641,6 +792,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                     }
                 }
                 __syncthreads();
+                if (tracing && tid == 0 && u == 0 && i0 == 0) stamp(trace, 21);
             }
         }
         __syncthreads();
@@ -653,7 +805,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         __syncthreads();
         off += dn_unit;
     }
-    if (tracing && tid == 0) trace[5] = globaltimer_ns();
+    if (tracing && tid == 0) stamp(trace, 5);
 
     // ---- 7. never leave with copies in flight --------------------------------------------
     if (S.abort && tid == 0)

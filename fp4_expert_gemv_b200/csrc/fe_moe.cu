@@ -49,7 +49,7 @@ struct fe_moe_s {
     float* o = nullptr;
     unsigned long long* act_ll = nullptr;   // fused decode: tagged act words
     int32_t* plan = nullptr;                // fused decode: work split per nd
-    unsigned* dec_sync = nullptr;           // fused decode: finished CTAs, epoch
+    unsigned* dec_epoch = nullptr;          // fused decode: per-CTA launch counts (act tags)
     unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
     uint32_t* status = nullptr;
     uint16_t* x_stage = nullptr;
@@ -105,14 +105,14 @@ void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
-                    h->act_ll, h->dec_sync, h->plan};
+                    h->act_ll, h->dec_epoch, h->plan};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
     h->pair_row = nullptr; h->active = nullptr; h->n_active = nullptr; h->max_count = nullptr; h->act = nullptr;
     h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
     h->act_ll = nullptr;
-    h->dec_sync = nullptr;
+    h->dec_epoch = nullptr;
     h->plan = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
@@ -143,7 +143,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t decode_weight_bytes(const fe_moe_s* h, int T, int k)
 {
     const int P = T * k;
-    if (P > fe::kDecMaxPairs || h->sm_count <= 0 || h->I > 1024 || h->E > 1024) return 0;
+    if (P > fe::kDecMaxPairs || h->sm_count <= 0 || h->I > 1024 || h->E > fe::kDecMaxE) return 0;
     size_t worst = 0;
     const int nd_max = std::min(h->E, P);
     std::vector<int> gf, df;
@@ -196,12 +196,12 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     dp.idx = h->idx; dp.w = h->w; dp.counts = h->counts; dp.offsets = h->offsets;
     dp.sorted_pair = h->sorted_pair; dp.pair_row = h->pair_row;
     dp.act = h->act_ll;
-    dp.sync = h->dec_sync;
+    dp.epoch = h->dec_epoch;
     dp.trace = h->trace;
     dp.status = h->status;
     dp.timeout_ns = 200ull * 1000 * 1000;
     dp.weight_bytes = (uint32_t)wbytes;
-    dp.bulk_inputs = aligned16(x) && aligned16(logits) && ((size_t)T * h->E) % 4 == 0;
+    dp.bulk_inputs = aligned16(x);   // 2*T*H bytes: a multiple of 16 (H % 64 == 0)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(h->sm_count);
     cfg.blockDim = dim3(fe::kDecThreads);
@@ -352,8 +352,8 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = dmalloc(&h->y_stage, (size_t)max_T * h->H, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->act_ll, (size_t)fe::kDecMaxPairs * h->I, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->act_ll, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
-    if (e == cudaSuccess) e = dmalloc(&h->dec_sync, 2, &acc);
-    if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, 2 * sizeof(unsigned));
+    if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count, &acc);
+    if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned) * (size_t)h->sm_count);
     h->work_bytes = 0;
     if (e == cudaSuccess) e = build_plan_table(h);
     if (e != cudaSuccess) {

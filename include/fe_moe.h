@@ -132,11 +132,16 @@ fe_status fe_moe_set_path(fe_moe_t h, int path);
  * enqueued. */
 fe_status fe_moe_last_forward_info(fe_moe_t h, int* path, int* kernels);
 
-/* Diagnostics: when device_buf (device memory, [number of SMs][16] uint64)
- * is set, the fused decode kernel writes %globaltimer stamps of its phases
- * there (0 start, 8 logits loaded, 9 routed, 10 routing shared, 11 work split,
- * 12 barriers initialised, 1 loads issued, 2 x staged, 3 gate_up done, 4 act
- * read back, 5 down done, 6 end).  NULL switches it off. */
+/* Diagnostics: when device_buf (device memory, [number of SMs][64] uint64)
+ * is set, every CTA of the fused decode kernel writes stamps of its phases
+ * there: slot i (0..31) holds %globaltimer in ns and slot 32 + i the SM's
+ * clock64 at the same point (0 start, 8 previous grid done, 10 routed,
+ * 12 routing shared, 9 grouped, 15 barriers armed, 1 loads issued, 2 x
+ * staged, 11 / 13 first / last gate_up unit landed, 16-19 first gate_up
+ * unit: mma done, partials shared, reduced, done, 3 gate_up done, 14 down
+ * weights landed, 4 act read back, 6 first down unit landed, 20 / 7 / 21
+ * first down unit: mma done, partials shared, reduced, 5 end).  Slots a
+ * CTA does not reach keep their old contents.  NULL switches it off. */
 fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf);
 
 /* Human-readable text of a status code (static storage). */

@@ -226,6 +226,46 @@ def test_edge_cases(torch_cuda, path):
     assert st == fe.FE_OK and bits == 0
 
 
+def fused_routing_cases(E, k, T):
+    """Router logits [T, E] that stress the single-launch kernel's top-k
+    selection: the per-lane maxima threshold (lane l holds experts l, l+32, ...),
+    its fallback when more than 128 keys tie above it, ties, signed zeros and
+    -inf rows."""
+    rng = np.random.default_rng(1000 * E + 10 * k + T)
+    out = []
+    base = rng.standard_normal((T, E)).astype(np.float32)
+    out.append(("random", base))
+    one_lane = base.copy()
+    one_lane[:, ::32] += 10.0          # one lane holds every large key
+    out.append(("one lane holds the top", one_lane))
+    if E >= 512:
+        many = base.copy()
+        for lane in range(16):         # lanes 0..15: all 16 keys above the 16th lane maximum
+            for j in range(E // 32):
+                many[:, lane + 32 * j] = np.float32(100.0 + lane + 0.01 * j)
+        out.append(("more than 128 candidates", many))
+    out.append(("all equal", np.zeros((T, E), np.float32)))
+    ints = rng.integers(-2, 3, (T, E)).astype(np.float32)
+    ints[ints == 0] = np.where(rng.random(int((ints == 0).sum())) < 0.5, np.float32(0.0), np.float32(-0.0))
+    out.append(("integer ties and signed zeros", ints))
+    ninf = np.full((T, E), -np.inf, np.float32)
+    ninf[:, rng.integers(0, E, 2)] = 1.0
+    out.append(("-inf rows with two finite", ninf))
+    return out
+
+
+@pytest.mark.parametrize("E,k,T", [(512, 10, 1), (512, 16, 1), (128, 8, 2), (20, 4, 4), (8, 2, 8)])
+def test_fused_routing_cases(torch_cuda, E, k, T):
+    import fp4_expert_gemv_b200 as fe
+    H, I, seed = 256, 128, 31
+    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=k)
+    osd = harness.OracleSide(E, H, I, seed)
+    x = synth.activations_bf16(70, T, H)
+    for what, lg in fused_routing_cases(E, k, T):
+        run_and_check(gl, osd, x, lg, k, what=f"E={E} k={k} T={T}: {what}")
+        assert gl.layer.last_forward_info()[0] == fe.PATH_FUSED_DECODE, what
+
+
 def test_large_activations_use_power_of_two_shift(torch_cuda):
     E, H, I, seed = 8, 256, 128, 0
     gl = harness.GpuLayer(E, H, I, seed, max_T=4, max_k=2, source="host")
