@@ -42,11 +42,12 @@
 
 namespace fe {
 
-constexpr int kDecThreads = 512;
+constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecMaxPairs = 16;   // T * top_k handled by the fused kernel
 constexpr int kDecMaxItems = 48;   // weight units (mbarriers) per CTA
 constexpr int kDecMaxE = 512;      // experts routed by one warp: 16 logits per lane
+constexpr int kDecQuadsPerWarp = 4;   // gate_up quads whose x fragments a warp keeps in registers
 constexpr int kDecCandCap = 128;   // candidate keys per routing warp (in the gate_up partials' space)
 constexpr uint32_t kDevBarrierTimeout = 0x4;
 constexpr uint32_t kDevLoadTimeout = 0x8;
@@ -567,8 +568,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 if (xt == 0) S.xshift[t] = sh;
                 for (int r = xt; r < H / 2; r += XT) {
                     const uint32_t two = xw[r];
-                    xs[t * xrw + r] = f32x2_to_f16x2_rn(bf16_bits_to_f32((uint16_t)(two & 0xffff)) * scl,
-                                                       bf16_bits_to_f32((uint16_t)(two >> 16)) * scl);
+                    xs[t * xrw + bfrag_word(r)] = f32x2_to_f16x2_rn(bf16_bits_to_f32((uint16_t)(two & 0xffff)) * scl,
+                                                                   bf16_bits_to_f32((uint16_t)(two >> 16)) * scl);
                 }
             }
         }
@@ -591,74 +592,106 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     }
 
     // ---- 5. gate_up units -> tagged act ------------------------------------------------
+    // Warp w runs quads w, w + W, ... (W = warps) of every unit.  Its x fragments
+    // for those quads stay in registers while the n-block's rows stay the same
+    // (always, for one token): the inner loop then reads only weights.
     uint32_t off = 0;
-    for (int u = 0; u < ngu; ++u) {
-        const uint32_t bar = mbar0 + 8 * u;
-        if (!mbar_wait0(bar, p.timeout_ns)) {
-            if (tid == 0) { atomicOr(p.status, kDevLoadTimeout); S.abort = 1; }
-        }
-        __syncthreads();
-        if (tracing && tid == 0 && (u == 0 || u == ngu - 1)) stamp(trace, u == 0 ? 11 : 13);
-        if (S.abort) break;
-        const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
-        const uint8_t* blk0 = wbuf + off;
-        const uint8_t* blk1 = blk0 + block_bytes(H);
-        const int r0 = S.dstart[dd], r1 = S.dstart[dd + 1];
-        for (int nb = r0; nb < r1; nb += 8) {
-            const int nvalid = min(8, r1 - nb);
-            const uint32_t* brow = xs + (g < nvalid ? S.sp[nb + g] / k : T) * xrw;
-            float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 2
-            for (int q = warp; q < H / 64; q += kDecWarps) quad_mma2(blk0, blk1, H, brow, q, lane, t0, t1);
-            if (tracing && tid == 0 && u == 0) stamp(trace, 16);
-            // partials of the valid token columns only: red[warp][column][gate 16 | up 16];
-            // lane (g, c) holds rows g, g+8 of columns 2c, 2c+1
-            {
-                const int c = lane & 3;
-                float* rw = red + warp * (8 * 32);
-                if (2 * c < nvalid) {
-                    rw[(2 * c) * 32 + g] = t0[0];
-                    rw[(2 * c) * 32 + g + 8] = t0[2];
-                    rw[(2 * c) * 32 + 16 + g] = t1[0];
-                    rw[(2 * c) * 32 + 24 + g] = t1[2];
-                }
-                if (2 * c + 1 < nvalid) {
-                    rw[(2 * c + 1) * 32 + g] = t0[1];
-                    rw[(2 * c + 1) * 32 + g + 8] = t0[3];
-                    rw[(2 * c + 1) * 32 + 16 + g] = t1[1];
-                    rw[(2 * c + 1) * 32 + 24 + g] = t1[3];
-                }
+    {
+        const int nq = H / 64;
+        constexpr int QPW = kDecQuadsPerWarp;
+        const int npass = (nq + QPW * kDecWarps - 1) / (QPW * kDecWarps);
+        uint32_t bx[QPW][8];
+        int bkey = -1;
+        for (int u = 0; u < ngu; ++u) {
+            if (!mbar_wait0(mbar0 + 8 * u, p.timeout_ns)) {
+                S.abort = 1;
+                atomicOr(p.status, kDevLoadTimeout);
             }
-            __syncthreads();
-            if (tracing && tid == 0 && u == 0) stamp(trace, 17);
-            // 4 threads per (column, output): each adds 4 warps' partials, then 2 shuffles
-            {
-                const int qtr = tid & 3, n = (tid >> 2) & 15, jt = tid >> 6;   // jt < 8: all threads take part
-                float gs = 0.0f, us = 0.0f;
-                if (jt < nvalid) {
+            if (tracing && tid == 0 && (u == 0 || u == ngu - 1)) stamp(trace, u == 0 ? 11 : 13);
+            const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
+            const uint8_t* blk0 = wbuf + off;
+            const uint8_t* blk1 = blk0 + block_bytes(H);
+            const int r0 = S.dstart[dd], r1 = S.dstart[dd + 1];
+            bool stop = false;
+            for (int nb = r0; nb < r1 && !stop; nb += 8) {
+                const int nvalid = min(8, r1 - nb);
+                const int key = T == 1 ? 0 : (dd << 8) + (nb - r0);
+                const uint32_t* brow = xs + (g < nvalid ? S.sp[nb + g] / k : T) * xrw;
+                float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int pass = 0; pass < npass; ++pass) {
+                    const int qbase = pass * QPW * kDecWarps + warp;
+                    // quads past nq (H not a multiple of 64 QPW W) repeat quad qbase with a
+                    // zero B, so the unrolled body has no branches between its quads
+                    if (key != bkey || npass > 1) {
 #pragma unroll
-                    for (int w2 = 0; w2 < kDecWarps / 4; ++w2) {
-                        const float* rw = red + (qtr * (kDecWarps / 4) + w2) * (8 * 32) + jt * 32;
-                        gs += rw[n];
-                        us += rw[16 + n];
+                        for (int i = 0; i < QPW; ++i) {
+                            const bool ok = qbase + kDecWarps * i < nq;
+                            load_bfrag(ok ? brow : xs + T * xrw, ok ? qbase + kDecWarps * i : 0, lane, bx[i]);
+                        }
+                        bkey = key;
+                    }
+                    if (qbase < nq) {
+#pragma unroll
+                        for (int i = 0; i < QPW; ++i) {
+                            const int q = qbase + kDecWarps * i < nq ? qbase + kDecWarps * i : qbase;
+                            quad_mma2_b(blk0, blk1, H, bx[i], q, lane, t0, t1);
+                        }
                     }
                 }
-                gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-                us += __shfl_xor_sync(0xffffffffu, us, 1);
-                gs += __shfl_xor_sync(0xffffffffu, gs, 2);
-                us += __shfl_xor_sync(0xffffffffu, us, 2);
-                if (jt < nvalid && qtr == 0) {
-                    const int pid = S.sp[nb + jt], t = pid / k;
-                    const float m = pow2f(S.xshift[t]);
-                    const float a = silu_mul(gs * m, us * m);
-                    st_volatile_u64(p.act + (size_t)pid * I + 16 * j + n, ((unsigned long long)S.tag << 32) | __float_as_uint(a));
+                if (tracing && tid == 0 && u == 0) stamp(trace, 16);
+                // partials of the valid token columns only: red[warp][column][gate 16 | up 16];
+                // lane (g, c) holds rows g, g+8 of columns 2c, 2c+1
+                {
+                    const int c = lane & 3;
+                    float* rw = red + warp * (8 * 32);
+                    if (2 * c < nvalid) {
+                        rw[(2 * c) * 32 + g] = t0[0];
+                        rw[(2 * c) * 32 + g + 8] = t0[2];
+                        rw[(2 * c) * 32 + 16 + g] = t1[0];
+                        rw[(2 * c) * 32 + 24 + g] = t1[2];
+                    }
+                    if (2 * c + 1 < nvalid) {
+                        rw[(2 * c + 1) * 32 + g] = t0[1];
+                        rw[(2 * c + 1) * 32 + g + 8] = t0[3];
+                        rw[(2 * c + 1) * 32 + 16 + g] = t1[1];
+                        rw[(2 * c + 1) * 32 + 24 + g] = t1[3];
+                    }
                 }
+                __syncthreads();
+                if (tracing && tid == 0 && u == 0) stamp(trace, 17);
+                if (S.abort) {
+                    stop = true;
+                    continue;
+                }
+                // 2 threads per (column, output): each adds half the warps' partials, then 1 shuffle
+                {
+                    const int half = tid & 1, n = (tid >> 1) & 15, jt = tid >> 5;   // jt < 8
+                    float gs = 0.0f, us = 0.0f;
+                    if (jt < nvalid) {
+#pragma unroll
+                        for (int w2 = 0; w2 < kDecWarps / 2; ++w2) {
+                            const float* rw = red + (half * (kDecWarps / 2) + w2) * (8 * 32) + jt * 32;
+                            gs += rw[n];
+                            us += rw[16 + n];
+                        }
+                    }
+                    gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+                    us += __shfl_xor_sync(0xffffffffu, us, 1);
+                    if (jt < nvalid && half == 0) {
+                        const int pid = S.sp[nb + jt], t = pid / k;
+                        const float m = pow2f(S.xshift[t]);
+                        const float a = silu_mul(gs * m, us * m);
+                        st_volatile_u64(p.act + (size_t)pid * I + 16 * j + n,
+                                        ((unsigned long long)S.tag << 32) | __float_as_uint(a));
+                    }
+                }
+                if (tracing && tid == 0 && u == 0) stamp(trace, 18);
+                __syncthreads();
+                if (tracing && tid == 0 && u == 0) stamp(trace, 19);
             }
-            if (tracing && tid == 0 && u == 0) stamp(trace, 18);
-            __syncthreads();
-            if (tracing && tid == 0 && u == 0) stamp(trace, 19);
+            if (stop) break;
+            off += gu_unit;
         }
-        off += gu_unit;
     }
     if (tracing && tid == 0) stamp(trace, 3);
     if (tracing) {
@@ -668,6 +701,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     }
 
     // ---- 6. down units: read act back (tagged), compute, combine ------------------------
+    off = (uint32_t)ngu * gu_unit;
     const unsigned tag = S.tag;
     if (ndn > 0 && !S.abort) {
         // warp pp stages pair pp: up to 16 chunks of two tagged words per lane, all
@@ -717,8 +751,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;
                 if (2 * r < I)
-                    as[pp * arw + r] = f32x2_to_f16x2_rn(__uint_as_float((uint32_t)a0[i]) * scl,
-                                                        __uint_as_float((uint32_t)a1[i]) * scl);
+                    as[pp * arw + bfrag_word(r)] = f32x2_to_f16x2_rn(__uint_as_float((uint32_t)a0[i]) * scl,
+                                                                    __uint_as_float((uint32_t)a1[i]) * scl);
             }
         }
         __syncthreads();
@@ -750,17 +784,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 for (int m = 0; m < TPW; ++m)
 #pragma unroll
                     for (int c2 = 0; c2 < 4; ++c2) tot[m][c2] = 0.0f;
-                for (int q = qa; q < qb; ++q) {
+                // the tasks' B rows and weight blocks, resolved once; tasks past the last
+                // item redo item i0 and are not stored, so the body has no branches
+                const uint32_t* brow[TPW];
+                const uint8_t* dblk[TPW];
 #pragma unroll
-                    for (int m = 0; m < TPW; ++m) {
-                        const int i = (warp >> 2) + (kDecWarps / 4) * m;
-                        if (i < dn) {
-                            const int it = i0 + i;
-                            const int r0 = S.item_r[it], nvalid = S.item_n[it];
-                            const uint32_t* brow = as + (g < nvalid ? S.sp[r0 + g] : P) * arw;
-                            quad_mma(wbuf + off + S.item_d[it] * dn_blk, I, brow, q, lane, tot[m]);
-                        }
-                    }
+                for (int m = 0; m < TPW; ++m) {
+                    const int i = (warp >> 2) + (kDecWarps / 4) * m;
+                    const int it = i0 + (i < dn ? i : 0);
+                    const int r0 = S.item_r[it], nvalid = S.item_n[it];
+                    brow[m] = as + (g < nvalid ? S.sp[r0 + g] : P) * arw;
+                    dblk[m] = wbuf + off + S.item_d[it] * dn_blk;
+                }
+                for (int q = qa; q < qb; ++q) {
+                    uint32_t b[TPW][8];
+#pragma unroll
+                    for (int m = 0; m < TPW; ++m) load_bfrag(brow[m], q, lane, b[m]);
+#pragma unroll
+                    for (int m = 0; m < TPW; ++m) quad_mma_b(dblk[m], I, b[m], q, lane, tot[m]);
                 }
 #pragma unroll
                 for (int m = 0; m < TPW; ++m) {

@@ -101,6 +101,87 @@ FE_DEV void quad_mma2(const uint8_t* blk0, const uint8_t* blk1, int K, const uin
     }
 }
 
+// ---- B operands held in registers --------------------------------------------
+// A staged row in "fragment order": the 8 words lane (g, t) feeds to the 4
+// k-steps of quad q (k-pairs 8(4q+s)+t and 8(4q+s)+t+4, s = 0..3) sit
+// together at q*32 + t*8 + 2s + {0, 1}, so a quad's B fragments are two
+// 16-byte loads.  Row strides stay K/2 + 4 words (4 banks apart per row).
+__host__ __device__ inline uint32_t bfrag_word(uint32_t kp)
+{
+    return (kp & ~31u) | ((kp & 3u) << 3) | (((kp >> 3) & 3u) << 1) | ((kp >> 2) & 1u);
+}
+
+FE_DEV void load_bfrag(const uint32_t* row, int q, int lane, uint32_t (&b)[8])
+{
+    const uint4 lo = *reinterpret_cast<const uint4*>(row + q * 32 + (lane & 3) * 8);
+    const uint4 hi = *reinterpret_cast<const uint4*>(row + q * 32 + (lane & 3) * 8 + 4);
+    b[0] = lo.x; b[1] = lo.y; b[2] = lo.z; b[3] = lo.w;
+    b[4] = hi.x; b[5] = hi.y; b[6] = hi.z; b[7] = hi.w;
+}
+
+// quad_mma / quad_mma2 with the quad's B fragments in registers (b[2s], b[2s+1]
+// for k-step s).
+FE_DEV void quad_mma_b(const uint8_t* blk, int K, const uint32_t (&b)[8], int q, int lane, float (&tot)[4])
+{
+    const int g = lane >> 2;
+    const uint4 cw = *reinterpret_cast<const uint4*>(blk + 512 * q + 16 * lane);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+        float dg[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ss = 0; ss < 2; ++ss) {
+            const int s = 2 * gi + ss;
+            uint32_t a[4];
+            e2m1x8_to_f16x2x4(words[s], a);
+            mma16816(dg, a, b[2 * s], b[2 * s + 1]);
+        }
+        const uint32_t sw = *reinterpret_cast<const uint32_t*>(blk + 8 * K + 4 * ((2 * q + gi) * 8 + g));
+        const float slo = __uint_as_float(sw << 16), shi = __uint_as_float(sw & 0xffff0000u);
+        tot[0] = fmaf(dg[0], slo, tot[0]);
+        tot[1] = fmaf(dg[1], slo, tot[1]);
+        tot[2] = fmaf(dg[2], shi, tot[2]);
+        tot[3] = fmaf(dg[3], shi, tot[3]);
+    }
+}
+
+FE_DEV void quad_mma2_b(const uint8_t* blk0, const uint8_t* blk1, int K, const uint32_t (&b)[8], int q, int lane,
+                        float (&tot0)[4], float (&tot1)[4])
+{
+    const int g = lane >> 2;
+    const uint4 c0 = *reinterpret_cast<const uint4*>(blk0 + 512 * q + 16 * lane);
+    const uint4 c1 = *reinterpret_cast<const uint4*>(blk1 + 512 * q + 16 * lane);
+    const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w};
+    const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+        float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ss = 0; ss < 2; ++ss) {
+            const int s = 2 * gi + ss;
+            uint32_t a[4];
+            e2m1x8_to_f16x2x4(w0[s], a);
+            mma16816(d0, a, b[2 * s], b[2 * s + 1]);
+            e2m1x8_to_f16x2x4(w1[s], a);
+            mma16816(d1, a, b[2 * s], b[2 * s + 1]);
+        }
+        const int wo = 4 * ((2 * q + gi) * 8 + g);
+        const uint32_t s0 = *reinterpret_cast<const uint32_t*>(blk0 + 8 * K + wo);
+        const uint32_t s1 = *reinterpret_cast<const uint32_t*>(blk1 + 8 * K + wo);
+        const float s0l = __uint_as_float(s0 << 16), s0h = __uint_as_float(s0 & 0xffff0000u);
+        const float s1l = __uint_as_float(s1 << 16), s1h = __uint_as_float(s1 & 0xffff0000u);
+        tot0[0] = fmaf(d0[0], s0l, tot0[0]);
+        tot0[1] = fmaf(d0[1], s0l, tot0[1]);
+        tot0[2] = fmaf(d0[2], s0h, tot0[2]);
+        tot0[3] = fmaf(d0[3], s0h, tot0[3]);
+        tot1[0] = fmaf(d1[0], s1l, tot1[0]);
+        tot1[1] = fmaf(d1[1], s1l, tot1[1]);
+        tot1[2] = fmaf(d1[2], s1h, tot1[2]);
+        tot1[3] = fmaf(d1[3], s1h, tot1[3]);
+    }
+}
+
 // Power-of-two shift s >= 0 with m * 2^-s < 2^15 (m = max |v| of a row), so
 // that a row staged as fp16 cannot overflow.
 FE_DEV int fp16_shift(float m)
