@@ -152,18 +152,22 @@ FE_DEV void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar
 // Phase stamp i of the optional trace: %globaltimer and the SM's cycle counter.
 FE_DEV void stamp(unsigned long long* trace, int i)
 {
+    asm volatile("" ::: "memory");
     trace[i] = globaltimer_ns();
     trace[32 + i] = (unsigned long long)clock64();
+    asm volatile("" ::: "memory");
 }
 
-FE_DEV void st_volatile_u64(unsigned long long* p, unsigned long long v)
+// Tagged act words: device-scope relaxed accesses (each 64-bit word is
+// single-copy atomic, so a reader sees either the old tag or the new value).
+FE_DEV void st_relaxed_u64(unsigned long long* p, unsigned long long v)
 {
-    asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-FE_DEV void ld_volatile_2u64(const unsigned long long* p, unsigned long long& a, unsigned long long& b)
+FE_DEV void ld_relaxed_2u64(const unsigned long long* p, unsigned long long& a, unsigned long long& b)
 {
-    asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
 
 // ---- routing ---------------------------------------------------------------------
@@ -406,6 +410,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     for (int i = tid; i < arw; i += kDecThreads) as[P * arw + i] = 0u;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     if (tracing && tid == 0) stamp(trace, 8);
     if (warp == 1 && lane == 16 && p.bulk_inputs) {
         const uint32_t xb = 2u * T * H;
@@ -423,23 +428,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(red) + warp * cap;
 
     // ---- 1. routing: warp t selects the top-k logits of token t ----------------------
-    // With T = 1, warp 0 routes and goes straight on to the loads (the softmax
-    // and the published routing come after them); with T > 1 every token's
-    // warp also takes its softmax, then the CTA meets before the grouping.
+    // With T = 1, warp 0 routes and hands the selection to warp 1, which groups
+    // and issues the loads (a warp fresh from the divergent selection code ran
+    // the short serial steps after it several times slower); the softmax and the
+    // published routing come after.  With T > 1 every token's warp also takes its
+    // softmax, then the CTA meets before the grouping.
     if (warp < nroute) {
         for (int t = warp; t < T; t += kDecWarps) {
             const bool nan = warp_route(p.logits + (size_t)t * E, E, k, lane, cand, cap, S.sel_e + t * k, S.sel_w + t * k);
             if (nan && lane == 0 && blockIdx.x == 0) atomicOr(p.status, kDevNanLogit);
             if (T > 1) warp_softmax(S.sel_w + t * k, k, lane);
         }
+        if (T == 1) asm volatile("bar.arrive 3, 64;" ::: "memory");
     }
     if (tracing && tid == 0) stamp(trace, 10);
     if (T > 1) __syncthreads();
     if (tracing && tid == 0) stamp(trace, 12);
 
-    if (warp == 0) {
+    if (warp == 1) {
         // ---- 2. grouping: stable order of the P pairs by expert --------------------------
         if (T == 1) {
+            asm volatile("bar.sync 3, 64;" ::: "memory");
             group_single_token(S, k, lane);
         } else {
             const int ep = lane < P ? S.sel_e[lane] : 0x7fffffff;
@@ -484,9 +493,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         }
         __syncwarp();
         if (tracing && lane == 0) stamp(trace, 9);
-        // the other warps were parked until now, so that the path to the loads had
+        // the staging warps were parked until now, so that the path to the loads had
         // the SM to itself; the copy issue below is paced by the TMA unit
-        asm volatile("bar.arrive 2, %0;" ::"n"(kDecThreads) : "memory");
+        asm volatile("bar.arrive 2, %0;" ::"n"(kDecThreads - 32) : "memory");
 
         // ---- 3. every weight load of this CTA, issued now ------------------------------
         {
@@ -511,7 +520,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             }
         }
         if (tracing && lane == 0) stamp(trace, 1);
-
+    } else if (warp == 0) {
         // ---- the routing's remaining outputs ------------------------------------------------
         if (T == 1) warp_softmax(S.sel_w, k, lane);
         if (blockIdx.x == 0) {
@@ -521,10 +530,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             }
         }
     } else {
-        asm volatile("bar.sync 2, %0;" ::"n"(kDecThreads) : "memory");
-        // ---- 4. (warps 1..) x rows as fp16 pairs with a power-of-two shift per token -----
-        constexpr int XT = kDecThreads - 32;
-        const int xt = tid - 32;
+        asm volatile("bar.sync 2, %0;" ::"n"(kDecThreads - 32) : "memory");
+        // ---- 4. (warps 2..) x rows as fp16 pairs with a power-of-two shift per token -----
+        constexpr int XT = kDecThreads - 64;
+        const int xt = tid - 64;
         if (blockIdx.x == 0) {
             for (int e = xt; e <= E; e += XT) {
                 int below = 0, eq = 0;
@@ -562,7 +571,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 asm volatile("bar.sync 1, %0;" ::"n"(XT) : "memory");
                 float mm = 0.0f;
 #pragma unroll
-                for (int w2 = 1; w2 < kDecWarps; ++w2) mm = fmaxf(mm, S.wmax[t & 1][w2]);
+                for (int w2 = 2; w2 < kDecWarps; ++w2) mm = fmaxf(mm, S.wmax[t & 1][w2]);
                 const int sh = fp16_shift(mm);
                 const float scl = pow2f(-sh);
                 if (xt == 0) S.xshift[t] = sh;
@@ -608,6 +617,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 atomicOr(p.status, kDevLoadTimeout);
             }
             if (tracing && tid == 0 && (u == 0 || u == ngu - 1)) stamp(trace, u == 0 ? 11 : 13);
+            if (tracing && tid == 0 && u == 1) stamp(trace, 24);
             const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
             const uint8_t* blk0 = wbuf + off;
             const uint8_t* blk1 = blk0 + block_bytes(H);
@@ -638,7 +648,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                         }
                     }
                 }
-                if (tracing && tid == 0 && u == 0) stamp(trace, 16);
+                if (tracing && tid == 0 && u < 2) stamp(trace, u == 0 ? 16 : 25);
                 // partials of the valid token columns only: red[warp][column][gate 16 | up 16];
                 // lane (g, c) holds rows g, g+8 of columns 2c, 2c+1
                 {
@@ -681,7 +691,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                         const int pid = S.sp[nb + jt], t = pid / k;
                         const float m = pow2f(S.xshift[t]);
                         const float a = silu_mul(gs * m, us * m);
-                        st_volatile_u64(p.act + (size_t)pid * I + 16 * j + n,
+                        st_relaxed_u64(p.act + (size_t)pid * I + 16 * j + n,
                                         ((unsigned long long)S.tag << 32) | __float_as_uint(a));
                     }
                 }
@@ -715,7 +725,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 const int r = lane + 32 * i;
                 a0[i] = a1[i] = 0ull;
                 if (2 * r < I) {
-                    ld_volatile_2u64(src + 2 * r, a0[i], a1[i]);
+                    ld_relaxed_2u64(src + 2 * r, a0[i], a1[i]);
                     if ((unsigned)(a0[i] >> 32) != tag || (unsigned)(a1[i] >> 32) != tag) pending |= 1u << i;
                 }
             }
@@ -723,11 +733,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 const unsigned long long t0 = globaltimer_ns();
                 bool late = false;
                 while (__any_sync(0xffffffffu, pending != 0) && !late) {
-                    __nanosleep(100);
+                    __nanosleep(64);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         if ((pending >> i) & 1u) {
-                            ld_volatile_2u64(src + 2 * (lane + 32 * i), a0[i], a1[i]);
+                            ld_relaxed_2u64(src + 2 * (lane + 32 * i), a0[i], a1[i]);
                             if ((unsigned)(a0[i] >> 32) == tag && (unsigned)(a1[i] >> 32) == tag) pending &= ~(1u << i);
                         }
                     }
@@ -747,6 +757,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             const int sh = fp16_shift(m);
             const float scl = pow2f(-sh);
             if (lane == 0) S.ashift[pp] = sh;
+            if (tracing && lane == 0 && pp == 0) stamp(trace, 26);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;
