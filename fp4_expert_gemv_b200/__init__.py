@@ -26,6 +26,9 @@ FE_ERR_CUDA = -6
 FE_ERR_DEVICE_STATUS = -7
 FE_DEVICE_BAD_EXPERT = 0x1
 FE_DEVICE_NAN_LOGIT = 0x2
+FE_DEVICE_EXCHANGE_TIMEOUT = 0x4
+FE_DEVICE_LOAD_TIMEOUT = 0x8
+FE_DEVICE_TC_TIMEOUT = 0x10
 
 PATH_AUTO, PATH_GEMV, PATH_TCGEN05, PATH_FUSED_DECODE = 0, 1, 2, 3
 

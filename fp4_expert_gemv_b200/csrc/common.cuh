@@ -17,6 +17,7 @@ namespace fe {
 // Device status bits (same values as the public FE_DEVICE_* macros).
 constexpr uint32_t kDevBadExpert = 0x1;
 constexpr uint32_t kDevNanLogit = 0x2;
+constexpr uint32_t kDevTcTimeout = 0x10;   // a tensor-core tile gave up waiting for its MMAs
 
 // ---------------------------------------------------------------------------
 // E2M1 -> f16x2.  One byte holds two codes, the low nibble for the even k.

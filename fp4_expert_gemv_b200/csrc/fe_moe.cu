@@ -18,6 +18,7 @@
 #include "gmma.cuh"
 #include "pack.cuh"
 #include "route.cuh"
+#include "tcgen05.cuh"
 
 namespace fe_host {
 void pack(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales);
@@ -51,6 +52,14 @@ struct fe_moe_s {
     int32_t* plan = nullptr;                // fused decode: work split per nd
     unsigned* dec_epoch = nullptr;          // fused decode: per-CTA launch counts (act tags)
     unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
+    // tensor-core path (tcgen05.cuh)
+    bool tc_scales_ok = false;              // every group scale in the exact-f16 range
+    uint16_t* tc_x = nullptr;               // x rows as f16 [max_T][H]
+    int32_t* tc_xshift = nullptr;           // [max_T]
+    uint16_t* tc_act = nullptr;             // act rows as f16 [P][I], by sorted position
+    int32_t* tc_ashift = nullptr;           // [P]
+    int32_t* tc_tiles = nullptr;            // [max tiles][3]
+    int32_t* tc_ntiles = nullptr;           // [1]
     uint32_t* status = nullptr;
     uint16_t* x_stage = nullptr;
     float* logits_stage = nullptr;
@@ -105,7 +114,8 @@ void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
-                    h->act_ll, h->dec_epoch, h->plan};
+                    h->act_ll, h->dec_epoch, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
+                    h->tc_tiles, h->tc_ntiles};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
@@ -114,6 +124,8 @@ void free_workspace(fe_moe_s* h)
     h->act_ll = nullptr;
     h->dec_epoch = nullptr;
     h->plan = nullptr;
+    h->tc_x = nullptr; h->tc_xshift = nullptr; h->tc_act = nullptr; h->tc_ashift = nullptr;
+    h->tc_tiles = nullptr; h->tc_ntiles = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -220,6 +232,19 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
 // outside any stream capture).  Function attributes are process-wide, so a
 // handle of another shape must never lower the limit below what this
 // handle's launches request.
+// Shapes the tensor-core tiles cover: 128 act columns (64 gate + 64 up pairs of
+// rows) and 256 output columns per tile.
+bool tc_shape_ok(const fe_moe_s* h) { return h->I % 128 == 0 && h->H % 256 == 0; }
+
+// Token-expert pairs from which the automatic path choice takes the tensor
+// cores (below it the grouped mma.sync kernels keep the weights' single pass).
+constexpr int kTcAutoPairs = 4096;
+
+size_t tc_max_tiles(const fe_moe_s* h, size_t P)
+{
+    return (P + fe::kTcN - 1) / fe::kTcN + std::min((size_t)h->E, P);
+}
+
 cudaError_t configure_kernels(const fe_moe_s* h)
 {
     const int optin = h->smem_optin;
@@ -227,6 +252,10 @@ cudaError_t configure_kernels(const fe_moe_s* h)
     if (e == cudaSuccess) e = cudaFuncSetAttribute(fe::gmma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(fe::gmma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(fe::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fe::tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fe::tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     return e;
 }
 
@@ -261,6 +290,48 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
     gp.act_in = h->act;
     gp.out = h->o;
     fe::gmma_kernel<false><<<max_active * gp.n_units, fe::kGmmaThreads, fe::gmma_smem_bytes(false, h->I), s>>>(gp);
+    FE_CUDA_TRY(cudaGetLastError());
+    return FE_OK;
+}
+
+// Large-T path on the tensor cores: tile list, x rows to f16, gate_up tiles
+// (SwiGLU into act), act rows to f16, down tiles (into o).  The routing and
+// grouping ran before; the ordered combine runs after.
+fe_status tcgen05_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s)
+{
+    const int P = T * k;
+    const int max_tiles = (int)tc_max_tiles(h, (size_t)P);
+    fe::tc_tiles_kernel<<<1, 32, 0, s>>>(h->counts, h->offsets, h->E, h->tc_tiles, h->tc_ntiles);
+    fe::tc_rows_to_f16_kernel<true><<<(T + 7) / 8, 256, 0, s>>>(x, T, h->H, h->tc_x, h->tc_xshift);
+    fe::TcParams tp{};
+    tp.tiles = h->tc_tiles;
+    tp.n_tiles = h->tc_ntiles;
+    tp.sorted_pair = h->sorted_pair;
+    tp.top_k = k;
+    tp.status = h->status;
+    tp.timeout_ns = 200ull * 1000 * 1000;
+    tp.trace = h->trace;
+    tp.tile_trace = h->trace ? h->trace + 1024 : nullptr;
+    tp.blocks = h->gu_blocks;
+    tp.K = h->H;
+    tp.blocks_per_expert = 2 * (h->I / 16);
+    tp.bsrc = h->tc_x;
+    tp.bshift = h->tc_xshift;
+    tp.out = h->act;
+    tp.out_ld = h->I;
+    fe::tc_gemm_kernel<true><<<dim3(h->I / 128, max_tiles), fe::kTcThreads, fe::tc_smem_bytes(), s>>>(tp);
+    FE_CUDA_TRY(cudaGetLastError());
+    fe::tc_rows_to_f16_kernel<false><<<(P + 7) / 8, 256, 0, s>>>(h->act, P, h->I, h->tc_act, h->tc_ashift);
+    tp.blocks = h->dn_blocks;
+    tp.K = h->I;
+    tp.blocks_per_expert = h->H / 16;
+    tp.bsrc = h->tc_act;
+    tp.bshift = h->tc_ashift;
+    tp.out = h->o;
+    tp.out_ld = h->H;
+    tp.trace = h->trace ? h->trace + 256 : nullptr;
+    tp.tile_trace = h->trace ? h->trace + 1024 + 4 * (size_t)(h->I / 128) * max_tiles : nullptr;
+    fe::tc_gemm_kernel<false><<<dim3(h->H / fe::kTcM, max_tiles), fe::kTcThreads, fe::tc_smem_bytes(), s>>>(tp);
     FE_CUDA_TRY(cudaGetLastError());
     return FE_OK;
 }
@@ -354,6 +425,14 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = cudaMemset(h->act_ll, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
     if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned) * (size_t)h->sm_count);
+    if (tc_shape_ok(h)) {
+        if (e == cudaSuccess) e = dmalloc(&h->tc_x, (size_t)max_T * h->H, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->tc_xshift, (size_t)max_T, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->tc_act, P * h->I, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->tc_ashift, P, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->tc_tiles, 3 * tc_max_tiles(h, P), &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->tc_ntiles, 1, &acc);
+    }
     h->work_bytes = 0;
     if (e == cudaSuccess) e = build_plan_table(h);
     if (e != cudaSuccess) {
@@ -408,6 +487,21 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
     rp.K = I; rp.N = H; rp.gate_up = 0;
     fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
     FE_CUDA_TRY(cudaGetLastError());
+    // the tensor-core path needs every scale in the range where code x scale is an
+    // exact f16; checked once here (this waits for the stream)
+    h->tc_scales_ok = false;
+    if (tc_shape_ok(h)) {
+        uint32_t* bad = nullptr;
+        FE_CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&bad), sizeof(uint32_t), s));
+        FE_CUDA_TRY(cudaMemsetAsync(bad, 0, sizeof(uint32_t), s));
+        fe::tc_scale_check_kernel<<<296, 256, 0, s>>>(sgs, gu_s, bad);
+        fe::tc_scale_check_kernel<<<296, 256, 0, s>>>(sds, dn_s, bad);
+        uint32_t hbad = 1;
+        FE_CUDA_TRY(cudaMemcpyAsync(&hbad, bad, sizeof(uint32_t), cudaMemcpyDeviceToHost, s));
+        FE_CUDA_TRY(cudaFreeAsync(bad, s));
+        FE_CUDA_TRY(cudaStreamSynchronize(s));
+        h->tc_scales_ok = hbad == 0;
+    }
     if (staging) FE_CUDA_TRY(cudaFreeAsync(staging, s));
     h->loaded = true;
     return FE_OK;
@@ -424,7 +518,8 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     if ((reinterpret_cast<uintptr_t>(x_bf16) & 3u) || (reinterpret_cast<uintptr_t>(y_bf16) & 3u) ||
         (reinterpret_cast<uintptr_t>(router_logits) & 3u))
         return FE_ERR_INVALID_ARG;
-    if (h->path == FE_PATH_TCGEN05) return FE_ERR_UNSUPPORTED;
+    const bool tc_ok = tc_shape_ok(h) && h->tc_scales_ok && h->tc_x != nullptr;
+    if (h->path == FE_PATH_TCGEN05 && !tc_ok) return FE_ERR_UNSUPPORTED;
     DeviceGuard g(h->device);
     if (!g.ok) return FE_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
@@ -454,7 +549,9 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     fe::route_group_kernel<<<1, rthreads, fe::route_smem_bytes(h->E, rthreads), s>>>(rp);
     FE_CUDA_TRY(cudaGetLastError());
 
-    fe_status st = gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
+    const bool use_tc = tc_ok && (h->path == FE_PATH_TCGEN05 || (h->path == FE_PATH_AUTO && P >= kTcAutoPairs));
+    fe_status st = use_tc ? tcgen05_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s)
+                          : gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
     if (st != FE_OK) return st;
 
     dim3 cgrid((h->H / 2 + 255) / 256, T);
@@ -463,8 +560,8 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     FE_CUDA_TRY(cudaGetLastError());
     h->last_T = T;
     h->last_k = top_k;
-    h->last_path = FE_PATH_GEMV;
-    h->last_kernels = 4;
+    h->last_path = use_tc ? FE_PATH_TCGEN05 : FE_PATH_GEMV;
+    h->last_kernels = use_tc ? 8 : 4;
     return FE_OK;
 }
 

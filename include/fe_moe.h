@@ -68,6 +68,9 @@ typedef enum {
 /* Device-side problem bits, reported through fe_moe_get_status. */
 #define FE_DEVICE_BAD_EXPERT 0x1   /* an expert id outside [0, E) reached a kernel */
 #define FE_DEVICE_NAN_LOGIT 0x2    /* a NaN router logit (treated as -inf) */
+#define FE_DEVICE_EXCHANGE_TIMEOUT 0x4  /* single-launch decode: act from other CTAs never arrived */
+#define FE_DEVICE_LOAD_TIMEOUT 0x8      /* a weight copy into shared memory never completed */
+#define FE_DEVICE_TC_TIMEOUT 0x10       /* a tensor-core tile gave up waiting for its MMAs */
 
 /* Create a handle for a layer of E experts, hidden size H and expert
  * intermediate size I on the current CUDA device.  group must be 32; H and I

@@ -112,7 +112,7 @@ def test_tiny_layer_device_packed_equals_host_packed(torch_cuda):
     assert np.array_equal(ya, yb)
 
 
-PATHS = {"auto": 0, "gemv": 1}
+PATHS = {"auto": 0, "gemv": 1, "tc": 2}
 
 
 @pytest.mark.parametrize("path", ["auto", "gemv"])
@@ -183,13 +183,40 @@ def _cached_oracle(E, H, I, seed):
     return _ORACLES[key]
 
 
-def test_prefill_t4096_sampled(torch_cuda):
+@pytest.mark.parametrize("path", ["auto", "tc"])
+def test_prefill_t4096_sampled(torch_cuda, path):
+    import fp4_expert_gemv_b200 as fe
     cfg, seed, x, lg = harness.workload_inputs("prefill_e128_t4096")
     E, H, I, k, T = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"], cfg["T"]
-    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=k)
+    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=k, path=PATHS[path])
     osd = harness.OracleSide(E, H, I, seed)
     run_and_check(gl, osd, x, lg, k, sample=[0, 1, 2047, 4095], what="prefill sampled")
+    if path == "tc":
+        assert gl.layer.last_forward_info()[0] == fe.PATH_TCGEN05
     _LAYERS.clear()
+
+
+def test_tcgen05_tiles(torch_cuda):
+    """Tensor-core tiles: partial tiles, experts without tokens, several
+    tiles for one expert, all tokens on one expert."""
+    import fp4_expert_gemv_b200 as fe
+    E, H, I, seed = 8, 256, 128, 0
+    gl = harness.GpuLayer(E, H, I, seed, max_T=600, max_k=8, source="host", path=fe.PATH_TCGEN05)
+    osd = harness.OracleSide(E, H, I, seed)
+    x = synth.activations_bf16(90, 600, H)
+    lg = synth.router_logits(90, 600, E)
+    run_and_check(gl, osd, x[:5], lg[:5], 1, what="tc T=5 k=1 (most experts empty)")
+    assert gl.layer.last_forward_info()[0] == fe.PATH_TCGEN05
+    run_and_check(gl, osd, x[:40], lg[:40], 2, what="tc T=40 k=2")
+    run_and_check(gl, osd, x[:64], lg[:64], 8, what="tc T=64 k=8 (every expert, 64 rows)")
+    lg_hot = lg.copy()
+    lg_hot[:, 3] += 100.0
+    run_and_check(gl, osd, x, lg_hot, 1, sample=list(range(0, 600, 37)) + [599],
+                  what="tc 600 tokens on one expert: tiles of 256, 256, 88")
+    run_and_check(gl, osd, x[:300], lg[:300], 8, sample=list(range(0, 300, 23)) + [299],
+                  what="tc T=300 k=8 (2400 pairs, ~300 rows per expert)")
+    st, bits = gl.layer.status()
+    assert st == fe.FE_OK and bits == 0
 
 
 @pytest.mark.parametrize("path", ["auto", "gemv"])
@@ -369,10 +396,20 @@ def test_argument_errors(torch_cuda):
         assert fe.fe_moe_forward(h, 16, 16, 1, 2, 16, None) == fe.FE_ERR_INVALID_ARG   # y aliases x
         assert fe.fe_moe_forward(h, 16, 16, -1, 2, 32, None) == fe.FE_ERR_INVALID_ARG
         assert fe.fe_moe_set_path(h, 4) == fe.FE_ERR_INVALID_ARG
-        assert fe.fe_moe_set_path(h, fe.PATH_TCGEN05) == fe.FE_OK
-        assert fe.fe_moe_forward(h, 16, 16, 1, 2, 32, None) == fe.FE_ERR_UNSUPPORTED
         assert fe.fe_moe_set_path(h, fe.PATH_AUTO) == fe.FE_OK
         st, = [fe.fe_moe_get_status(h, None)]
         assert st == fe.FE_OK
     finally:
         fe.fe_moe_destroy(h)
+    # the tensor-core tiles need I % 128 == 0: asking for them on I = 64 is refused
+    # before anything is launched
+    h2 = ctypes.c_void_p()
+    assert fe.fe_moe_create(8, 256, 64, 32, ctypes.byref(h2)) == fe.FE_OK
+    try:
+        assert fe.fe_moe_reserve(h2, 4, 2) == fe.FE_OK
+        z = np.zeros(1 << 20, np.uint8)
+        assert fe.fe_moe_load_packed(h2, z.ctypes.data, z.ctypes.data, z.ctypes.data, z.ctypes.data, 0, None) == 0
+        assert fe.fe_moe_set_path(h2, fe.PATH_TCGEN05) == fe.FE_OK
+        assert fe.fe_moe_forward(h2, 16, 16, 1, 2, 32, None) == fe.FE_ERR_UNSUPPORTED
+    finally:
+        fe.fe_moe_destroy(h2)
