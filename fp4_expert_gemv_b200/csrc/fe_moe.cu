@@ -18,6 +18,7 @@
 #include "gmma.cuh"
 #include "pack.cuh"
 #include "route.cuh"
+#include "route_large.cuh"
 #include "tcgen05.cuh"
 
 namespace fe_host {
@@ -60,6 +61,7 @@ struct fe_moe_s {
     int32_t* tc_ashift = nullptr;           // [P]
     int32_t* tc_tiles = nullptr;            // [max tiles][3]
     int32_t* tc_ntiles = nullptr;           // [1]
+    int32_t* grp_bh = nullptr;              // grouping for many tokens: [P / kGroupChunk + 1][E]
     uint32_t* status = nullptr;
     uint16_t* x_stage = nullptr;
     float* logits_stage = nullptr;
@@ -115,7 +117,7 @@ void free_workspace(fe_moe_s* h)
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
                     h->act_ll, h->dec_epoch, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
-                    h->tc_tiles, h->tc_ntiles};
+                    h->tc_tiles, h->tc_ntiles, h->grp_bh};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
@@ -126,6 +128,7 @@ void free_workspace(fe_moe_s* h)
     h->plan = nullptr;
     h->tc_x = nullptr; h->tc_xshift = nullptr; h->tc_act = nullptr; h->tc_ashift = nullptr;
     h->tc_tiles = nullptr; h->tc_ntiles = nullptr;
+    h->grp_bh = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -240,6 +243,9 @@ bool tc_shape_ok(const fe_moe_s* h) { return h->I % 128 == 0 && h->H % 256 == 0;
 // cores (below it the grouped mma.sync kernels keep the weights' single pass).
 constexpr int kTcAutoPairs = 4096;
 
+// Tokens from which routing and grouping run on the whole GPU.
+constexpr int kRouteLargeTokens = 32;
+
 size_t tc_max_tiles(const fe_moe_s* h, size_t P)
 {
     return (P + fe::kTcN - 1) / fe::kTcN + std::min((size_t)h->E, P);
@@ -290,6 +296,34 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
     gp.act_in = h->act;
     gp.out = h->o;
     fe::gmma_kernel<false><<<max_active * gp.n_units, fe::kGmmaThreads, fe::gmma_smem_bytes(false, h->I), s>>>(gp);
+    FE_CUDA_TRY(cudaGetLastError());
+    return FE_OK;
+}
+
+// Router + grouping outputs (idx, w, counts, offsets, sorted_pair, pair_row,
+// active, n_active, max_count) for the non-fused paths: the single-CTA kernel
+// for a few tokens, the GPU-wide kernels for many.
+fe_status route_and_group(fe_moe_s* h, const float* logits, int T, int k, cudaStream_t s)
+{
+    const int P = T * k;
+    fe::RouteParams rp{};
+    rp.logits = logits; rp.T = T; rp.E = h->E; rp.k = k;
+    rp.idx = h->idx; rp.w = h->w; rp.counts = h->counts; rp.offsets = h->offsets;
+    rp.sorted_pair = h->sorted_pair; rp.pair_row = h->pair_row; rp.active = h->active;
+    rp.n_active = h->n_active; rp.max_count = h->max_count; rp.status = h->status;
+    if (T >= kRouteLargeTokens && fe::route_large_ok(h->E, k)) {
+        const int nblk = (P + fe::kGroupChunk - 1) / fe::kGroupChunk;
+        fe::route_tokens_kernel<<<(T + fe::kRouteWarps - 1) / fe::kRouteWarps, fe::kRouteWarps * 32, 0, s>>>(rp);
+        fe::group_hist_kernel<<<nblk, fe::kGroupThreads, sizeof(int32_t) * h->E, s>>>(h->idx, P, h->E, h->grp_bh);
+        fe::group_scan_kernel<<<1, 1024, 2 * sizeof(int32_t) * h->E, s>>>(h->grp_bh, nblk, h->E, h->counts,
+                                                                          h->offsets, h->active, h->n_active,
+                                                                          h->max_count);
+        fe::group_scatter_kernel<<<nblk, fe::kGroupThreads, sizeof(int32_t) * h->E * (fe::kGroupThreads / 32 + 1),
+                                   s>>>(h->idx, P, h->E, h->grp_bh, h->sorted_pair, h->pair_row, h->status);
+    } else {
+        const int rthreads = std::min(fe::kRouteMaxThreads, std::max(32, roundup32(std::max(P, 32 * T))));
+        fe::route_group_kernel<<<1, rthreads, fe::route_smem_bytes(h->E, rthreads), s>>>(rp);
+    }
     FE_CUDA_TRY(cudaGetLastError());
     return FE_OK;
 }
@@ -425,6 +459,7 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = cudaMemset(h->act_ll, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
     if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned) * (size_t)h->sm_count);
+    if (e == cudaSuccess) e = dmalloc(&h->grp_bh, (P / fe::kGroupChunk + 1) * (size_t)h->E, &acc);
     if (tc_shape_ok(h)) {
         if (e == cudaSuccess) e = dmalloc(&h->tc_x, (size_t)max_T * h->H, &acc);
         if (e == cudaSuccess) e = dmalloc(&h->tc_xshift, (size_t)max_T, &acc);
@@ -540,14 +575,10 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
         if (h->path == FE_PATH_FUSED_DECODE) return FE_ERR_UNSUPPORTED;
     }
 
-    fe::RouteParams rp{};
-    rp.logits = router_logits; rp.T = T; rp.E = h->E; rp.k = top_k;
-    rp.idx = h->idx; rp.w = h->w; rp.counts = h->counts; rp.offsets = h->offsets;
-    rp.sorted_pair = h->sorted_pair; rp.pair_row = h->pair_row; rp.active = h->active;
-    rp.n_active = h->n_active; rp.max_count = h->max_count; rp.status = h->status;
-    const int rthreads = std::min(fe::kRouteMaxThreads, std::max(32, roundup32(std::max(P, 32 * T))));
-    fe::route_group_kernel<<<1, rthreads, fe::route_smem_bytes(h->E, rthreads), s>>>(rp);
-    FE_CUDA_TRY(cudaGetLastError());
+    {
+        const fe_status rs = route_and_group(h, router_logits, T, top_k, s);
+        if (rs != FE_OK) return rs;
+    }
 
     const bool use_tc = tc_ok && (h->path == FE_PATH_TCGEN05 || (h->path == FE_PATH_AUTO && P >= kTcAutoPairs));
     fe_status st = use_tc ? tcgen05_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s)
