@@ -30,7 +30,8 @@
 
 namespace fe {
 
-constexpr int kTcThreads = 128;   // 4 warps; warp 0 also allocates TMEM and issues the MMAs
+constexpr int kTcThreads = 256;   // 8 warps; warp 0 also allocates TMEM and issues the MMAs
+constexpr int kTcWarps = kTcThreads / 32;
 constexpr int kTcM = 256;         // A rows (weight columns) per tile: two 128-row accumulators
 constexpr int kTcN = 256;         // B rows (tokens) per tile
 constexpr int kTcRawStages = 4;   // raw code/scale chunks in flight
@@ -233,11 +234,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // this thread's B rows: chunk column tid & 7 of rows (tid >> 3) + 16 m
-    const uint16_t* brow[16];
+    // this thread's B rows: chunk column tid & 7 of rows (tid >> 3) + RS m
+    constexpr int RS = kTcThreads / 8, NBR = kTcN / RS;
+    const uint16_t* brow[NBR];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-        const int r = (tid >> 3) + 16 * m;
+    for (int m = 0; m < NBR; ++m) {
+        const int r = (tid >> 3) + RS * m;
         const uint16_t* src = p.bsrc;
         if (r < rows) {
             const int pos = pos0 + r;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
     auto load_raw = [&](int q) {
         const uint32_t dst = raw_addr + (q % kTcRawStages) * kTcRawBytes;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < 512 / kTcThreads; ++m) {
             const int c = tid + kTcThreads * m, bi = c >> 5, w16 = c & 31;
             cp_async16(dst + bi * 512 + 16 * w16, blk0 + (size_t)bi * (9 * K) + 512 * q + 16 * w16, 16);
         }
@@ -264,8 +266,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
         const uint32_t dst = b_addr + (q % kTcBStages) * kTcBBytes;
         const int c = tid & 7;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int r = (tid >> 3) + 16 * m;
+        for (int m = 0; m < NBR; ++m) {
+            const int r = (tid >> 3) + RS * m;
             cp_async16(dst + tc_swz(r, c), brow[m] + 64 * q + 8 * c, r < rows ? 16u : 0u);
         }
     };
@@ -293,8 +295,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
             const uint8_t* raw = raw_ring + (i % kTcRawStages) * kTcRawBytes;
             uint8_t* A = a_ring + (i % kTcAStages) * kTcABytes;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int bi = 4 * warp + m;
+            for (int m = 0; m < 16 / kTcWarps; ++m) {
+                const int bi = (16 / kTcWarps) * warp + m;
                 const uint4 cw = *reinterpret_cast<const uint4*>(raw + bi * 512 + 16 * lane);
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
                 const uint32_t* sc = reinterpret_cast<const uint32_t*>(raw + 8192 + bi * 64);
@@ -312,7 +314,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int col = g + 8 * (j & 1);
-                        const int row = GATE_UP ? 32 * (bi >> 1) + 2 * col + (bi & 1) : 16 * bi + col;
+                        // gate_up: unit bi/2 owns rows 32 (bi/2) .. +31, gate columns first, up 16 rows
+                        // later (row & 7 = col & 7: the 8 lanes of a store hit 8 swizzle phases)
+                        const int row = GATE_UP ? 32 * (bi >> 1) + 16 * (bi & 1) + col : 16 * bi + col;
                         const int chunk = 2 * s4 + (j >> 1);
                         __half2 v = *reinterpret_cast<const __half2*>(&h[j]);
                         v = __hmul2(v, s2[s4 >> 1][j & 1]);
@@ -373,27 +377,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
         const int ocol0 = GATE_UP ? (kTcM / 2) * mt : kTcM * mt;
 #pragma unroll 1
         for (int c0 = 0; c0 < nb; c0 += 32) {
-#pragma unroll
-            for (int acc = 0; acc < 2; ++acc) {
-                const int row = 128 * acc + 32 * warp + lane;   // A row of this thread's TMEM lane
+            {
+                // warps 0-3 read accumulator 0, warps 4-7 accumulator 1 (TMEM lanes 32 (warp % 4) ...)
+                const int acc = warp >> 2;
+                const int row = 128 * acc + 32 * (warp & 3) + lane;   // A row of this thread's TMEM lane
                 uint32_t r[32];
-                const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + 256 * acc + c0;
+                const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 256 * acc + c0;
                 tc_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
                 tc_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
                 tc_wait_ld();
                 if (GATE_UP) {
-                    // lane pair (gate, up) of one act column: the even lane takes
-                    // tokens 0-15, the odd lane tokens 16-31
-                    const bool odd = lane & 1;
+                    // lanes l and l + 16 hold gate and up of one act column: the gate lane
+                    // takes tokens 0-15, the up lane tokens 16-31
+                    const bool up = lane & 16;
+                    const int acol = 16 * (row >> 5) + (lane & 15);   // act column within the tile
 #pragma unroll
                     for (int n = 0; n < 16; ++n) {
                         const float lo = __uint_as_float(r[n]), hi = __uint_as_float(r[16 + n]);
-                        const float other = __shfl_xor_sync(0xffffffffu, odd ? lo : hi, 1);   // what the partner needs
-                        const int tn = odd ? 16 + n : n;
-                        const float own = odd ? hi : lo;
-                        const float gv = odd ? other : own, uv = odd ? own : other;
+                        const float other = __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);   // what the partner needs
+                        const int tn = up ? 16 + n : n;
+                        const float own = up ? hi : lo;
+                        const float gv = up ? other : own, uv = up ? own : other;
                         const float m = rmul[c0 + tn];
-                        st[tn * OC + (row >> 1)] = silu_mul(gv * m, uv * m);
+                        st[tn * OC + acol] = silu_mul(gv * m, uv * m);
                     }
                 } else {
 #pragma unroll
