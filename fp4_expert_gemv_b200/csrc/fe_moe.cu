@@ -592,7 +592,8 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     h->last_T = T;
     h->last_k = top_k;
     h->last_path = use_tc ? FE_PATH_TCGEN05 : FE_PATH_GEMV;
-    h->last_kernels = use_tc ? 8 : 4;
+    const bool large_route = T >= kRouteLargeTokens && fe::route_large_ok(h->E, top_k);
+    h->last_kernels = (large_route ? 4 : 1) + (use_tc ? 6 : 2) + 1;   // routing, projections, combine
     return FE_OK;
 }
 
