@@ -37,6 +37,10 @@ KERNEL_NAMES = {1: "grouped mma.sync projections (routing, gate_up, down, combin
                 2: "tensor-core tiles tc_gemm_kernel (gate_up + down) with routing, row conversion and combine",
                 3: "decode_kernel (whole layer, one cooperative launch); per-launch time = step time / layers"}
 PREFILL_METRIC = "MoE-layer prefill tokens/s and tensor-core TFLOP/s at T=4096"
+# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu
+# captures summarised in profiles/ (recaptured whenever that kernel changes)
+TRAFFIC = {"decode_e128_t1": (21385728, "decode_kernel", "profiles/decode_kernel_decode_e128_t1.md"),
+           "prefill_e128_t4096": (345764608, "tc_gemm_kernel gate_up", "profiles/tc_gemm_kernel_prefill_e128_t4096.md")}
 BYTES_PER_EXPERT = lambda H, I: (H // 2) * 2 * I + (H // 32) * 2 * I * 2 + (I // 2) * H + (I // 32) * H * 2  # noqa: E731
 
 
@@ -368,13 +372,16 @@ def run_gpu(args):
         tf = flops_layer * layers / (ms_local / 1e3) / 1e12
         tpeak, tpeak_kind = measured_tensor_peak()
         roofline = {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
-                    "traffic": None, "kernel": KERNEL_NAMES.get(path, str(path)), "peak_kind": tpeak_kind,
+                    "traffic": TRAFFIC.get(workload, (None,))[0], "kernel": KERNEL_NAMES.get(path, str(path)), "peak_kind": tpeak_kind,
                     "algorithmic_flops_per_layer": flops_layer,
                     "frac_of_nominal_fp4_9pflops": tf / 9000.0}
     else:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": None, "kernel": KERNEL_NAMES.get(path, str(path)),
+                    "traffic": TRAFFIC.get(workload, (None,))[0], "kernel": KERNEL_NAMES.get(path, str(path)),
                     "peak_kind": peak_kind, "algorithmic_bytes_per_layer": bytes_layer[0]}
+    if workload in TRAFFIC:
+        roofline["traffic_kernel"] = TRAFFIC[workload][1]
+        roofline["traffic_source"] = TRAFFIC[workload][2]
     line = {
         "metric": PREFILL_METRIC if prefill else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
