@@ -74,8 +74,10 @@ typedef enum {
 
 /* Create a handle for a layer of E experts, hidden size H and expert
  * intermediate size I on the current CUDA device.  group must be 32; H and I
- * must be positive multiples of 32; E in [1, 1024].  Allocates the weight
- * buffers (E * (H*2I + I*H) * 9/16 bytes) but no workspace. */
+ * must be positive multiples of 32 (FE_ERR_INVALID_ARG otherwise) and of 64
+ * (FE_ERR_UNSUPPORTED otherwise: the kernels read K in quads of 64); E in
+ * [1, 1024].  Allocates the weight buffers (E * (H*2I + I*H) * 9/16 bytes) but
+ * no workspace. */
 fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out);
 
 /* Allocate the forward workspace for up to max_T tokens and top_k <= max_top_k.
@@ -87,9 +89,12 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k);
  *   gate_up_codes  uint8 [E][H/2][2I],  gate_up_scales bf16 [E][H/32][2I],
  *   down_codes     uint8 [E][I/2][H],   down_scales    bf16 [E][I/32][H].
  * src_on_device = 1: the four pointers are device memory; 0: host memory.
- * The library re-lays the bytes out into its own device buffers (column tiles
- * for the kernels); the caller's buffers may be freed after the stream has
- * passed this call.  Enqueued on stream; returns after enqueueing. */
+ * The library re-lays the bytes out into its own device buffers (16-column
+ * blocks in tensor-core fragment order); the caller's buffers may be freed
+ * after this call returns.  Work is enqueued on stream; when I % 128 == 0 and
+ * H % 256 == 0 the call then waits for the stream once, to learn whether every
+ * scale allows exact f16 weights (nonzero |scale| in [2^-13, 2^13)), which the
+ * tensor-core path needs. */
 fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
                              const uint8_t* down_codes, const uint16_t* down_scales, int src_on_device,
                              fe_stream_t stream);
@@ -123,8 +128,9 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
 
 /* Compute paths of fe_moe_forward. */
 #define FE_PATH_AUTO 0          /* chosen per call from T, top_k and the shape */
-#define FE_PATH_GEMV 1          /* route kernel + grouped GEMV gate_up + GEMV down + combine (any T) */
-#define FE_PATH_TCGEN05 2       /* tcgen05 tensor-core grouped GEMM (large T) */
+#define FE_PATH_GEMV 1          /* routing + grouped mma.sync gate_up and down + combine (any T) */
+#define FE_PATH_TCGEN05 2       /* routing + tcgen05 tensor-core tiles + combine (large T; I % 128 == 0,
+                                   H % 256 == 0, scales in the exact-f16 range) */
 #define FE_PATH_FUSED_DECODE 3  /* one cooperative kernel for the whole layer (T * top_k <= 16) */
 
 /* Force a compute path (FE_PATH_*); FE_ERR_UNSUPPORTED from forward if the
