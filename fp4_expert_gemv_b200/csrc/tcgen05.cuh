@@ -30,23 +30,29 @@
 
 namespace fe {
 
-constexpr int kTcThreads = 256;   // 8 warps; warp 0 also allocates TMEM and issues the MMAs
-constexpr int kTcWarps = kTcThreads / 32;
+constexpr int kTcDqWarps = 4;     // warps 0-3: dequantise A
+constexpr int kTcLdWarps = 4;     // warps 4-7: cp.async loads
+constexpr int kTcMmaWarp = 8;     // warp 8: TMEM allocation and the MMAs
+constexpr int kTcThreads = 32 * (kTcDqWarps + kTcLdWarps + 1);
+constexpr int kTcDqThreads = 32 * kTcDqWarps, kTcLdThreads = 32 * kTcLdWarps;
 constexpr int kTcM = 256;         // A rows (weight columns) per tile: two 128-row accumulators
 constexpr int kTcN = 256;         // B rows (tokens) per tile
-constexpr int kTcRawStages = 4;   // raw code/scale chunks in flight
-constexpr int kTcAStages = 2;     // f16 A tiles
-constexpr int kTcBStages = 3;     // f16 B tiles
+constexpr int kTcAStages = 3;     // f16 A tiles
+constexpr int kTcInStages = 3;    // raw code/scale chunks and f16 B tiles (one index)
 constexpr uint32_t kTcABytes = kTcM * 128;            // one f16 A chunk: 256 rows x 64 k
 constexpr uint32_t kTcBBytes = kTcN * 128;            // one f16 B chunk: 256 rows x 64 k
 constexpr uint32_t kTcRawBytes = 16 * 512 + 16 * 64;  // 16 blocks: one quad of codes + its scales
 constexpr uint32_t kTcTmemCols = 512;                 // two 256-column fp32 accumulators
+// mbarrier kinds (offsets into the barrier array)
+constexpr int kRawFull = 0, kBFull = kTcInStages, kInEmpty = 2 * kTcInStages, kAFull = 3 * kTcInStages,
+              kAEmpty = 3 * kTcInStages + kTcAStages, kAccFull = 3 * kTcInStages + 2 * kTcAStages,
+              kTcBars = kAccFull + 1;
 
 // Dynamic shared memory: 1024 bytes of alignment slack, then the rings, then
 // the barriers and the TMEM address.
 __host__ __device__ inline uint32_t tc_smem_bytes()
 {
-    return 1024 + kTcAStages * kTcABytes + kTcBStages * kTcBBytes + kTcRawStages * kTcRawBytes + 64 + 4 * kTcN;
+    return 1024 + kTcAStages * kTcABytes + kTcInStages * (kTcBBytes + kTcRawBytes) + 8 * kTcBars + 16 + 4 * kTcN;
 }
 
 struct TcParams {
@@ -177,7 +183,15 @@ FE_DEV uint32_t tc_swz(int r, int c) { return (uint32_t)r * 128u + (uint32_t)((c
 // ---- the grouped GEMM tile ---------------------------------------------------------
 // grid: (A tiles of one expert, tile slots); block: kTcThreads.  Tile slot y
 // holds tiles[y] = (expert e, first sorted position pos0, rows); slots past
-// n_tiles exit at once.
+// n_tiles exit at once.  Warp roles, linked only by mbarriers in the K loop:
+//   warps 0-3  dequantise chunk i's codes into the A ring (stage i % kTcAStages)
+//              once its raw bytes have landed and the MMAs of chunk i - 3 are done;
+//   warps 4-7  load chunk i's codes, scales and token rows with cp.async into
+//              stage i % kTcInStages once the MMAs of chunk i - 3 are done, and
+//              let the copies' completion arrive on the stage's "full" barriers;
+//   warp 8     issues chunk i's 8 MMAs when its A and B stages are full and
+//              commits them to the stages' "empty" barriers.
+// After the loop all warps meet, warps 0-7 read the accumulators.
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
 {
@@ -203,13 +217,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
     uint8_t* sm = tc_dyn + pad;
     uint8_t* a_ring = sm;
     uint8_t* b_ring = a_ring + kTcAStages * kTcABytes;
-    uint8_t* raw_ring = b_ring + kTcBStages * kTcBBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(raw_ring + kTcRawStages * kTcRawBytes);   // [kTcBStages]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kTcBStages);
-    int* flags = reinterpret_cast<int*>(tmem_slot + 1);                                     // [0]: abort
-    float* rmul = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 64);         // [kTcN] row scale
+    uint8_t* raw_ring = b_ring + kTcInStages * kTcBBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(raw_ring + kTcInStages * kTcRawBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kTcBars);
+    volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);                    // [0]: abort
+    float* rmul = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tmem_slot) + 16);     // [kTcN] row scale
     const uint32_t a_addr = tc_saddr(a_ring), b_addr = tc_saddr(b_ring), raw_addr = tc_saddr(raw_ring);
     const uint32_t bar0 = tc_saddr(bars);
+    auto bar = [&](int kind, int s) { return bar0 + 8u * (uint32_t)(kind + s); };
 
     // 2^shift of every B row: undoes the row's power-of-two scaling in the epilogue
     for (int r = tid; r < kTcN; r += kTcThreads) {
@@ -221,11 +236,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
         rmul[r] = m;
     }
     if (tid == 0) {
-        for (int i = 0; i < kTcBStages; ++i) tc_mbar_init(bar0 + 8 * i, 1);
+        for (int s = 0; s < kTcInStages; ++s) {
+            tc_mbar_init(bar(kRawFull, s), kTcLdThreads);
+            tc_mbar_init(bar(kBFull, s), kTcLdThreads);
+            tc_mbar_init(bar(kInEmpty, s), 1);
+        }
+        for (int s = 0; s < kTcAStages; ++s) {
+            tc_mbar_init(bar(kAFull, s), kTcDqThreads);
+            tc_mbar_init(bar(kAEmpty, s), 1);
+        }
+        tc_mbar_init(bar(kAccFull, 0), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
     }
-    if (warp == 0) {
+    if (warp == kTcMmaWarp) {
         tc_alloc(tc_saddr(tmem_slot), kTcTmemCols);
         tc_relinquish();
     }
@@ -233,70 +257,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    // this thread's B rows: chunk column tid & 7 of rows (tid >> 3) + RS m
-    constexpr int RS = kTcThreads / 8, NBR = kTcN / RS;
-    const uint16_t* brow[NBR];
-#pragma unroll
-    for (int m = 0; m < NBR; ++m) {
-        const int r = (tid >> 3) + RS * m;
-        const uint16_t* src = p.bsrc;
-        if (r < rows) {
-            const int pos = pos0 + r;
-            const int row = GATE_UP ? p.sorted_pair[pos] / p.top_k : pos;
-            src = p.bsrc + (size_t)row * K;
-        }
-        brow[m] = src;
-    }
     const uint8_t* blk0 = p.blocks + ((size_t)e * p.blocks_per_expert + 16 * mt) * (size_t)(9 * K);
 
-    auto load_raw = [&](int q) {
-        const uint32_t dst = raw_addr + (q % kTcRawStages) * kTcRawBytes;
+    if (warp < kTcDqWarps) {
+        // ---- dequantise: raw codes x group scales -> f16 A rows ------------------------
+        for (int i = 0; i < nk; ++i) {
+            const int si = i % kTcInStages, sa = i % kTcAStages;
+            if (!tc_mbar_wait(bar(kRawFull, si), (i / kTcInStages) & 1, p.timeout_ns) ||
+                (i >= kTcAStages && !tc_mbar_wait(bar(kAEmpty, sa), ((i - kTcAStages) / kTcAStages) & 1, p.timeout_ns)))
+                flags[0] = 1;
+            if (flags[0]) break;
+            const uint8_t* raw = raw_ring + si * kTcRawBytes;
+            uint8_t* A = a_ring + sa * kTcABytes;
 #pragma unroll
-        for (int m = 0; m < 512 / kTcThreads; ++m) {
-            const int c = tid + kTcThreads * m, bi = c >> 5, w16 = c & 31;
-            cp_async16(dst + bi * 512 + 16 * w16, blk0 + (size_t)bi * (9 * K) + 512 * q + 16 * w16, 16);
-        }
-        if (tid < 64) {
-            const int bi = tid >> 2, w16 = tid & 3;
-            cp_async16(dst + 8192 + bi * 64 + 16 * w16, blk0 + (size_t)bi * (9 * K) + 8 * K + 64 * q + 16 * w16, 16);
-        }
-    };
-    auto load_b = [&](int q) {
-        const uint32_t dst = b_addr + (q % kTcBStages) * kTcBBytes;
-        const int c = tid & 7;
-#pragma unroll
-        for (int m = 0; m < NBR; ++m) {
-            const int r = (tid >> 3) + RS * m;
-            cp_async16(dst + tc_swz(r, c), brow[m] + 64 * q + 8 * c, r < rows ? 16u : 0u);
-        }
-    };
-
-    // prologue: raw 0, 1, 2 and B 0, 1 in three groups
-    load_raw(0);
-    cp_async_commit();
-    if (nk > 1) load_raw(1);
-    load_b(0);
-    cp_async_commit();
-    if (nk > 2) load_raw(2);
-    if (nk > 1) load_b(1);
-    cp_async_commit();
-
-    const uint32_t idesc = tc_instr_desc(128, nb);
-    bool abort = false;
-    int issued = -1;   // last chunk whose MMAs were issued
-    const bool tr = p.trace != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0;
-    for (int i = 0; i < nk; ++i) {
-        cp_async_wait<1>();
-        __syncthreads();
-        if (tr && i < 64) p.trace[3 * i] = clock64();
-        // ---- dequantise chunk i: raw codes x group scales -> f16 A rows --------------
-        {
-            const uint8_t* raw = raw_ring + (i % kTcRawStages) * kTcRawBytes;
-            uint8_t* A = a_ring + (i % kTcAStages) * kTcABytes;
-#pragma unroll
-            for (int m = 0; m < 16 / kTcWarps; ++m) {
-                const int bi = (16 / kTcWarps) * warp + m;
+            for (int m = 0; m < 16 / kTcDqWarps; ++m) {
+                const int bi = (16 / kTcDqWarps) * warp + m;
                 const uint4 cw = *reinterpret_cast<const uint4*>(raw + bi * 512 + 16 * lane);
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
                 const uint32_t* sc = reinterpret_cast<const uint32_t*>(raw + 8192 + bi * 64);
@@ -324,49 +299,88 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
                     }
                 }
             }
+            fence_proxy_async_smem();
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar(kAFull, sa)) : "memory");
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tr && i < 64) p.trace[3 * i + 1] = clock64();
-        // ---- one thread issues chunk i's MMAs: 2 accumulators x 4 k-steps ----------
-        if (warp == 0) {
+    } else if (warp < kTcDqWarps + kTcLdWarps) {
+        // ---- load: codes + scales and token rows of chunk i ------------------------------
+        const int lt = tid - kTcDqThreads;
+        const int c = lt & 7;
+        const uint16_t* brow[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const int r = (lt >> 3) + 16 * m;
+            const uint16_t* src = p.bsrc;
+            if (r < rows) {
+                const int pos = pos0 + r;
+                src = p.bsrc + (size_t)(GATE_UP ? p.sorted_pair[pos] / p.top_k : pos) * K;
+            }
+            brow[m] = src;
+        }
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % kTcInStages;
+            if (i >= kTcInStages && !tc_mbar_wait(bar(kInEmpty, s), ((i - kTcInStages) / kTcInStages) & 1, p.timeout_ns))
+                flags[0] = 1;
+            if (flags[0]) break;
+            const uint32_t rdst = raw_addr + s * kTcRawBytes;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cc = lt + kTcLdThreads * m, bi = cc >> 5, w16 = cc & 31;
+                cp_async16(rdst + bi * 512 + 16 * w16, blk0 + (size_t)bi * (9 * K) + 512 * i + 16 * w16, 16);
+            }
+            if (lt < 64) {
+                const int bi = lt >> 2, w16 = lt & 3;
+                cp_async16(rdst + 8192 + bi * 64 + 16 * w16, blk0 + (size_t)bi * (9 * K) + 8 * K + 64 * i + 16 * w16, 16);
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(kRawFull, s)) : "memory");
+            const uint32_t bdst = b_addr + s * kTcBBytes;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int r = (lt >> 3) + 16 * m;
+                cp_async16(bdst + tc_swz(r, c), brow[m] + 64 * i + 8 * c, r < rows ? 16u : 0u);
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(kBFull, s)) : "memory");
+        }
+        cp_async_wait<0>();   // no copy outlives the loop
+    } else {
+        // ---- one thread issues the MMAs of every chunk -----------------------------------
+        const uint32_t idesc = tc_instr_desc(128, nb);
+        int issued = -1;
+        for (int i = 0; i < nk; ++i) {
+            const int si = i % kTcInStages, sa = i % kTcAStages;
+            if (!tc_mbar_wait(bar(kAFull, sa), (i / kTcAStages) & 1, p.timeout_ns) ||
+                !tc_mbar_wait(bar(kBFull, si), (i / kTcInStages) & 1, p.timeout_ns))
+                flags[0] = 1;
+            if (flags[0]) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t aa = a_addr + (i % kTcAStages) * kTcABytes;
-                const uint32_t ba = b_addr + (i % kTcBStages) * kTcBBytes;
+                if (p.trace && blockIdx.x == 0 && blockIdx.y == 0 && i < 64) p.trace[i] = (unsigned long long)clock64();
+                const uint32_t aa = a_addr + sa * kTcABytes;
+                const uint32_t ba = b_addr + si * kTcBBytes;
 #pragma unroll
                 for (int acc = 0; acc < 2; ++acc)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         tc_mma_f16(tmem + 256 * acc, tc_smem_desc(aa + acc * (kTcABytes / 2) + 32 * ks),
                                    tc_smem_desc(ba + 32 * ks), idesc, (i > 0 || ks > 0) ? 1u : 0u);
-                tc_commit(bar0 + 8 * (i % kTcBStages));
+                tc_commit(bar(kAEmpty, sa));
+                tc_commit(bar(kInEmpty, si));
             }
             __syncwarp();
+            issued = i;
         }
-        issued = i;
-        // ---- chunk i-1's MMAs done: its B stage and A stage may be refilled ----------
-        if (i >= 1 && !tc_mbar_wait(bar0 + 8 * ((i - 1) % kTcBStages), ((i - 1) / kTcBStages) & 1, p.timeout_ns))
-            flags[0] = 1;
-        if (__syncthreads_or(flags[0] != 0)) {
-            abort = true;
-            break;
-        }
-        if (tr && i < 64) p.trace[3 * i + 2] = clock64();
-        if (i + 2 < nk) load_b(i + 2);
-        if (i + 3 < nk) load_raw(i + 3);
-        cp_async_commit();
+        if (lane == 0 && issued >= 0) tc_commit(bar(kAccFull, 0));   // every MMA issued so far
+        __syncwarp();
+        // never leave with MMAs in flight (bounded): they read shared memory and TMEM
+        if (issued >= 0 && !tc_mbar_wait(bar(kAccFull, 0), 0, p.timeout_ns)) flags[0] = 1;
+        if (issued < nk - 1) flags[0] = 1;
     }
-    cp_async_wait<0>();
+    __syncthreads();
     if (ttr && tid == 0) ttr[1] = globaltimer_ns();
 
-    // ---- epilogue: the last chunk's MMAs, then TMEM -> registers -> global -------------
-    if (!abort && !tc_mbar_wait(bar0 + 8 * ((nk - 1) % kTcBStages), ((nk - 1) / kTcBStages) & 1, p.timeout_ns))
-        flags[0] = 1;
-    abort = __syncthreads_or(flags[0] != 0);
+    // ---- epilogue: TMEM -> registers -> global ---------------------------------------------
+    const bool abort = flags[0] != 0;
     if (abort) {
-        // never free TMEM under MMAs in flight: wait (bounded) for the last issued chunk
-        if (issued >= 0) tc_mbar_wait(bar0 + 8 * (issued % kTcBStages), (issued / kTcBStages) & 1, p.timeout_ns);
         if (tid == 0) atomicOr(p.status, kDevTcTimeout);
     } else {
         tc_fence_after();
@@ -377,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
         const int ocol0 = GATE_UP ? (kTcM / 2) * mt : kTcM * mt;
 #pragma unroll 1
         for (int c0 = 0; c0 < nb; c0 += 32) {
-            {
+            if (warp < 8) {
                 // warps 0-3 read accumulator 0, warps 4-7 accumulator 1 (TMEM lanes 32 (warp % 4) ...)
                 const int acc = warp >> 2;
                 const int row = 128 * acc + 32 * (warp & 3) + lane;   // A row of this thread's TMEM lane
@@ -419,7 +433,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tc_dealloc(tmem, kTcTmemCols);
+    if (warp == kTcMmaWarp) tc_dealloc(tmem, kTcTmemCols);
     if (ttr && tid == 0) ttr[2] = globaltimer_ns();
 }
 
