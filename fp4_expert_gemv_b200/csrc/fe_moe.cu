@@ -335,7 +335,7 @@ fe_status tcgen05_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_
 {
     const int P = T * k;
     const int max_tiles = (int)tc_max_tiles(h, (size_t)P);
-    fe::tc_tiles_kernel<<<1, 32, 0, s>>>(h->counts, h->offsets, h->E, h->tc_tiles, h->tc_ntiles);
+    fe::tc_tiles_kernel<<<1, 1024, 0, s>>>(h->counts, h->offsets, h->E, h->tc_tiles, h->tc_ntiles);
     fe::tc_rows_to_f16_kernel<true><<<(T + 7) / 8, 256, 0, s>>>(x, T, h->H, h->tc_x, h->tc_xshift);
     fe::TcParams tp{};
     tp.tiles = h->tc_tiles;

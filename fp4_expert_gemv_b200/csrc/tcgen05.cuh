@@ -440,23 +440,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
 // ---- small kernels around the tiles -------------------------------------------------
 
 // Tile list: for every expert with tokens, ceil(count / kTcN) tiles of at
-// most kTcN sorted positions.  One thread (E is small; this runs once per
-// forward on a few hundred entries).
-__global__ void tc_tiles_kernel(const int32_t* counts, const int32_t* offsets, int E, int32_t* tiles,
-                                int32_t* n_tiles)
+// most kTcN sorted positions, experts in ascending order.  One block of 1024
+// threads: thread e counts expert e's tiles, a block scan gives its first slot.
+__global__ void __launch_bounds__(1024) tc_tiles_kernel(const int32_t* counts, const int32_t* offsets, int E,
+                                                        int32_t* tiles, int32_t* n_tiles)
 {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int n = 0;
-    for (int e = 0; e < E; ++e) {
-        const int c = counts[e], o = offsets[e];
-        for (int r0 = 0; r0 < c; r0 += kTcN) {
-            tiles[3 * n] = e;
-            tiles[3 * n + 1] = o + r0;
-            tiles[3 * n + 2] = min(kTcN, c - r0);
-            ++n;
+    __shared__ int wsum[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 1024) {
+        const int e = e0 + (int)threadIdx.x;
+        const int c = e < E ? counts[e] : 0;
+        const int nt = (c + kTcN - 1) / kTcN;
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int v = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            wsum[lane] = v;   // inclusive over warps
+        }
+        __syncthreads();
+        const int base = carry + (warp > 0 ? wsum[warp - 1] : 0) + incl - nt;
+        if (e < E) {
+            const int o = offsets[e];
+            for (int i = 0; i < nt; ++i) {
+                tiles[3 * (base + i)] = e;
+                tiles[3 * (base + i) + 1] = o + kTcN * i;
+                tiles[3 * (base + i) + 2] = min(kTcN, c - kTcN * i);
+            }
+        }
+        carry += wsum[31];
+        __syncthreads();
     }
-    *n_tiles = n;
+    if (threadIdx.x == 0) *n_tiles = carry;
 }
 
 // Rows of n values -> f16 scaled by 2^-s with s = fp16_shift(row max); one warp
