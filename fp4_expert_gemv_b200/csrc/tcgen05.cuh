@@ -387,10 +387,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
         // 32 tokens at a time: TMEM -> registers -> a [token][column] tile in the
         // (now idle) A ring -> coalesced 16-byte row stores
         constexpr int OC = GATE_UP ? kTcM / 2 : kTcM;   // output columns of the tile
-        float* st = reinterpret_cast<float*>(a_ring);    // [32][OC]
         const int ocol0 = GATE_UP ? (kTcM / 2) * mt : kTcM * mt;
 #pragma unroll 1
         for (int c0 = 0; c0 < nb; c0 += 32) {
+            // two staging tiles [32][OC] (column j of token n stored at j ^ (n & 16), so the
+            // gate and up lanes of one column, writing tokens n and n + 16, use different banks)
+            float* st = reinterpret_cast<float*>(a_ring) + ((c0 >> 5) & 1) * (32 * OC);
             if (warp < 8) {
                 // warps 0-3 read accumulator 0, warps 4-7 accumulator 1 (TMEM lanes 32 (warp % 4) ...)
                 const int acc = warp >> 2;
@@ -413,11 +415,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
                         const float own = up ? hi : lo;
                         const float gv = up ? other : own, uv = up ? own : other;
                         const float m = rmul[c0 + tn];
-                        st[tn * OC + acol] = silu_mul(gv * m, uv * m);
+                        const float gs = gv * m;
+                        st[tn * OC + (acol ^ (tn & 16))] = __fdividef(gs, 1.0f + __expf(-gs)) * (uv * m);
                     }
                 } else {
 #pragma unroll
-                    for (int n = 0; n < 32; ++n) st[n * OC + row] = __uint_as_float(r[n]) * rmul[c0 + n];
+                    for (int n = 0; n < 32; ++n) st[n * OC + (row ^ (n & 16))] = __uint_as_float(r[n]) * rmul[c0 + n];
                 }
             }
             __syncthreads();
@@ -425,10 +428,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
             constexpr int V4 = OC / 4;   // float4 per token row
             for (int idx = tid; idx < nrows * V4; idx += kTcThreads) {
                 const int n = idx / V4, v = idx - n * V4;
-                const float4 val = reinterpret_cast<const float4*>(st + n * OC)[v];
+                const float4 val = reinterpret_cast<const float4*>(st + n * OC)[v ^ ((n & 16) >> 2)];
                 reinterpret_cast<float4*>(p.out + (size_t)(pos0 + c0 + n) * p.out_ld + ocol0)[v] = val;
             }
-            __syncthreads();
+            // the next 32 tokens go to the other staging tile: no barrier needed here
         }
     }
     tc_fence_before();
