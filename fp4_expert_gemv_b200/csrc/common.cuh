@@ -78,6 +78,10 @@ FE_DEV float silu_mul(float g, float u)
     return g / (1.0f + expf(-g)) * u;
 }
 
+// The same with the fast exponential and division (a few ulp; 0 for g below
+// about -88, where exp(-g) overflows).
+FE_DEV float silu_mul_fast(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
 FE_DEV unsigned long long globaltimer_ns()
 {
     unsigned long long t;

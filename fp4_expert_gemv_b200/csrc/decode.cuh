@@ -49,6 +49,16 @@ constexpr int kDecMaxItems = 48;   // weight units (mbarriers) per CTA
 constexpr int kDecMaxE = 512;      // experts routed by one warp: 16 logits per lane
 constexpr int kDecQuadsPerWarp = 4;   // gate_up quads whose x fragments a warp keeps in registers
 constexpr int kDecCandCap = 128;   // candidate keys per routing warp (in the gate_up partials' space)
+constexpr int kDecRedFloats = 4096;   // gate_up partials held before one reduction (also the down partials)
+#ifndef FE_DEC_ARRIVE_SLACK
+#define FE_DEC_ARRIVE_SLACK 16
+#endif
+constexpr int kDecArriveSlack = FE_DEC_ARRIVE_SLACK;   // producers still out when consumers start reading act
+constexpr int kDecMaxJobs = kDecRedFloats / (kDecWarps * 32);   // act columns one reduction serves
+#ifndef FE_DEC_DOWN_LATE
+#define FE_DEC_DOWN_LATE 1
+#endif
+constexpr int kDecDownLate = FE_DEC_DOWN_LATE;   // down copies issued once this many gate_up units landed
 constexpr uint32_t kDevBarrierTimeout = 0x4;
 constexpr uint32_t kDevLoadTimeout = 0x8;
 
@@ -66,8 +76,8 @@ struct DecodeParams {
     int32_t* offsets;
     int32_t* sorted_pair;
     int32_t* pair_row;
-    unsigned long long* act;  // [kDecMaxPairs][I] by pair id: (epoch tag << 32) | fp32 bits
-    unsigned* epoch;          // [grid]: launches CTA c has run on this handle (the act tag of the last)
+    unsigned long long* act;  // [kDecMaxPairs][I] by pair id: (launch tag << 32) | fp32 bits
+    unsigned long long* epoch;  // [grid + 1]: launches CTA c has run on this handle; [grid]: arrivals
     uint32_t* status;
     unsigned long long timeout_ns;  // bound of every wait
     uint32_t weight_bytes;    // shared memory reserved for weight units
@@ -158,8 +168,14 @@ FE_DEV void stamp(unsigned long long* trace, int i)
     asm volatile("" ::: "memory");
 }
 
-// Tagged act words: device-scope relaxed accesses (each 64-bit word is
-// single-copy atomic, so a reader sees either the old tag or the new value).
+// The act exchange.  act words carry the launch's tag next to the value
+// (each 64-bit word is single-copy atomic, so a reader sees the old tag or the
+// new value): a word with this launch's tag is this launch's value, whatever
+// order the memory system delivers things in.  So that consumers do not flood
+// L2 with polls of data that is not there yet, every CTA also adds 1 to an
+// arrival counter after its act stores, and a consumer reads act only once the
+// counter shows every CTA of the launch; the counter carries no ordering (no
+// fence), the tags still decide, and the few words still in flight are read again.
 FE_DEV void st_relaxed_u64(unsigned long long* p, unsigned long long v)
 {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -169,6 +185,22 @@ FE_DEV void ld_relaxed_2u64(const unsigned long long* p, unsigned long long& a, 
 {
     asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
+
+FE_DEV void arrive_relaxed(unsigned long long* counter)
+{
+    asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(counter) : "memory");
+}
+
+FE_DEV unsigned long long ld_relaxed_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Act tag of launch ep (1, 2, ...): never 0 (the value act starts from) and
+// different for consecutive launches, also across the wrap of 32 bits.
+FE_DEV unsigned act_tag(unsigned long long ep) { return (unsigned)(ep % 0xffffffffull) + 1u; }
 
 // ---- routing ---------------------------------------------------------------------
 // Orderable key of logit v of expert e: a larger key ranks first.  NaN ranks
@@ -310,6 +342,10 @@ struct DecodeShared {
     int dstart[kDecMaxPairs + 1]; // first sorted position of each distinct expert
     int plan[kDecMaxPairs + 1][4];  // per nd: gate_up first/end, down first/end of this CTA
     int xshift[kDecMaxPairs];
+    int job_act[kDecMaxJobs];     // pending act columns: act offset (pair row, unit block),
+    int job_red[kDecMaxJobs];     // first partial, partial stride between warps, x shift
+    int job_stride[kDecMaxJobs];
+    int job_shift[kDecMaxJobs];
     int ashift[kDecMaxPairs];
     int item_d[kDecMaxPairs + 1];   // down items: (distinct expert, first sorted pair, pairs <= 8)
     int item_r[kDecMaxPairs + 1];
@@ -317,7 +353,8 @@ struct DecodeShared {
     int n_items;
     int nd;
     int abort;
-    unsigned tag;
+    unsigned long long target;    // arrivals that complete this launch's act
+    unsigned tag;                 // this launch's act tag
     float wmax[2][kDecWarps];
     float ob[kDecMaxPairs * 16];  // down: [pair][16] outputs
 };
@@ -348,6 +385,18 @@ FE_DEV void group_single_token(DecodeShared& S, int k, int lane)
     __syncwarp();
 }
 
+// Bulk copies of the CTA's down units (one per routed expert and unit), issued
+// by the lanes of one warp; their barriers' byte counts are already armed.
+FE_DEV void issue_down(const DecodeParams& p, const DecodeShared& S, uint32_t dst, int nd, int dn0, int ndn, int ngu,
+                       uint32_t dn_blk, uint32_t mbar0, int lane)
+{
+    for (int i = lane; i < ndn * nd; i += 32) {
+        const int u = i / nd, dd = i - u * nd, j = dn0 + u;
+        bulk_g2s(dst + (u * nd + dd) * dn_blk, p.dn_blocks + ((size_t)S.dex[dd] * (p.H / 16) + j) * dn_blk, dn_blk,
+                 mbar0 + 8 * (ngu + u));
+    }
+}
+
 // Byte offsets of the dynamic shared memory regions.
 struct DecodeSmem {
     uint32_t mbar, shared, red, dred, xs, as, xr, total;
@@ -363,7 +412,8 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(uint32_t weight_bytes, 
     L.shared = L.mbar + 8 * (kDecMaxItems + 1);
     L.red = align16(L.shared + (uint32_t)sizeof(DecodeShared));
     L.dred = L.red;   // gate_up partials and down partials are never live together
-    L.xs = L.red + 4u * (kDecWarps * 32 * 8 > 8 * 4 * 32 * 4 ? kDecWarps * 32 * 8 : 8 * 4 * 32 * 4);
+    static_assert(kDecRedFloats >= kDecWarps * 32 * 8 && kDecRedFloats >= 8 * 4 * 32 * 4, "partials space");
+    L.xs = L.red + 4u * kDecRedFloats;
     L.as = L.xs + 4u * (T + 1) * brow_words(H);
     L.xr = align16(L.as + 4u * (T * k + 1) * brow_words(I));
     L.total = align16(L.xr + 2u * T * H);
@@ -417,11 +467,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         mbar_expect_tx(in_bar, xb);
         bulk_g2s(smem_addr(xr), p.x, xb, in_bar);
     }
-    // this launch's act tag: every launch runs every CTA once, so the per-CTA
-    // launch counts move in lockstep and all CTAs derive the same tag without
-    // talking to each other; the load is consumed only when act is about to be written
-    unsigned ep_e0 = 0;
-    if (tid == kDecThreads - 1) ep_e0 = *reinterpret_cast<volatile unsigned*>(p.epoch + blockIdx.x);
+    // this launch's arrival target: every launch runs every CTA (the grid is
+    // fixed per handle) and each CTA arrives once, so the per-CTA launch counts
+    // move in lockstep and all CTAs derive the same target without talking to
+    // each other; the load is consumed only when the staging warps finish
+    unsigned long long ep_e0 = 0;
+    if (tid == kDecThreads - 1) ep_e0 = *reinterpret_cast<volatile unsigned long long*>(p.epoch + blockIdx.x);
     // candidate keys of the routing warps live in the gate_up partials' space
     const int nroute = min(T, kDecWarps);
     const int cap = (kDecWarps * kDecCandCap) / nroute;
@@ -513,11 +564,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 bulk_g2s(wb + u * gu_unit, p.gu_blocks + ((size_t)S.dex[dd] * ntu + j) * gu_unit, gu_unit,
                          mbar0 + 8 * u);
             }
-            for (int i = lane; i < ndn * nd; i += 32) {
-                const int u = i / nd, dd = i - u * nd, j = dn0 + u;
-                bulk_g2s(wb + ngu * gu_unit + u * dn_unit + dd * dn_blk,
-                         p.dn_blocks + ((size_t)S.dex[dd] * (H / 16) + j) * dn_blk, dn_blk, mbar0 + 8 * (ngu + u));
-            }
+            if (kDecDownLate == 0 || ngu == 0) issue_down(p, S, wb + ngu * gu_unit, nd, dn0, ndn, ngu, dn_blk, mbar0, lane);
         }
         if (tracing && lane == 0) stamp(trace, 1);
     } else if (warp == 0) {
@@ -584,9 +631,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         }
         if (tracing && xt == 0) stamp(trace, 2);
         if (tid == kDecThreads - 1) {
-            const unsigned tg = (ep_e0 + 1u) ? (ep_e0 + 1u) : 1u;   // 0 is the never-written value
-            S.tag = tg;
-            p.epoch[blockIdx.x] = tg;
+            S.target = (ep_e0 + 1ull) * gridDim.x;
+            S.tag = act_tag(ep_e0 + 1ull);
+            p.epoch[blockIdx.x] = ep_e0 + 1ull;
         }
     }
     __syncthreads();
@@ -600,10 +647,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         trace[32 + 29] = (unsigned long long)ndn;
     }
 
-    // ---- 5. gate_up units -> tagged act ------------------------------------------------
+    // ---- 5. gate_up units -> act -------------------------------------------------------
     // Warp w runs quads w, w + W, ... (W = warps) of every unit.  Its x fragments
     // for those quads stay in registers while the n-block's rows stay the same
-    // (always, for one token): the inner loop then reads only weights.
+    // (always, for one token): the inner loop then reads only weights.  The
+    // per-warp partials of a tile (one unit, up to 8 tokens) wait in shared
+    // memory, and one reduction serves every tile computed since the last, so
+    // the warps meet once per layer rather than once per unit; act is read
+    // only after every CTA has written its part, so nothing waits on it sooner.
     uint32_t off = 0;
     {
         const int nq = H / 64;
@@ -611,20 +662,57 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         const int npass = (nq + QPW * kDecWarps - 1) / (QPW * kDecWarps);
         uint32_t bx[QPW][8];
         int bkey = -1;
+        int njobs = 0, red_used = 0;   // the same in every thread
+        const unsigned long long tg = (unsigned long long)S.tag << 32;
+        // reduce the pending act columns' partials over the warps and write act
+        auto flush = [&]() {
+            __syncthreads();
+            if (tracing && tid == 0) stamp(trace, 17);
+            if (!*reinterpret_cast<volatile int*>(&S.abort)) {
+                const int half = lane & 1, n = lane >> 1;
+                for (int jb = warp; jb < njobs; jb += kDecWarps) {
+                    const float* rw = red + S.job_red[jb] + half * (kDecWarps / 2) * S.job_stride[jb] + n;
+                    const int stride = S.job_stride[jb];
+                    float gs = 0.0f, us = 0.0f;
+#pragma unroll
+                    for (int w2 = 0; w2 < kDecWarps / 2; ++w2) {
+                        gs += rw[w2 * stride];
+                        us += rw[w2 * stride + 16];
+                    }
+                    gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+                    us += __shfl_xor_sync(0xffffffffu, us, 1);
+                    if (half == 0) {
+                        const float m = pow2f(S.job_shift[jb]);
+                        const float a = silu_mul_fast(gs * m, us * m);
+                        st_relaxed_u64(p.act + S.job_act[jb] + n, tg | __float_as_uint(a));
+                    }
+                }
+            }
+            if (tracing && tid == 0) stamp(trace, 18);
+            __syncthreads();
+            if (tracing && tid == 0) stamp(trace, 19);
+            njobs = 0;
+            red_used = 0;
+        };
         for (int u = 0; u < ngu; ++u) {
-            if (!mbar_wait0(mbar0 + 8 * u, p.timeout_ns)) {
+            // after a timed-out wait the other units are skipped (their work is
+            // discarded at the reduction, which every thread still reaches)
+            if (*reinterpret_cast<volatile int*>(&S.abort) || !mbar_wait0(mbar0 + 8 * u, p.timeout_ns)) {
+                if (!S.abort) atomicOr(p.status, kDevLoadTimeout);
                 S.abort = 1;
-                atomicOr(p.status, kDevLoadTimeout);
             }
             if (tracing && tid == 0 && (u == 0 || u == ngu - 1)) stamp(trace, u == 0 ? 11 : 13);
             if (tracing && tid == 0 && u == 1) stamp(trace, 24);
+            if (kDecDownLate > 0 && warp == 1 && u == min(ngu, kDecDownLate) - 1)
+                issue_down(p, S, smem_addr(wbuf) + ngu * gu_unit, nd, dn0, ndn, ngu, dn_blk, mbar0, lane);
             const int gid = gu0 + u, dd = gid / ntu, j = gid - dd * ntu;
             const uint8_t* blk0 = wbuf + off;
             const uint8_t* blk1 = blk0 + block_bytes(H);
             const int r0 = S.dstart[dd], r1 = S.dstart[dd + 1];
-            bool stop = false;
-            for (int nb = r0; nb < r1 && !stop; nb += 8) {
+            for (int nb = r0; nb < r1; nb += 8) {
                 const int nvalid = min(8, r1 - nb);
+                const int need = kDecWarps * nvalid * 32;
+                if (red_used + need > kDecRedFloats) flush();
                 const int key = T == 1 ? 0 : (dd << 8) + (nb - r0);
                 const uint32_t* brow = xs + (g < nvalid ? S.sp[nb + g] / k : T) * xrw;
                 float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -649,11 +737,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                     }
                 }
                 if (tracing && tid == 0 && u < 2) stamp(trace, u == 0 ? 16 : 25);
-                // partials of the valid token columns only: red[warp][column][gate 16 | up 16];
+                // partials of the valid token columns only: [warp][column][gate 16 | up 16];
                 // lane (g, c) holds rows g, g+8 of columns 2c, 2c+1
                 {
                     const int c = lane & 3;
-                    float* rw = red + warp * (8 * 32);
+                    float* rw = red + red_used + warp * nvalid * 32;
                     if (2 * c < nvalid) {
                         rw[(2 * c) * 32 + g] = t0[0];
                         rw[(2 * c) * 32 + g + 8] = t0[2];
@@ -667,42 +755,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                         rw[(2 * c + 1) * 32 + 24 + g] = t1[3];
                     }
                 }
-                __syncthreads();
-                if (tracing && tid == 0 && u == 0) stamp(trace, 17);
-                if (S.abort) {
-                    stop = true;
-                    continue;
+                if (tid < nvalid) {
+                    // column tid of this tile: its act word, partials and x shift
+                    const int pid = S.sp[nb + tid];
+                    S.job_act[njobs + tid] = pid * I + 16 * j;
+                    S.job_red[njobs + tid] = red_used + tid * 32;
+                    S.job_stride[njobs + tid] = nvalid * 32;
+                    S.job_shift[njobs + tid] = S.xshift[pid / k];
                 }
-                // 2 threads per (column, output): each adds half the warps' partials, then 1 shuffle
-                {
-                    const int half = tid & 1, n = (tid >> 1) & 15, jt = tid >> 5;   // jt < 8
-                    float gs = 0.0f, us = 0.0f;
-                    if (jt < nvalid) {
-#pragma unroll
-                        for (int w2 = 0; w2 < kDecWarps / 2; ++w2) {
-                            const float* rw = red + (half * (kDecWarps / 2) + w2) * (8 * 32) + jt * 32;
-                            gs += rw[n];
-                            us += rw[16 + n];
-                        }
-                    }
-                    gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-                    us += __shfl_xor_sync(0xffffffffu, us, 1);
-                    if (jt < nvalid && half == 0) {
-                        const int pid = S.sp[nb + jt], t = pid / k;
-                        const float m = pow2f(S.xshift[t]);
-                        const float a = silu_mul(gs * m, us * m);
-                        st_relaxed_u64(p.act + (size_t)pid * I + 16 * j + n,
-                                        ((unsigned long long)S.tag << 32) | __float_as_uint(a));
-                    }
-                }
-                if (tracing && tid == 0 && u == 0) stamp(trace, 18);
-                __syncthreads();
-                if (tracing && tid == 0 && u == 0) stamp(trace, 19);
+                njobs += nvalid;
+                red_used += need;
             }
-            if (stop) break;
             off += gu_unit;
         }
+        flush();
     }
+    // every CTA arrives once per launch, on every path, so the counts stay in lockstep
+    if (tid == 0) arrive_relaxed(p.epoch + gridDim.x);
     if (tracing && tid == 0) stamp(trace, 3);
     if (tracing) {
         // diagnostics only: when the down weights have landed
@@ -710,13 +779,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         if (tid == 0) stamp(trace, 14);
     }
 
-    // ---- 6. down units: read act back (tagged), compute, combine ------------------------
+    // ---- 6. down units: read every CTA's act back (tagged), compute, combine -----------
     off = (uint32_t)ngu * gu_unit;
-    const unsigned tag = S.tag;
     if (ndn > 0 && !S.abort) {
+        const unsigned long long t_poll = globaltimer_ns();
+        if (tid == 0) {
+            // one thread polls the arrival counter (bounded) until all but the last
+            // few CTAs have arrived; the CTA meets after it and reads act, polling
+            // only the words those few CTAs still have to deliver
+            const unsigned long long target = S.target;
+            const unsigned long long* ctr = p.epoch + gridDim.x;
+            while ((long long)(ld_relaxed_u64(ctr) - (target - kDecArriveSlack)) < 0) {
+                if (globaltimer_ns() - t_poll > p.timeout_ns) {
+                    atomicOr(p.status, kDevBarrierTimeout);
+                    S.abort = 1;
+                    break;
+                }
+            }
+            if (tracing) stamp(trace, 26);
+        }
+        __syncthreads();
+        const unsigned tag = S.tag;
         // warp pp stages pair pp: up to 16 chunks of two tagged words per lane, all
-        // requested at once, then only the late ones again
-        for (int pp = warp; pp < P; pp += kDecWarps) {
+        // requested at once, then only the ones not yet carrying this launch's tag again
+        for (int pp = warp; pp < P && !S.abort; pp += kDecWarps) {
             const unsigned long long* src = p.act + (size_t)pp * I;
             unsigned long long a0[16], a1[16];
             uint32_t pending = 0;
@@ -724,29 +810,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;
                 a0[i] = a1[i] = 0ull;
-                if (2 * r < I) {
-                    ld_relaxed_2u64(src + 2 * r, a0[i], a1[i]);
-                    if ((unsigned)(a0[i] >> 32) != tag || (unsigned)(a1[i] >> 32) != tag) pending |= 1u << i;
-                }
+                if (2 * r < I) ld_relaxed_2u64(src + 2 * r, a0[i], a1[i]);
             }
-            if (__any_sync(0xffffffffu, pending != 0)) {
-                const unsigned long long t0 = globaltimer_ns();
-                bool late = false;
-                while (__any_sync(0xffffffffu, pending != 0) && !late) {
-                    __nanosleep(64);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        if ((pending >> i) & 1u) {
-                            ld_relaxed_2u64(src + 2 * (lane + 32 * i), a0[i], a1[i]);
-                            if ((unsigned)(a0[i] >> 32) == tag && (unsigned)(a1[i] >> 32) == tag) pending &= ~(1u << i);
-                        }
+            for (int i = 0; i < 16; ++i)
+                if (2 * (lane + 32 * i) < I && ((unsigned)(a0[i] >> 32) != tag || (unsigned)(a1[i] >> 32) != tag))
+                    pending |= 1u << i;
+            bool late = false;
+            if (tracing && lane == 0 && pp == 0) stamp(trace, 22);
+            int rounds = 0;
+            while (__any_sync(0xffffffffu, pending != 0) && !late) {
+                ++rounds;
+                __nanosleep(32);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    if ((pending >> i) & 1u) {
+                        ld_relaxed_2u64(src + 2 * (lane + 32 * i), a0[i], a1[i]);
+                        if ((unsigned)(a0[i] >> 32) == tag && (unsigned)(a1[i] >> 32) == tag) pending &= ~(1u << i);
                     }
-                    late = __any_sync(0xffffffffu, globaltimer_ns() - t0 > p.timeout_ns);
                 }
-                if (late && lane == 0) {
-                    atomicOr(p.status, kDevBarrierTimeout);
-                    S.abort = 1;
-                }
+                late = __any_sync(0xffffffffu, globaltimer_ns() - t_poll > p.timeout_ns);
+            }
+            if (late && lane == 0) {
+                atomicOr(p.status, kDevBarrierTimeout);
+                S.abort = 1;
+            }
+            if (tracing && lane == 0 && pp == 0) {
+                stamp(trace, 23);
+                trace[27] = rounds;
             }
             float m = 0.0f;
 #pragma unroll
@@ -757,7 +848,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             const int sh = fp16_shift(m);
             const float scl = pow2f(-sh);
             if (lane == 0) S.ashift[pp] = sh;
-            if (tracing && lane == 0 && pp == 0) stamp(trace, 26);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;

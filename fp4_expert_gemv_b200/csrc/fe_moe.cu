@@ -49,9 +49,9 @@ struct fe_moe_s {
     int32_t* max_count = nullptr;
     float* act = nullptr;
     float* o = nullptr;
-    unsigned long long* act_ll = nullptr;   // fused decode: tagged act words
+    unsigned long long* dec_act = nullptr;  // fused decode: tagged act words by pair id
     int32_t* plan = nullptr;                // fused decode: work split per nd
-    unsigned* dec_epoch = nullptr;          // fused decode: per-CTA launch counts (act tags)
+    unsigned long long* dec_epoch = nullptr;  // fused decode: per-CTA launch counts, then the arrival counter
     unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
     // tensor-core path (tcgen05.cuh)
     bool tc_scales_ok = false;              // every group scale in the exact-f16 range
@@ -116,14 +116,14 @@ void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
-                    h->act_ll, h->dec_epoch, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
+                    h->dec_act, h->dec_epoch, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
                     h->tc_tiles, h->tc_ntiles, h->grp_bh};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
     h->pair_row = nullptr; h->active = nullptr; h->n_active = nullptr; h->max_count = nullptr; h->act = nullptr;
     h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
-    h->act_ll = nullptr;
+    h->dec_act = nullptr;
     h->dec_epoch = nullptr;
     h->plan = nullptr;
     h->tc_x = nullptr; h->tc_xshift = nullptr; h->tc_act = nullptr; h->tc_ashift = nullptr;
@@ -210,7 +210,7 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     dp.plan = h->plan;
     dp.idx = h->idx; dp.w = h->w; dp.counts = h->counts; dp.offsets = h->offsets;
     dp.sorted_pair = h->sorted_pair; dp.pair_row = h->pair_row;
-    dp.act = h->act_ll;
+    dp.act = h->dec_act;
     dp.epoch = h->dec_epoch;
     dp.trace = h->trace;
     dp.status = h->status;
@@ -455,10 +455,10 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = dmalloc(&h->x_stage, (size_t)max_T * h->H, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->logits_stage, (size_t)max_T * h->E, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->y_stage, (size_t)max_T * h->H, &acc);
-    if (e == cudaSuccess) e = dmalloc(&h->act_ll, (size_t)fe::kDecMaxPairs * h->I, &acc);
-    if (e == cudaSuccess) e = cudaMemset(h->act_ll, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
-    if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count, &acc);
-    if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned) * (size_t)h->sm_count);
+    if (e == cudaSuccess) e = dmalloc(&h->dec_act, (size_t)fe::kDecMaxPairs * h->I, &acc);
+    if (e == cudaSuccess) e = cudaMemset(h->dec_act, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
+    if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count + 1, &acc);
+    if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned long long) * ((size_t)h->sm_count + 1));
     if (e == cudaSuccess) e = dmalloc(&h->grp_bh, (P / fe::kGroupChunk + 1) * (size_t)h->E, &acc);
     if (tc_shape_ok(h)) {
         if (e == cudaSuccess) e = dmalloc(&h->tc_x, (size_t)max_T * h->H, &acc);
