@@ -9,26 +9,30 @@
 // of the down weights overlaps the gate_up work and no launch boundary sits
 // inside the layer:
 //
-//   1. one bulk copy brings the T router-logit rows and the T x rows into
-//      shared memory; every CTA routes the T tokens itself (the rank of each
-//      logit among the E logits of its token, counted by all threads in
-//      parallel: rank < k selects it as slot rank, ties to the lower index)
-//      and groups the T*k pairs by expert; CTA 0 also publishes the routing;
+//   1. every CTA routes the T tokens itself (one warp per token: warp top-k
+//      over orderable keys, ties to the lower index, softmax over the k
+//      selected) and groups the T*k pairs by expert; CTA 0 publishes the
+//      routing; a bulk copy brings the x rows into shared memory meanwhile;
 //   2. from the number of distinct routed experts every CTA reads, in a
 //      table built at reserve time, its range of gate_up units (16 gate + 16
 //      up columns of one routed expert) and its range of down units (16
 //      output columns over all routed experts), balanced in bytes;
-//   3. one thread issues cp.async.bulk copies of ALL the CTA's weight bytes
-//      (both phases) into shared memory at once, one mbarrier per unit;
+//   3. one warp issues cp.async.bulk copies of the CTA's gate_up units into
+//      shared memory, one mbarrier per unit; the down units follow once the
+//      first gate_up unit has landed, so the bytes the exchange waits for
+//      come first;
 //   4. gate_up units: mma.m16n8k16 with the tokens of the unit's expert as
-//      the N columns (mma.cuh), SiLU(gate)*up, act written to global memory
-//      (L2) as 64-bit words holding the fp32 value and the launch's epoch tag;
-//   5. each CTA that owns down units reads act back, polling (bounded) until
-//      every word carries this launch's tag -- the data is its own ready
-//      flag, so no grid-wide barrier round trip is needed;
-//   6. down units: one warp per routed expert, its pairs as the N columns;
-//      the 16 outputs of every pair are combined in slot order, so y is
-//      written once, without atomics.
+//      the N columns (mma.cuh); the per-warp partials of all units wait in
+//      shared memory for one reduction, which writes SiLU(gate)*up to global
+//      memory (L2) as 64-bit words holding the fp32 value and the launch's tag;
+//      then the CTA adds 1 to an arrival counter;
+//   5. each CTA that owns down units polls the counter (one thread) until all
+//      but a few CTAs have arrived, then reads act back; a word carrying this
+//      launch's tag is this launch's value (the data is its own ready flag),
+//      and only words without it are read again;
+//   6. down units: the routed experts' quads spread over all warps, the
+//      pairs as the N columns; the 16 outputs of every pair are combined in
+//      slot order, so y is written once, without atomics.
 //
 // The kernel is launched with programmatic dependent launch: its CTAs load
 // only static data before griddepcontrol.wait, so the next layer's CTAs can
@@ -50,15 +54,9 @@ constexpr int kDecMaxE = 512;      // experts routed by one warp: 16 logits per 
 constexpr int kDecQuadsPerWarp = 4;   // gate_up quads whose x fragments a warp keeps in registers
 constexpr int kDecCandCap = 128;   // candidate keys per routing warp (in the gate_up partials' space)
 constexpr int kDecRedFloats = 4096;   // gate_up partials held before one reduction (also the down partials)
-#ifndef FE_DEC_ARRIVE_SLACK
-#define FE_DEC_ARRIVE_SLACK 16
-#endif
-constexpr int kDecArriveSlack = FE_DEC_ARRIVE_SLACK;   // producers still out when consumers start reading act
+constexpr int kDecArriveSlack = 16;   // producers still out when consumers start reading act
 constexpr int kDecMaxJobs = kDecRedFloats / (kDecWarps * 32);   // act columns one reduction serves
-#ifndef FE_DEC_DOWN_LATE
-#define FE_DEC_DOWN_LATE 1
-#endif
-constexpr int kDecDownLate = FE_DEC_DOWN_LATE;   // down copies issued once this many gate_up units landed
+constexpr int kDecDownLate = 1;   // down copies issued once this many gate_up units landed (0: at once)
 constexpr uint32_t kDevBarrierTimeout = 0x4;
 constexpr uint32_t kDevLoadTimeout = 0x8;
 
@@ -413,6 +411,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(uint32_t weight_bytes, 
     L.red = align16(L.shared + (uint32_t)sizeof(DecodeShared));
     L.dred = L.red;   // gate_up partials and down partials are never live together
     static_assert(kDecRedFloats >= kDecWarps * 32 * 8 && kDecRedFloats >= 8 * 4 * 32 * 4, "partials space");
+    static_assert(kDecRedFloats * 4 >= kDecWarps * kDecCandCap * 8, "routing candidates space");
     L.xs = L.red + 4u * kDecRedFloats;
     L.as = L.xs + 4u * (T + 1) * brow_words(H);
     L.xr = align16(L.as + 4u * (T * k + 1) * brow_words(I));
@@ -716,6 +715,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
                 const int key = T == 1 ? 0 : (dd << 8) + (nb - r0);
                 const uint32_t* brow = xs + (g < nvalid ? S.sp[nb + g] / k : T) * xrw;
                 float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                if (nq == QPW * kDecWarps) {
+                    // one pass, every quad of the warp valid: fixed offsets, no selects
+                    if (key != bkey) {
+#pragma unroll
+                        for (int i = 0; i < QPW; ++i) load_bfrag(brow, warp + kDecWarps * i, lane, bx[i]);
+                        bkey = key;
+                    }
+#pragma unroll
+                    for (int i = 0; i < QPW; ++i) quad_mma2_b(blk0, blk1, H, bx[i], warp + kDecWarps * i, lane, t0, t1);
+                } else
                 for (int pass = 0; pass < npass; ++pass) {
                     const int qbase = pass * QPW * kDecWarps + warp;
                     // quads past nq (H not a multiple of 64 QPW W) repeat quad qbase with a
@@ -801,21 +810,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         __syncthreads();
         const unsigned tag = S.tag;
         // warp pp stages pair pp: up to 16 chunks of two tagged words per lane, all
-        // requested at once, then only the ones not yet carrying this launch's tag again
+        // requested at once, then only the ones not yet carrying this launch's tag
+        // again; the values are kept, the tags only checked
         for (int pp = warp; pp < P && !S.abort; pp += kDecWarps) {
             const unsigned long long* src = p.act + (size_t)pp * I;
-            unsigned long long a0[16], a1[16];
+            float v0[16], v1[16];
             uint32_t pending = 0;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;
-                a0[i] = a1[i] = 0ull;
-                if (2 * r < I) ld_relaxed_2u64(src + 2 * r, a0[i], a1[i]);
+                unsigned long long w0 = 0ull, w1 = 0ull;
+                if (2 * r < I) {
+                    ld_relaxed_2u64(src + 2 * r, w0, w1);
+                    if ((unsigned)(w0 >> 32) != tag || (unsigned)(w1 >> 32) != tag) pending |= 1u << i;
+                }
+                v0[i] = __uint_as_float((uint32_t)w0);
+                v1[i] = __uint_as_float((uint32_t)w1);
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (2 * (lane + 32 * i) < I && ((unsigned)(a0[i] >> 32) != tag || (unsigned)(a1[i] >> 32) != tag))
-                    pending |= 1u << i;
             bool late = false;
             if (tracing && lane == 0 && pp == 0) stamp(trace, 22);
             int rounds = 0;
@@ -825,8 +836,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     if ((pending >> i) & 1u) {
-                        ld_relaxed_2u64(src + 2 * (lane + 32 * i), a0[i], a1[i]);
-                        if ((unsigned)(a0[i] >> 32) == tag && (unsigned)(a1[i] >> 32) == tag) pending &= ~(1u << i);
+                        unsigned long long w0, w1;
+                        ld_relaxed_2u64(src + 2 * (lane + 32 * i), w0, w1);
+                        if ((unsigned)(w0 >> 32) == tag && (unsigned)(w1 >> 32) == tag) pending &= ~(1u << i);
+                        v0[i] = __uint_as_float((uint32_t)w0);
+                        v1[i] = __uint_as_float((uint32_t)w1);
                     }
                 }
                 late = __any_sync(0xffffffffu, globaltimer_ns() - t_poll > p.timeout_ns);
@@ -841,8 +855,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             }
             float m = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                m = fmaxf(m, fmaxf(fabsf(__uint_as_float((uint32_t)a0[i])), fabsf(__uint_as_float((uint32_t)a1[i]))));
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, fmaxf(fabsf(v0[i]), fabsf(v1[i])));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             const int sh = fp16_shift(m);
@@ -851,9 +864,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = lane + 32 * i;
-                if (2 * r < I)
-                    as[pp * arw + bfrag_word(r)] = f32x2_to_f16x2_rn(__uint_as_float((uint32_t)a0[i]) * scl,
-                                                                    __uint_as_float((uint32_t)a1[i]) * scl);
+                if (2 * r < I) as[pp * arw + bfrag_word(r)] = f32x2_to_f16x2_rn(v0[i] * scl, v1[i] * scl);
             }
         }
         __syncthreads();
