@@ -19,6 +19,7 @@
 #include "pack.cuh"
 #include "route.cuh"
 #include "route_large.cuh"
+#include "stream.cuh"
 #include "tcgen05.cuh"
 
 namespace fe_host {
@@ -52,6 +53,7 @@ struct fe_moe_s {
     unsigned long long* dec_act = nullptr;  // fused decode: tagged act words by pair id
     int32_t* plan = nullptr;                // fused decode: work split per nd
     unsigned long long* dec_epoch = nullptr;  // fused decode: per-CTA launch counts, then the arrival counter
+    int32_t* sg_table = nullptr;            // streaming kernels: [2][SMs][4] work split
     unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
     // tensor-core path (tcgen05.cuh)
     bool tc_scales_ok = false;              // every group scale in the exact-f16 range
@@ -116,7 +118,7 @@ void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
-                    h->dec_act, h->dec_epoch, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
+                    h->dec_act, h->dec_epoch, h->sg_table, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
                     h->tc_tiles, h->tc_ntiles, h->grp_bh};
     for (void* p : ptrs)
         if (p) cudaFree(p);
@@ -125,6 +127,7 @@ void free_workspace(fe_moe_s* h)
     h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
     h->dec_act = nullptr;
     h->dec_epoch = nullptr;
+    h->sg_table = nullptr;
     h->plan = nullptr;
     h->tc_x = nullptr; h->tc_xshift = nullptr; h->tc_act = nullptr; h->tc_ashift = nullptr;
     h->tc_tiles = nullptr; h->tc_ntiles = nullptr;
@@ -251,6 +254,58 @@ size_t tc_max_tiles(const fe_moe_s* h, size_t P)
     return (P + fe::kTcN - 1) / fe::kTcN + std::min((size_t)h->E, P);
 }
 
+// Streaming kernels: 8-token blocks staged at once (gate_up rows are 4 times
+// the bytes of down rows at the 30B-like shape).
+constexpr int kSgGateUpBlocks = 2;
+constexpr int kSgDownBlocks = 8;
+constexpr int kSgStaticReserve = 256;   // static shared bytes of the streaming kernels, rounded up
+
+struct SgPlan {
+    int slots = 0, chunk = 0;
+    size_t smem = 0;
+};
+
+// Largest token chunk (down to 8) that leaves room for min_slots ring slots,
+// then as many slots as fit (at most kSgMaxSlots); slots = 0 if nothing fits.
+SgPlan sg_plan(const fe_moe_s* h, bool gate_up, int K, uint32_t unit_bytes, int max_blocks, int min_slots, int slot_step)
+{
+    const size_t limit = (size_t)h->smem_optin - kSgStaticReserve;
+    SgPlan best;
+    for (int want = min_slots; want >= 2 && best.slots == 0; want = want > 2 ? want - 1 : 1) {
+        for (int chunk = 8 * max_blocks; chunk >= 8; chunk -= 8) {
+            int slots = 0;
+            for (int r = fe::kSgMaxSlots / slot_step * slot_step; r >= want; r -= slot_step)
+                if (fe::sg_smem_layout(gate_up, K, unit_bytes, r, chunk).total <= limit) {
+                    slots = r;
+                    break;
+                }
+            if (slots) {
+                best.slots = slots;
+                best.chunk = chunk;
+                best.smem = fe::sg_smem_layout(gate_up, K, unit_bytes, slots, chunk).total;
+                break;
+            }
+        }
+    }
+    return best;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 cudaError_t configure_kernels(const fe_moe_s* h)
 {
     const int optin = h->smem_optin;
@@ -262,6 +317,13 @@ cudaError_t configure_kernels(const fe_moe_s* h)
         e = cudaFuncSetAttribute(fe::tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fe::tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    // (the streaming kernels hold a little static shared state besides)
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fe::sg_kernel<true, kSgGateUpBlocks>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 optin - kSgStaticReserve);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fe::sg_kernel<false, kSgDownBlocks>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 optin - kSgStaticReserve);
     return e;
 }
 
@@ -300,10 +362,89 @@ fe_status gemv_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s
     return FE_OK;
 }
 
+// Plans of the two streaming kernels and the work-split arguments the grouping
+// step uses to fill the range table; false when a ring does not fit.
+struct SgSetup {
+    SgPlan gu, dn;
+    fe::SgSplit split{};
+};
+
+bool stream_setup(const fe_moe_s* h, int T, SgSetup& st)
+{
+    const uint32_t gu_unit = 2u * fe::block_bytes(h->H), dn_unit = fe::block_bytes(h->I);
+    // an expert has at most T pairs: no chunk longer than that
+    const int tb = (T + 7) / 8;
+    st.gu = sg_plan(h, true, h->H, gu_unit, std::min(kSgGateUpBlocks, tb), 3, 1);
+    st.dn = sg_plan(h, false, h->I, dn_unit, std::min(kSgDownBlocks, tb), 16, 1);
+    if (st.gu.slots == 0 || st.dn.slots < fe::kSgComputeWarps) return false;
+    fe::SgSplit& sp = st.split;
+    sp.table = h->sg_table;
+    sp.G = h->sm_count;
+    // cost of a unit in ~100-cycle units: its bytes at the per-SM share of HBM,
+    // the A conversion per chunk, the MMAs per 8-token block, the restaging of
+    // a chunk's rows
+    const int K[2] = {h->H, h->I};
+    const SgPlan* pl[2] = {&st.gu, &st.dn};
+    const uint32_t ub[2] = {gu_unit, dn_unit};
+    sp.n_units[0] = h->I / 16;
+    sp.n_units[1] = h->H / 16;
+    for (int ph = 0; ph < 2; ++ph) {
+        sp.chunk[ph] = pl[ph]->chunk;
+        sp.c_bytes[ph] = std::max(1, (int)(ub[ph] / 2300));
+        sp.c_chunk[ph] = std::max(1, K[ph] / 320);
+        sp.c_block[ph] = std::max(1, K[ph] / 340);
+        sp.c_restage[ph] = std::max(1, (int)((size_t)pl[ph]->chunk * K[ph] * 2 / 6400));
+    }
+    return true;
+}
+
+// Moderate-T path on the streaming kernels: gate_up units (x rows staged as
+// fp16 in the kernel, SwiGLU into act), then down units (act rows likewise,
+// into o), each CTA on the range the grouping step put in the table.  The
+// routing and grouping ran before; the ordered combine runs after.
+fe_status stream_path(fe_moe_s* h, const uint16_t* x, int k, const SgSetup& st, cudaStream_t s)
+{
+    fe::SgParams sp{};
+    sp.offsets = h->offsets;
+    sp.active = h->active;
+    sp.n_active = h->n_active;
+    sp.sorted_pair = h->sorted_pair;
+    sp.top_k = k;
+    sp.status = h->status;
+    sp.timeout_ns = 200ull * 1000 * 1000;
+    sp.trace = h->trace;
+    // gate_up: K = H, units of 16 gate + 16 up columns
+    sp.blocks = h->gu_blocks;
+    sp.K = h->H;
+    sp.n_units = h->I / 16;
+    sp.unit_bytes = 2u * fe::block_bytes(h->H);
+    sp.N_out = h->I;
+    sp.bsrc = x;
+    sp.out = h->act;
+    sp.slots = st.gu.slots;
+    sp.chunk = st.gu.chunk;
+    sp.range = h->sg_table;
+    FE_CUDA_TRY(launch_pdl(fe::sg_kernel<true, kSgGateUpBlocks>, dim3(h->sm_count), dim3(fe::kSgThreads), st.gu.smem, s, sp));
+    // down: K = I, units of 16 output columns, one warp each
+    sp.blocks = h->dn_blocks;
+    sp.K = h->I;
+    sp.n_units = h->H / 16;
+    sp.unit_bytes = fe::block_bytes(h->I);
+    sp.N_out = h->H;
+    sp.bsrc = h->act;
+    sp.out = h->o;
+    sp.slots = st.dn.slots;
+    sp.chunk = st.dn.chunk;
+    sp.range = h->sg_table + 4 * (size_t)h->sm_count;
+    sp.trace = h->trace ? h->trace + 8 * (size_t)h->sm_count : nullptr;
+    FE_CUDA_TRY(launch_pdl(fe::sg_kernel<false, kSgDownBlocks>, dim3(h->sm_count), dim3(fe::kSgThreads), st.dn.smem, s, sp));
+    return FE_OK;
+}
+
 // Router + grouping outputs (idx, w, counts, offsets, sorted_pair, pair_row,
 // active, n_active, max_count) for the non-fused paths: the single-CTA kernel
 // for a few tokens, the GPU-wide kernels for many.
-fe_status route_and_group(fe_moe_s* h, const float* logits, int T, int k, cudaStream_t s)
+fe_status route_and_group(fe_moe_s* h, const float* logits, int T, int k, const fe::SgSplit* split, cudaStream_t s)
 {
     const int P = T * k;
     fe::RouteParams rp{};
@@ -311,13 +452,15 @@ fe_status route_and_group(fe_moe_s* h, const float* logits, int T, int k, cudaSt
     rp.idx = h->idx; rp.w = h->w; rp.counts = h->counts; rp.offsets = h->offsets;
     rp.sorted_pair = h->sorted_pair; rp.pair_row = h->pair_row; rp.active = h->active;
     rp.n_active = h->n_active; rp.max_count = h->max_count; rp.status = h->status;
+    if (split) rp.split = *split;
     if (T >= kRouteLargeTokens && fe::route_large_ok(h->E, k)) {
         const int nblk = (P + fe::kGroupChunk - 1) / fe::kGroupChunk;
         fe::route_tokens_kernel<<<(T + fe::kRouteWarps - 1) / fe::kRouteWarps, fe::kRouteWarps * 32, 0, s>>>(rp);
         fe::group_hist_kernel<<<nblk, fe::kGroupThreads, sizeof(int32_t) * h->E, s>>>(h->idx, P, h->E, h->grp_bh);
-        fe::group_scan_kernel<<<1, 1024, 2 * sizeof(int32_t) * h->E, s>>>(h->grp_bh, nblk, h->E, h->counts,
+        const size_t scan_smem = sizeof(int32_t) * 2 * (size_t)((h->E + 1) & ~1) + sizeof(long long) * (2 * ((size_t)h->E + 1) + 32);
+        fe::group_scan_kernel<<<1, 1024, scan_smem, s>>>(h->grp_bh, nblk, h->E, h->counts,
                                                                           h->offsets, h->active, h->n_active,
-                                                                          h->max_count);
+                                                                          h->max_count, rp.split);
         fe::group_scatter_kernel<<<nblk, fe::kGroupThreads, sizeof(int32_t) * h->E * (fe::kGroupThreads / 32 + 1),
                                    s>>>(h->idx, P, h->E, h->grp_bh, h->sorted_pair, h->pair_row, h->status);
     } else {
@@ -458,13 +601,16 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = dmalloc(&h->dec_act, (size_t)fe::kDecMaxPairs * h->I, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->dec_act, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
     if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count + 1, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->sg_table, 8 * (size_t)h->sm_count, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned long long) * ((size_t)h->sm_count + 1));
     if (e == cudaSuccess) e = dmalloc(&h->grp_bh, (P / fe::kGroupChunk + 1) * (size_t)h->E, &acc);
+    // fp16 token and act rows (row-major for the tensor-core tiles, fragment
+    // order for the streaming kernels: each forward writes before it reads)
+    if (e == cudaSuccess) e = dmalloc(&h->tc_x, (size_t)max_T * h->H, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->tc_xshift, (size_t)max_T, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->tc_act, P * h->I, &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->tc_ashift, P, &acc);
     if (tc_shape_ok(h)) {
-        if (e == cudaSuccess) e = dmalloc(&h->tc_x, (size_t)max_T * h->H, &acc);
-        if (e == cudaSuccess) e = dmalloc(&h->tc_xshift, (size_t)max_T, &acc);
-        if (e == cudaSuccess) e = dmalloc(&h->tc_act, P * h->I, &acc);
-        if (e == cudaSuccess) e = dmalloc(&h->tc_ashift, P, &acc);
         if (e == cudaSuccess) e = dmalloc(&h->tc_tiles, 3 * tc_max_tiles(h, P), &acc);
         if (e == cudaSuccess) e = dmalloc(&h->tc_ntiles, 1, &acc);
     }
@@ -575,14 +721,20 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
         if (h->path == FE_PATH_FUSED_DECODE) return FE_ERR_UNSUPPORTED;
     }
 
+    const bool use_tc = tc_ok && (h->path == FE_PATH_TCGEN05 || (h->path == FE_PATH_AUTO && P >= kTcAutoPairs));
+    SgSetup sg;
+    const bool use_stream = !use_tc && stream_setup(h, T, sg);
     {
-        const fe_status rs = route_and_group(h, router_logits, T, top_k, s);
+        const fe_status rs = route_and_group(h, router_logits, T, top_k, use_stream ? &sg.split : nullptr, s);
         if (rs != FE_OK) return rs;
     }
-
-    const bool use_tc = tc_ok && (h->path == FE_PATH_TCGEN05 || (h->path == FE_PATH_AUTO && P >= kTcAutoPairs));
-    fe_status st = use_tc ? tcgen05_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s)
-                          : gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
+    fe_status st = FE_OK;
+    if (use_tc)
+        st = tcgen05_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
+    else if (use_stream)
+        st = stream_path(h, static_cast<const uint16_t*>(x_bf16), top_k, sg, s);
+    else
+        st = gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
     if (st != FE_OK) return st;
 
     dim3 cgrid((h->H / 2 + 255) / 256, T);

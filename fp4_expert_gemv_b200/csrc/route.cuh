@@ -9,6 +9,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "stream.cuh"   // SgSplit, sg_plan_ranges
 
 namespace fe {
 
@@ -25,6 +26,7 @@ struct RouteParams {
     int32_t* n_active;     // [1]
     int32_t* max_count;    // [1]      largest per-expert count
     uint32_t* status;
+    SgSplit split;         // work split of the streaming kernels, filled when split.table is set
 };
 
 // (value, index) order of the router: larger logit first, equal logits by
@@ -39,6 +41,8 @@ constexpr int kRouteMaxPerLane = 32;  // E <= 1024
 constexpr int kRouteMaxThreads = 512;
 
 // Dynamic shared memory: cnt[E] | cursor[E] | wcnt[nwarps][E]
+__host__ __device__ inline int route_plan_offset(int E, int nthreads);
+
 __global__ void __launch_bounds__(kRouteMaxThreads) route_group_kernel(RouteParams p)
 {
     extern __shared__ int32_t sm[];
@@ -142,6 +146,10 @@ __global__ void __launch_bounds__(kRouteMaxThreads) route_group_kernel(RoutePara
         }
     }
     __syncthreads();
+    if (p.split.table) {
+        long long* scratch = reinterpret_cast<long long*>(sm + route_plan_offset(E, nthreads));
+        sg_plan_ranges(p.split, p.counts, p.active, *p.n_active, scratch);
+    }
 
     // stable scatter, one chunk of nthreads pairs at a time: the position of a
     // pair is its expert's cursor + pairs of that expert in earlier warps of the
@@ -176,6 +184,12 @@ __global__ void __launch_bounds__(kRouteMaxThreads) route_group_kernel(RoutePara
     }
 }
 
-inline size_t route_smem_bytes(int E, int nthreads) { return sizeof(int32_t) * (size_t)E * (2 + nthreads / 32); }
+// Shared memory of route_group_kernel: counts, cursors, per-warp counts, then
+// (8-byte aligned) the scratch of the streaming kernels' work split.
+__host__ __device__ inline int route_plan_offset(int E, int nthreads) { return (E * (2 + nthreads / 32) + 1) & ~1; }
+inline size_t route_smem_bytes(int E, int nthreads)
+{
+    return sizeof(int32_t) * (size_t)route_plan_offset(E, nthreads) + sizeof(long long) * (2 * ((size_t)E + 1) + 32);
+}
 
 }  // namespace fe

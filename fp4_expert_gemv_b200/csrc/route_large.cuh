@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_hist_kernel(const int32_t
 // active list, n_active, max_count.  Thread e walks the blocks of expert e.
 __global__ void __launch_bounds__(1024) group_scan_kernel(int32_t* bh, int nblocks, int E, int32_t* counts,
                                                           int32_t* offsets, int32_t* active, int32_t* n_active,
-                                                          int32_t* max_count)
+                                                          int32_t* max_count, SgSplit split)
 {
     extern __shared__ int32_t grp_scan_sm[];   // [E] counts, then [E] scan
     int32_t* sc = grp_scan_sm;
@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(1024) group_scan_kernel(int32_t* bh, int nbloc
         *max_count = mx;
     }
     __syncthreads();
+    if (split.table) sg_plan_ranges(split, counts, active, *n_active, reinterpret_cast<long long*>(sc + 2 * ((E + 1) & ~1)));
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = sc[E + e];
         for (int b = 0; b < nblocks; ++b) {

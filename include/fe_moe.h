@@ -128,7 +128,8 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
 
 /* Compute paths of fe_moe_forward. */
 #define FE_PATH_AUTO 0          /* chosen per call from T, top_k and the shape */
-#define FE_PATH_GEMV 1          /* routing + grouped mma.sync gate_up and down + combine (any T) */
+#define FE_PATH_GEMV 1          /* routing + grouped mma.sync gate_up and down + combine (any T): persistent
+                                   streaming kernels, or one CTA per unit when their ring does not fit */
 #define FE_PATH_TCGEN05 2       /* routing + tcgen05 tensor-core tiles + combine (large T; I % 128 == 0,
                                    H % 256 == 0, scales in the exact-f16 range) */
 #define FE_PATH_FUSED_DECODE 3  /* one cooperative kernel for the whole layer (T * top_k <= 16) */
@@ -150,7 +151,10 @@ fe_status fe_moe_last_forward_info(fe_moe_t h, int* path, int* kernels);
  * unit: mma done, partials shared, reduced, done, 3 gate_up done, 14 down
  * weights landed, 4 act read back, 6 first down unit landed, 20 / 7 / 21
  * first down unit: mma done, partials shared, reduced, 5 end).  Slots a
- * CTA does not reach keep their old contents.  NULL switches it off. */
+ * CTA does not reach keep their old contents.  The streaming kernels of the
+ * moderate-T path write [2][number of SMs][8] instead (gate_up, then down;
+ * per CTA clock64 at start, range known, first unit landed, end; its unit
+ * count; %globaltimer at start and end).  NULL switches it off. */
 fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf);
 
 /* Human-readable text of a status code (static storage). */
