@@ -33,7 +33,7 @@ WORKLOAD = "decode_e128_t1"
 LAYERS = 48
 NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126e6
-KERNEL_NAMES = {1: "grouped mma.sync projections (routing, gate_up, down, combine)",
+KERNEL_NAMES = {1: "streaming mma.sync projections sg_kernel (routing, gate_up, down, combine)",
                 2: "tensor-core tiles tc_gemm_kernel (gate_up + down) with routing, row conversion and combine",
                 3: "decode_kernel (whole layer, one cooperative launch); per-launch time = step time / layers"}
 PREFILL_METRIC = "MoE-layer prefill tokens/s and tensor-core TFLOP/s at T=4096"
