@@ -82,6 +82,13 @@ FE_DEV float silu_mul(float g, float u)
 // about -88, where exp(-g) overflows).
 FE_DEV float silu_mul_fast(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// Two floats -> bf16x2 (first in the low half), round to nearest even.
+FE_DEV uint32_t bf16x2_rn(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 FE_DEV unsigned long long globaltimer_ns()
 {
     unsigned long long t;

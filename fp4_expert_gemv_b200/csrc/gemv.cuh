@@ -127,8 +127,10 @@ inline size_t gemv_smem_bytes(int K, int TW, int nthreads)
            sizeof(int) * NT + 16;
 }
 
-// y[t][h] = sum_j w[t][j] * o[pair_row[t*k + j]][h], slot order, fp32, bf16 once.
-__global__ void combine_kernel(const float* __restrict__ o, const float* __restrict__ w,
+// y[t][h] = sum_j w[t][j] * o[pair_row[t*k + j]][h], slot order, fp32 sums, bf16 once;
+// o is fp32, or bf16 (O_BF16) as the tensor-core down tiles leave it.
+template <bool O_BF16>
+__global__ void combine_kernel(const void* __restrict__ o, const float* __restrict__ w,
                                const int32_t* __restrict__ pair_row, int H, int k, __nv_bfloat16* __restrict__ y)
 {
     const int t = blockIdx.y;
@@ -137,7 +139,13 @@ __global__ void combine_kernel(const float* __restrict__ o, const float* __restr
     float a0 = 0.0f, a1 = 0.0f;
     for (int j = 0; j < k; ++j) {
         const float wj = w[(size_t)t * k + j];
-        const float2 v = *reinterpret_cast<const float2*>(o + (size_t)pair_row[(size_t)t * k + j] * H + h);
+        const size_t at = (size_t)pair_row[(size_t)t * k + j] * H + h;
+        float2 v;
+        if (O_BF16) {
+            v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(o) + at));
+        } else {
+            v = *reinterpret_cast<const float2*>(static_cast<const float*>(o) + at);
+        }
         a0 = fmaf(wj, v.x, a0);
         a1 = fmaf(wj, v.y, a1);
     }

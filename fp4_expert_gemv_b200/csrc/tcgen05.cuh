@@ -425,11 +425,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
             }
             __syncthreads();
             const int nrows = min(32, rows - c0);
-            constexpr int V4 = OC / 4;   // float4 per token row
-            for (int idx = tid; idx < nrows * V4; idx += kTcThreads) {
-                const int n = idx / V4, v = idx - n * V4;
-                const float4 val = reinterpret_cast<const float4*>(st + n * OC)[v ^ ((n & 16) >> 2)];
-                reinterpret_cast<float4*>(p.out + (size_t)(pos0 + c0 + n) * p.out_ld + ocol0)[v] = val;
+            if (GATE_UP) {
+                constexpr int V4 = OC / 4;   // float4 per token row
+                for (int idx = tid; idx < nrows * V4; idx += kTcThreads) {
+                    const int n = idx / V4, v = idx - n * V4;
+                    const float4 val = reinterpret_cast<const float4*>(st + n * OC)[v ^ ((n & 16) >> 2)];
+                    reinterpret_cast<float4*>(p.out + (size_t)(pos0 + c0 + n) * p.out_ld + ocol0)[v] = val;
+                }
+            } else {
+                // o as bf16 (8 values per 16-byte store): the ordered combine reads half the bytes
+                constexpr int V8 = OC / 8;
+                uint16_t* o16 = reinterpret_cast<uint16_t*>(p.out);
+                for (int idx = tid; idx < nrows * V8; idx += kTcThreads) {
+                    const int n = idx / V8, v = idx - n * V8;
+                    const float4* rowp = reinterpret_cast<const float4*>(st + n * OC);
+                    const float4 a = rowp[(2 * v) ^ ((n & 16) >> 2)], b = rowp[(2 * v + 1) ^ ((n & 16) >> 2)];
+                    uint4 w;
+                    w.x = bf16x2_rn(a.x, a.y);
+                    w.y = bf16x2_rn(a.z, a.w);
+                    w.z = bf16x2_rn(b.x, b.y);
+                    w.w = bf16x2_rn(b.z, b.w);
+                    reinterpret_cast<uint4*>(o16 + (size_t)(pos0 + c0 + n) * p.out_ld + ocol0)[v] = w;
+                }
             }
             // the next 32 tokens go to the other staging tile: no barrier needed here
         }
