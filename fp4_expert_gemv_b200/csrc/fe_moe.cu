@@ -498,7 +498,8 @@ fe_status tcgen05_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_
     tp.out_ld = h->I;
     fe::tc_gemm_kernel<true><<<dim3(h->I / 128, max_tiles), fe::kTcThreads, fe::tc_smem_bytes(), s>>>(tp);
     FE_CUDA_TRY(cudaGetLastError());
-    fe::tc_rows_to_f16_kernel<false><<<(P + 7) / 8, 256, 0, s>>>(h->act, P, h->I, h->tc_act, h->tc_ashift);
+    // act was left as bf16 by the gate_up tiles
+    fe::tc_rows_to_f16_kernel<true><<<(P + 7) / 8, 256, 0, s>>>(h->act, P, h->I, h->tc_act, h->tc_ashift);
     tp.blocks = h->dn_blocks;
     tp.K = h->I;
     tp.blocks_per_expert = h->H / 16;

@@ -19,8 +19,8 @@
 //     memory (TMEM) and commits each chunk to an mbarrier, so the loads and the
 //     dequantisation of later chunks overlap the tensor-core work;
 //   * the epilogue reads TMEM with tcgen05.ld: gate_up applies SiLU(gate)*up
-//     (gate and up columns sit in adjacent rows) and writes act (fp32), down
-//     writes o (fp32) for the ordered combine.
+//     (gate and up columns sit in adjacent rows) and writes act, down writes
+//     o for the ordered combine, both as bf16 (the sums are fp32 until then).
 //
 // No TMA and no cluster features are used: every load is this CTA's own.
 #pragma once
@@ -65,7 +65,7 @@ struct TcParams {
     const int32_t* bshift;     // power-of-two shift of each B row (token or position)
     const int32_t* sorted_pair;  // gate_up: the token of a sorted position is sorted_pair[pos] / top_k
     int top_k;
-    float* out;                // gate_up: act [P][I]; down: o [P][H]; rows by sorted position
+    float* out;                // gate_up: act [P][I]; down: o [P][H]; bf16, rows by sorted position
     int out_ld;                // I or H
     uint32_t* status;
     unsigned long long timeout_ns;
@@ -425,15 +425,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(TcParams p)
             }
             __syncthreads();
             const int nrows = min(32, rows - c0);
-            if (GATE_UP) {
-                constexpr int V4 = OC / 4;   // float4 per token row
-                for (int idx = tid; idx < nrows * V4; idx += kTcThreads) {
-                    const int n = idx / V4, v = idx - n * V4;
-                    const float4 val = reinterpret_cast<const float4*>(st + n * OC)[v ^ ((n & 16) >> 2)];
-                    reinterpret_cast<float4*>(p.out + (size_t)(pos0 + c0 + n) * p.out_ld + ocol0)[v] = val;
-                }
-            } else {
-                // o as bf16 (8 values per 16-byte store): the ordered combine reads half the bytes
+            {
+                // act (gate_up) and o (down) as bf16, 8 values per 16-byte store: the next
+                // kernel (row conversion, ordered combine) reads half the bytes
                 constexpr int V8 = OC / 8;
                 uint16_t* o16 = reinterpret_cast<uint16_t*>(p.out);
                 for (int idx = tid; idx < nrows * V8; idx += kTcThreads) {
@@ -506,7 +500,7 @@ __global__ void __launch_bounds__(1024) tc_tiles_kernel(const int32_t* counts, c
 }
 
 // Rows of n values -> f16 scaled by 2^-s with s = fp16_shift(row max); one warp
-// per row.  BF16: bf16 bits (x); otherwise fp32 (act).
+// per row.  BF16: bf16 bits (x, and act as the gate_up tiles leave it); otherwise fp32.
 template <bool BF16>
 __global__ void tc_rows_to_f16_kernel(const void* src, int rows, int n, uint16_t* dst, int32_t* shift)
 {
