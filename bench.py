@@ -40,7 +40,8 @@ PREFILL_METRIC = "MoE-layer prefill tokens/s and tensor-core TFLOP/s at T=4096"
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu
 # captures summarised in profiles/ (recaptured whenever that kernel changes)
 TRAFFIC = {"decode_e128_t1": (21379072, "decode_kernel", "profiles/decode_kernel_decode_e128_t1.md"),
-           "prefill_e128_t4096": (343674624, "tc_gemm_kernel gate_up", "profiles/tc_gemm_kernel_prefill_e128_t4096.md")}
+           "prefill_e128_t4096": (299220224, "tc_gemm_kernel gate_up", "profiles/tc_gemm_kernel_prefill_e128_t4096.md"),
+           "decode_e128_t64_zipf": (95570432, "sg_kernel gate_up", "profiles/sg_kernel_decode_e128_t64_zipf.md")}
 BYTES_PER_EXPERT = lambda H, I: (H // 2) * 2 * I + (H // 32) * 2 * I * 2 + (I // 2) * H + (I // 32) * H * 2  # noqa: E731
 
 
