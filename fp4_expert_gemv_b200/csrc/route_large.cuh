@@ -74,27 +74,58 @@ __global__ void __launch_bounds__(1024) group_scan_kernel(int32_t* bh, int nbloc
                                                           int32_t* max_count, SgSplit split)
 {
     extern __shared__ int32_t grp_scan_sm[];   // [E] counts, then [E] scan
+    __shared__ int wsum[32], wact[32], wmx[32];
     int32_t* sc = grp_scan_sm;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int nthreads = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (E + nthreads - 1) / nthreads, e0 = tid * per;
+    // each thread: the counts of a contiguous run of experts
+    int loc = 0, lact = 0, lmx = 0;
+    for (int e = e0; e < e0 + per && e < E; ++e) {
         int c = 0;
         for (int b = 0; b < nblocks; ++b) c += bh[(size_t)b * E + e];
         sc[e] = c;
+        loc += c;
+        lact += c > 0;
+        lmx = max(lmx, c);
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0, na = 0, mx = 0;
-        for (int e = 0; e < E; ++e) {
-            const int c = sc[e];
-            sc[E + e] = run;
-            offsets[e] = run;
-            counts[e] = c;
-            if (c > 0) active[na++] = e;
-            mx = max(mx, c);
-            run += c;
+    // block scans of the pair counts and of the active flags, and the largest count
+    int incl = loc, iact = lact, mx = lmx;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, incl, o), c = __shfl_up_sync(0xffffffffu, iact, o);
+        if (lane >= o) {
+            incl += a;
+            iact += c;
         }
-        offsets[E] = run;
-        *n_active = na;
-        *max_count = mx;
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 31) {
+        wsum[warp] = incl;
+        wact[warp] = iact;
+    }
+    if (lane == 0) wmx[warp] = mx;
+    __syncthreads();
+    int base = 0, abase = 0, tmax = 0;
+    for (int w = 0; w < nthreads / 32; ++w) {
+        if (w < warp) {
+            base += wsum[w];
+            abase += wact[w];
+        }
+        tmax = max(tmax, wmx[w]);
+    }
+    int run = base + incl - loc, arun = abase + iact - lact;
+    for (int e = e0; e < e0 + per && e < E; ++e) {
+        const int c = sc[e];
+        sc[E + e] = run;
+        offsets[e] = run;
+        counts[e] = c;
+        if (c > 0) active[arun++] = e;
+        run += c;
+    }
+    if (tid == nthreads - 1) {
+        offsets[E] = base + incl;
+        *n_active = abase + iact;
+        *max_count = tmax;
     }
     __syncthreads();
     if (split.table) sg_plan_ranges(split, counts, active, *n_active, reinterpret_cast<long long*>(sc + 2 * ((E + 1) & ~1)));
