@@ -219,6 +219,25 @@ def test_tcgen05_tiles(torch_cuda):
     assert st == fe.FE_OK and bits == 0
 
 
+def test_streaming_chunks(torch_cuda):
+    """Streaming (moderate-T) kernels with more tokens on one expert than one
+    staged chunk holds: gate_up makes one pass over the expert's units per
+    16-row chunk, down stages several 64-row chunks per round of units."""
+    import fp4_expert_gemv_b200 as fe
+    E, H, I, seed, T = 8, 256, 128, 3, 200
+    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=2, source="host")
+    osd = harness.OracleSide(E, H, I, seed)
+    x = synth.activations_bf16(60, T, H)
+    lg = synth.router_logits(60, T, E)
+    lg[:, 2] += 100.0          # every token's first expert: 200 pairs on expert 2
+    lg[: T // 2, 6] += 50.0    # half the tokens' second expert: 100 pairs on expert 6
+    rows = np.arange(0, T, 7)
+    run_and_check(gl, osd, x, lg, 2, sample=rows, what="one expert over many chunks")
+    assert gl.layer.last_forward_info()[0] == fe.PATH_GEMV
+    st, bits = gl.layer.status()
+    assert st == fe.FE_OK and bits == 0
+
+
 @pytest.mark.parametrize("path", ["auto", "gemv"])
 def test_edge_cases(torch_cuda, path):
     torch = torch_cuda
