@@ -738,7 +738,7 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
         st = gemv_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
     if (st != FE_OK) return st;
 
-    dim3 cgrid((h->H / 2 + 255) / 256, T);
+    dim3 cgrid((h->H / 8 + 255) / 256, T);
     if (use_tc)   // the tensor-core down tiles leave o as bf16
         fe::combine_kernel<true><<<cgrid, 256, 0, s>>>(h->o, h->w, h->pair_row, h->H, top_k,
                                                         static_cast<__nv_bfloat16*>(y_bf16));
@@ -1023,7 +1023,7 @@ fe_status fe_moe_forward_noalloc(int E, int H, int I, const uint8_t* gate_up_cod
                  : launch_canonical<4, false>(cp, max_active * cp.n_tiles, threads, s);
     if (e != cudaSuccess) return record_cuda(e, "noalloc down launch");
 
-    dim3 cgrid((H / 2 + 255) / 256, T);
+    dim3 cgrid((H / 8 + 255) / 256, T);
     fe::combine_kernel<false><<<cgrid, 256, 0, s>>>(reinterpret_cast<const float*>(scr + L.o), rp.w, rp.pair_row, H, top_k,
                                               static_cast<__nv_bfloat16*>(y_bf16));
     FE_CUDA_TRY(cudaGetLastError());

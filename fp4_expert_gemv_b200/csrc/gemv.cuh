@@ -133,23 +133,36 @@ template <bool O_BF16>
 __global__ void combine_kernel(const void* __restrict__ o, const float* __restrict__ w,
                                const int32_t* __restrict__ pair_row, int H, int k, __nv_bfloat16* __restrict__ y)
 {
+    // 8 consecutive outputs per thread: 16-byte loads of o (the library's own buffer);
+    // y (the caller's) is written in 4-byte pairs, as before
     const int t = blockIdx.y;
-    const int h = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    const int h = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
     if (h >= H) return;
-    float a0 = 0.0f, a1 = 0.0f;
+    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
     for (int j = 0; j < k; ++j) {
         const float wj = w[(size_t)t * k + j];
         const size_t at = (size_t)pair_row[(size_t)t * k + j] * H + h;
-        float2 v;
+        float v[8];
         if (O_BF16) {
-            v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(o) + at));
+            const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + at);
+            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = __uint_as_float(qw[i] << 16);
+                v[2 * i + 1] = __uint_as_float(qw[i] & 0xffff0000u);
+            }
         } else {
-            v = *reinterpret_cast<const float2*>(static_cast<const float*>(o) + at);
+            const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + at);
+            const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + at + 4);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
         }
-        a0 = fmaf(wj, v.x, a0);
-        a1 = fmaf(wj, v.y, a1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
     }
-    *reinterpret_cast<__nv_bfloat162*>(y + (size_t)t * H + h) = __floats2bfloat162_rn(a0, a1);
+    uint32_t* yw = reinterpret_cast<uint32_t*>(y + (size_t)t * H + h);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) yw[i] = bf16x2_rn(acc[2 * i], acc[2 * i + 1]);
 }
 
 }  // namespace fe
