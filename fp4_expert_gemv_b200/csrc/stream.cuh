@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kSgThreads, 1) sg_kernel(SgParams p)
     __shared__ SgShared S;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2;
     const int K = p.K, rw = brow_words(K), C = p.chunk, R = p.slots;
-    constexpr int UB = 1;   // units per copy batch (one full barrier each); R is a multiple of UB
+    constexpr int UB = 1;   // units per copy batch (one full barrier per batch); R is a multiple of UB
     const SgSmem L = sg_smem_layout(GATE_UP, K, p.unit_bytes, R, C);
     uint8_t* ring = sg_sm + L.ring;
     const uint32_t full0 = sg_smem(sg_sm + L.full), empty0 = sg_smem(sg_sm + L.empty);
@@ -335,12 +335,12 @@ __global__ void __launch_bounds__(kSgThreads, 1) sg_kernel(SgParams p)
     if (warp == kSgComputeWarps) {
         // ---- producer: the range's units into the ring as slots free up, in the
         // order the compute warps take them (gate_up: one pass over an expert's
-        // units per chunk of its token rows).  Units go in batches of UB (down: 8
-        // units of 4.6-7 KB, so that consecutive units of an expert travel as one
-        // copy; gate_up: 1), one full barrier per batch, one empty barrier per
-        // unit.  Every lane walks the same sequence; lane l takes the l-th unit of
-        // each batch and waits for its slot; the first unit of each run of
-        // consecutive units issues the run's copy. ---------------------------------
+        // units per chunk of its token rows).  The walk is written for batches of
+        // UB units (one full barrier per batch, runs of consecutive units of an
+        // expert as one copy, one empty barrier per unit); UB is 1, one copy and
+        // one full barrier per unit, since 8-unit batches of down units made a
+        // wait time out (cause not found).  Every lane walks the same sequence;
+        // lane l takes the l-th unit of each batch and waits for its slot. ---------
         int a = S.a0, j = S.j0, left = nu, ch = 0, seg_i = 0, pu = 0;
         int seg_n = 0, passes = 1, e = 0;
         auto enter_segment = [&]() {
