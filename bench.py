@@ -1,20 +1,31 @@
 #!/usr/bin/env python3
-"""Benchmark of the packed FP4 MoE decode layer (fe_moe) on B200.
+"""Benchmark of the packed FP4 MoE layer (fe_moe) on B200.
 
-Workload: a stack of 48 independent decode layers shaped like a 30B-A3B
-128-expert model (E=128, H=2048, I=768, top-8, T=1 token), each with its own
-seeded weights (seed 1000 + layer), captured as one CUDA graph; the output of
-layer l is the input of layer l+1, the router logits of every layer are
-seeded inputs.  One step = one replay of the graph = 48 layer forwards.  The
-stack touches 48 x 21.2 MB = 1.02 GB of expert weights per step, more than
-the 126 MB L2, so no step finds its weights in L2 from the step before.
+Headline workload: a stack of 48 independent decode layers shaped like a
+30B-A3B 128-expert model (E=128, H=2048, I=768, top-8, T=1 token), each with
+its own seeded weights, x and router logits (seed 1000 + layer), run back to
+back on one stream through the library's stack entry point
+(fe_moe_stack_forward) and captured as one CUDA graph.  One step = one replay
+= 48 layer forwards.  The stack touches
+48 x 21.2 MB = 1.02 GB of expert weights per step, more than the 126 MB L2, so
+no step finds its weights in L2 from the step before.
+
+The other workloads of the layer run the same way, each as its own 48-layer
+stack, and are reported in the same JSON line under "workloads": the T=64
+decode batch with Zipf-skewed routing, the 512-expert layer at T=1 and T=4,
+and the T=4096 prefill layer (a tensor-core roofline).
+
+e2e: the same stack through fe_moe_stack_forward_host (the C-ABI call on host
+buffers): every step copies all 48 layers' x and logits from pinned host
+memory, runs the 48 layers and copies their y back.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
-a bounded sample of the same workload instead.
+a bounded sample of the headline workload instead.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -29,25 +40,63 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of B200 peak) at T=1"
-WORKLOAD = "decode_e128_t1"
+PREFILL_METRIC = "MoE-layer prefill tokens/s and tensor-core TFLOP/s at T=4096"
+HEADLINE = "decode_e128_t1"
+OTHERS = ["decode_e128_t64_zipf", "decode_e512_t1", "decode_e512_t4", "prefill_e128_t4096"]
 LAYERS = 48
 NOMINAL_HBM_GBS = 8000.0
+NOMINAL_FP4_TFLOPS = 9000.0
 L2_BYTES = 126e6
-KERNEL_NAMES = {1: "streaming mma.sync projections sg_kernel (routing, gate_up, down, combine)",
-                2: "tensor-core tiles tc_gemm_kernel (gate_up + down) with routing, row conversion and combine",
-                3: "decode_kernel (whole layer, one cooperative launch); per-launch time = step time / layers"}
-PREFILL_METRIC = "MoE-layer prefill tokens/s and tensor-core TFLOP/s at T=4096"
-# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu
-# captures summarised in profiles/ (recaptured whenever that kernel changes)
-TRAFFIC = {"decode_e128_t1": (21379072, "decode_kernel", "profiles/decode_kernel_decode_e128_t1.md"),
-           "prefill_e128_t4096": (299220224, "tc_gemm_kernel gate_up", "profiles/tc_gemm_kernel_prefill_e128_t4096.md"),
-           "decode_e128_t64_zipf": (95570432, "sg_kernel gate_up", "profiles/sg_kernel_decode_e128_t64_zipf.md")}
-BYTES_PER_EXPERT = lambda H, I: (H // 2) * 2 * I + (H // 32) * 2 * I * 2 + (I // 2) * H + (I // 32) * H * 2  # noqa: E731
+PATH_NAMES = {1: "moderate-T path: routing + streaming mma.sync projections (sg_kernel) + ordered combine",
+              2: "large-T path: routing + tensor-core tiles (tc_gemm_kernel) + ordered combine",
+              3: "decode_kernel (whole layer in one launch)"}
+CSRC = os.path.join(ROOT, "fp4_expert_gemv_b200", "csrc")
+
+# DRAM bytes (read + write) per launch of a workload's dominant kernel, read
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# kernel built from the sources whose hash is given: reported only while the
+# sources still hash to that value, null otherwise (the counters would describe
+# another kernel).
+NCU_TRAFFIC = {
+    # workload: (bytes per launch, kernel, sha256[:16] of the source files listed)
+}
+TRAFFIC_SOURCES = {"decode_kernel": ["decode.cuh", "mma.cuh", "common.cuh"],
+                   "sg_kernel gate_up": ["stream.cuh", "mma.cuh", "common.cuh"],
+                   "tc_gemm_kernel gate_up": ["tcgen05.cuh", "mma.cuh", "common.cuh"]}
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    if workload not in NCU_TRAFFIC:
+        return None, None
+    nbytes, kernel, digest = NCU_TRAFFIC[workload]
+    if source_hash(TRAFFIC_SOURCES[kernel]) != digest:
+        return None, kernel
+    return nbytes, kernel
+
+
+def bytes_per_expert(H, I):
+    """Packed codes + bf16 group scales of one expert's gate_up and down matrices."""
+    return (H // 2) * 2 * I + (H // 32) * 2 * I * 2 + (I // 2) * H + (I // 32) * H * 2
 
 
 def algorithmic_bytes_per_layer(E, H, I, T, distinct_experts):
     """Touched experts' packed codes + scales, plus x, logits and y."""
-    return distinct_experts * BYTES_PER_EXPERT(H, I) + T * H * 2 + T * E * 4 + T * H * 2
+    return distinct_experts * bytes_per_expert(H, I) + T * H * 2 + T * E * 4 + T * H * 2
+
+
+def distinct_routed(logits, k):
+    """Distinct experts the top-k of each row selects (ties to the lower index),
+    by a host sort of the logits: used for the byte count only."""
+    order = np.lexsort((np.broadcast_to(np.arange(logits.shape[-1]), logits.shape), -logits), axis=-1)
+    return len(np.unique(order[:, :k]))
 
 
 def measured_peaks():
@@ -55,19 +104,8 @@ def measured_peaks():
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
-
-
-def measured_tensor_peak():
-    """Dense bf16 TFLOP/s sustained under the power cap (the f16 tensor-core
-    rate is the same): the denominator for a kernel timed inside a long step."""
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
-        with open(path) as f:
-            d = json.load(f)
-        return float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured sustained bf16 (f16 operands)"
-    return 1400.0, "fallback sustained bf16"
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
 class ClockSampler:
@@ -154,18 +192,24 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
 # --------------------------------------------------------------------------------------------
 # CPU oracle timing (reference arm and cpu_baseline)
 # --------------------------------------------------------------------------------------------
 
 def oracle_sample_setup(cfg):
-    """Layer 0 of the stack, token 0: the oracle's weights for its 8 experts."""
+    """Layer 0 of the stack, token 0: the oracle's weights for its routed experts."""
     import oracle
     import synth
     E, H, I, k = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"]
     seed = synth.STACK_SEED0
     x = synth.activations_bf16(cfg["seeds"][0], 1, H)
-    lg = synth.router_logits(seed, 1, E)
+    lg = synth.router_logits(seed, 1, E, cfg["zipf"])
     orc = oracle.default()
     idx, _ = orc.route(lg, k)
     ex = sorted(set(int(e) for e in idx.reshape(-1)))
@@ -189,7 +233,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import synth
-    cfg = synth.WORKLOADS[args.workload]
+    cfg = synth.WORKLOADS[HEADLINE]
     orc, ew, x, lg, k = oracle_sample_setup(cfg)
     for _ in range(args.warmup):
         orc.moe_forward(ew, x, lg, k)
@@ -205,7 +249,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
-        "config": {"workload": args.workload, "E": cfg["E"], "H": cfg["H"], "I": cfg["I"], "top_k": cfg["top_k"],
+        "config": {"workload": HEADLINE, "E": cfg["E"], "H": cfg["H"], "I": cfg["I"], "top_k": cfg["top_k"],
                    "T": 1, "layers": 1, "parallelism": "cpu oracle, 1 thread"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -218,7 +262,9 @@ def run_reference(args):
 # GPU arm
 # --------------------------------------------------------------------------------------------
 
-def build_stack(cfg, layers, device):
+def build_stack(cfg, layers, device, max_T=None):
+    """`layers` fe_moe handles with the seeded weights of seeds 1000 + l, drawn
+    and packed on the device (the library's own packer)."""
     import torch
 
     import fp4_expert_gemv_b200 as fe
@@ -238,7 +284,7 @@ def build_stack(cfg, layers, device):
         synth.device_down(Wdn.data_ptr(), seed, E, I, H, st)
         fe.pack_device(Wgu, gc, gs)
         fe.pack_device(Wdn, dc, ds)
-        m = fe.MoELayer(E, H, I, max_T=cfg["T"], max_top_k=k)
+        m = fe.MoELayer(E, H, I, max_T=max_T or cfg["T"], max_top_k=k)
         m.load_packed(gc, gs, dc, ds)
         handles.append(m)
     torch.cuda.synchronize()
@@ -247,10 +293,182 @@ def build_stack(cfg, layers, device):
     return handles
 
 
+def stack_inputs(cfg, layers):
+    """Every layer's seeded inputs (seed 1000 + l): x bf16 bits [layers, T, H]
+    and router logits [layers, T, E]."""
+    import synth
+    T, H, E = cfg["T"], cfg["H"], cfg["E"]
+    x = np.stack([synth.activations_bf16(synth.STACK_SEED0 + l, T, H) for l in range(layers)])
+    lg = np.stack([synth.router_logits(synth.STACK_SEED0 + l, T, E, cfg["zipf"]) for l in range(layers)])
+    return np.ascontiguousarray(x), np.ascontiguousarray(lg, dtype=np.float32)
+
+
+def check_stack_parity(cfg, layers, x, lg, y_bits, check_layers, rows):
+    """The timed graph's outputs of the given layers, on the given token rows,
+    against the oracle (weights of seed 1000 + l), at the acceptance tolerance."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import harness
+    import synth
+    E, H, I, k = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"]
+    out = {"rows": [int(r) for r in rows], "tolerance": {"max_rel": harness.MAX_REL_TOL, "l2_rel": harness.L2_REL_TOL},
+           "layers": {}}
+    ok = True
+    for l in check_layers:
+        osd = harness.OracleSide(E, H, I, synth.STACK_SEED0 + l)
+        ref, _ = osd.forward(x[l][rows], lg[l][rows], k)
+        mr, l2 = harness.output_errors(y_bits[l][rows], ref)
+        good = bool(mr <= harness.MAX_REL_TOL and l2 <= harness.L2_REL_TOL)
+        out["layers"][str(l)] = {"max_rel": mr, "l2_rel": l2, "ok": good}
+        ok &= good
+    out["ok"] = ok
+    return out
+
+
+def run_workload(name, args, device, world, rank, headline=False):
+    """Build the workload's stack, time graph replays and the host-buffer call;
+    returns a dict of measurements."""
+    import torch
+
+    import fp4_expert_gemv_b200 as fe
+    import synth
+    cfg = synth.WORKLOADS[name]
+    E, H, I, k, T = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"], cfg["T"]
+    layers = args.layers
+    t_setup = time.perf_counter()
+    handles = build_stack(cfg, layers, device)
+    stack = fe.Stack(handles)
+    setup_s = time.perf_counter() - t_setup
+
+    x_host, lg = stack_inputs(cfg, layers)
+    x_pin = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+    lg_pin = torch.from_numpy(lg).pin_memory()
+    y_pin = torch.empty((layers, T, H), dtype=torch.int16).pin_memory()
+    x_dev = x_pin.to(device).view(torch.bfloat16)
+    lg_dev = lg_pin.to(device)
+    y_dev = torch.empty((layers, T, H), dtype=torch.bfloat16, device=device)
+    distinct = [distinct_routed(lg[l], k) for l in range(layers)]
+
+    s = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(s):
+        stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
+    torch.cuda.synchronize()
+    path, kernels_per_layer = handles[0].last_forward_info()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    cur = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(f"timed {name}")   # lets a profiler select the timed launches
+    e0.record(cur)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    # keep the GPU busy while the sampler catches the clocks of a loaded GPU
+    t_extra = time.perf_counter()
+    while time.perf_counter() - t_extra < 0.5:
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, world, device)
+    tokens_step = sum_over_ranks(layers * T, world, device)
+    value = tokens_step / (ms / 1e3)
+
+    # parity of the timed graph's outputs: layers 0 and 47 against the oracle
+    parity = None
+    if headline and not args.no_check:
+        torch.cuda.synchronize()
+        y_bits = y_dev.view(torch.int16).cpu().numpy().view(np.uint16)
+        rows = np.arange(T) if T <= 8 else np.array([0, T // 2, T - 1])
+        parity = check_stack_parity(cfg, layers, x_host, lg, y_bits, sorted({0, layers - 1}), rows)
+
+    # end to end through the C ABI on host buffers (fe_moe_stack_forward_host):
+    # H2D of x and every layer's logits, the layers, D2H of y, a stream sync
+    h2d = x_pin.numel() * 2 + lg_pin.numel() * 4
+    d2h = y_pin.numel() * 2
+    for _ in range(3):
+        stack.forward_host(x_pin, lg_pin, k, y_pin, stream=s)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        stack.forward_host(x_pin, lg_pin, k, y_pin, stream=s)
+    e2e_ms_local = (time.perf_counter() - t0) * 1e3 / args.steps
+    e2e_ms = max_over_ranks(e2e_ms_local, world, device)
+    e2e_value = tokens_step / (e2e_ms / 1e3)
+
+    peaks, peak_kind = measured_peaks()
+    bytes_layer = [algorithmic_bytes_per_layer(E, H, I, T, d) for d in distinct]
+    bytes_step = float(sum(bytes_layer))
+    us_layer = ms_local * 1e3 / layers
+    traffic, traffic_kernel = ncu_traffic(name)
+    prefill = name.startswith("prefill")
+    if prefill:
+        flops_layer = 2.0 * T * k * 3 * H * I
+        tf = flops_layer * layers / (ms_local / 1e3) / 1e12
+        tpeak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        roofline = {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
+                    "traffic": traffic, "kernel": PATH_NAMES.get(path, str(path)),
+                    "peak_kind": f"{peak_kind} sustained dense bf16 (f16 operands run at the same rate)",
+                    "algorithmic_flops_per_layer": flops_layer,
+                    "frac_of_nominal_fp4_9pflops": tf / NOMINAL_FP4_TFLOPS}
+    else:
+        achieved = bytes_step / (ms_local / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                    "frac": achieved / float(peaks["hbm_gbs"]), "traffic": traffic,
+                    "kernel": PATH_NAMES.get(path, str(path)), "peak_kind": f"{peak_kind} HBM copy",
+                    "algorithmic_bytes_per_layer_mean": bytes_step / layers,
+                    "distinct_experts_per_layer_mean": float(np.mean(distinct)),
+                    "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS}
+    if traffic_kernel:
+        roofline["traffic_kernel"] = traffic_kernel
+        roofline["traffic_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum per launch"
+                                    if traffic is not None else "kernel changed since its ncu capture")
+    res = {
+        "workload": name, "E": E, "H": H, "I": I, "top_k": k, "T": T, "layers_per_step": layers,
+        "steps": args.steps, "ms_per_step": ms, "us_per_layer": us_layer, "value": value,
+        "unit": "tokens/s", "roofline": roofline, "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms,
+                "call": "fe_moe_stack_forward_host on pinned host buffers (every layer's x and logits in, y out; "
+                        "synchronous)"},
+        "gpu_launches": kernels_per_layer * layers * args.steps,
+        "kernels_per_layer": kernels_per_layer,
+        "setup_s": setup_s,
+        "l2": (f"inputs larger than L2: each step streams {layers} layers' routed experts ({bytes_step / 1e9:.2f} GB)"
+               if bytes_step > L2_BYTES else
+               f"step bytes ({bytes_step / 1e6:.0f} MB) fit in L2: not a valid HBM measurement"),
+    }
+    if parity is not None:
+        res["parity"] = parity
+    del g
+    stack.close()
+    for m in handles:
+        m.close()
+    del handles
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_gpu(args):
     import torch
 
-    import synth
     world, rank, local = dist_setup()
     if world > 1:
         import datetime
@@ -261,157 +479,45 @@ def run_gpu(args):
     else:
         torch.cuda.set_device(0)
     device = torch.device("cuda", torch.cuda.current_device())
-    workload = args.workload
-    cfg = synth.WORKLOADS[workload]
-    E, H, I, k, T = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"], cfg["T"]
-    layers = args.layers
+    head_name = HEADLINE if args.workload == "all" else args.workload
+    others = [w for w in OTHERS if w != head_name] if args.workload == "all" else []
 
-    t_setup = time.perf_counter()
-    stack = build_stack(cfg, layers, device)
-    setup_s = time.perf_counter() - t_setup
+    head = run_workload(head_name, args, device, world, rank, headline=True)
+    extra = {}
+    for w in others:
+        extra[w] = run_workload(w, args, device, world, rank)
 
-    # inputs: x of layer 0, logits of every layer (seed 1000 + l); buffers reused by every replay
-    x0_host = synth.activations_bf16(cfg["seeds"][0], T, H)
-    lg_host = np.stack([synth.router_logits(synth.STACK_SEED0 + l, T, E, cfg["zipf"]) for l in range(layers)])
-    x_pin = torch.from_numpy(x0_host.view(np.int16)).pin_memory()
-    lg_pin = torch.from_numpy(lg_host).pin_memory()
-    x_dev = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-    lg_dev = torch.empty((layers, T, E), dtype=torch.float32, device=device)
-    acts = [torch.empty((T, H), dtype=torch.bfloat16, device=device) for _ in range(layers)]
-    y_pin = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    x_dev.copy_(x_pin.view(torch.bfloat16))
-    lg_dev.copy_(lg_pin)
-
-    s = torch.cuda.Stream(device=device)
-    distinct = []
-
-    def forward_all(stream):
-        inp = x_dev
-        for l, m in enumerate(stack):
-            m.forward(inp, lg_dev[l], k, acts[l], stream=stream)
-            inp = acts[l]
-
-    with torch.cuda.stream(s):
-        forward_all(s)
-    torch.cuda.synchronize()
-    # routing check of the stack: distinct experts per layer (for the byte count)
-    for l, m in enumerate(stack):
-        idx, _, _, _ = m.routing(T, k)
-        distinct.append(len(set(idx.cpu().numpy().reshape(-1).tolist())))
-    path, kernels_per_layer = stack[0].last_forward_info()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        forward_all(s)
-    torch.cuda.synchronize()
-
-    for _ in range(args.warmup):
-        g.replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
-    time.sleep(0.3)
-    cur = torch.cuda.current_stream()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.nvtx.range_push("timed")   # lets a profiler select the timed launches
-    e0.record(cur)
-    for _ in range(args.steps):
-        g.replay()
-    e1.record(cur)
-    torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    # keep the GPU busy while the sampler catches the clocks of a loaded GPU
-    t_extra = time.perf_counter()
-    while time.perf_counter() - t_extra < 0.5:
-        for _ in range(20):
-            g.replay()
-        torch.cuda.synchronize()
-    clk = clocks.stop()
-    ms_local = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms_local, world, device)
-    tokens_per_step_local = layers * T
-    tokens_per_step = sum_over_ranks(tokens_per_step_local, world, device)
-    value = tokens_per_step / (ms / 1e3)
-    us_per_layer = ms * 1e3 / layers
-
-    # end to end: pinned H2D of x and all logits, graph replay, D2H of the last layer's y
-    h2d = x_pin.numel() * 2 + lg_pin.numel() * 4
-    d2h = y_pin.numel() * 2
-    for _ in range(3):
-        x_dev.copy_(x_pin.view(torch.bfloat16), non_blocking=True)
-        lg_dev.copy_(lg_pin, non_blocking=True)
-        g.replay()
-        y_pin.copy_(acts[-1].view(torch.int16), non_blocking=True)
-        torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0.record(cur)
-    for _ in range(args.steps):
-        x_dev.copy_(x_pin.view(torch.bfloat16), non_blocking=True)
-        lg_dev.copy_(lg_pin, non_blocking=True)
-        g.replay()
-        y_pin.copy_(acts[-1].view(torch.int16), non_blocking=True)
-    e1.record(cur)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, device)
-    e2e_value = tokens_per_step / (e2e_ms / 1e3)
-
-    peak, peak_kind = measured_peaks()
-    bytes_layer = [algorithmic_bytes_per_layer(E, H, I, T, d) for d in distinct]
-    bytes_step = float(sum(bytes_layer))
-    achieved = bytes_step / (ms_local / 1e3) / 1e9
-    prefill = workload.startswith("prefill")
-    if prefill:
-        # a dense contraction: FLOPs of gate_up + down over all token-expert pairs
-        flops_layer = 2.0 * T * k * 3 * H * I
-        tf = flops_layer * layers / (ms_local / 1e3) / 1e12
-        tpeak, tpeak_kind = measured_tensor_peak()
-        roofline = {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
-                    "traffic": TRAFFIC.get(workload, (None,))[0], "kernel": KERNEL_NAMES.get(path, str(path)), "peak_kind": tpeak_kind,
-                    "algorithmic_flops_per_layer": flops_layer,
-                    "frac_of_nominal_fp4_9pflops": tf / 9000.0}
-    else:
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": TRAFFIC.get(workload, (None,))[0], "kernel": KERNEL_NAMES.get(path, str(path)),
-                    "peak_kind": peak_kind, "algorithmic_bytes_per_layer": bytes_layer[0]}
-    if workload in TRAFFIC:
-        roofline["traffic_kernel"] = TRAFFIC[workload][1]
-        roofline["traffic_source"] = TRAFFIC[workload][2]
+    prefill = head_name.startswith("prefill")
     line = {
-        "metric": PREFILL_METRIC if prefill else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32",
+        "metric": PREFILL_METRIC if prefill else METRIC, "value": head["value"], "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded counter-based generator; random-init weights quantised to E2M1)",
-        "config": {"workload": workload, "E": E, "H": H, "I": I, "top_k": k, "T": T, "layers_per_step": layers,
-                   "global_batch": T * world, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: each step streams {layers} layers' routed experts "
-                         f"({bytes_step / 1e9:.2f} GB)" if bytes_step > L2_BYTES else
-                         f"step bytes ({bytes_step / 1e6:.0f} MB) fit in L2: not a valid HBM measurement",
-                   "graph": f"one CUDA graph of {layers} chained fe_moe_forward calls"},
-        "us_per_layer": us_per_layer,
-        "hbm_gbs_achieved": achieved,
-        "hbm_frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-        "roofline": roofline,
-        "clocks": clk,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "gpu_launches": kernels_per_layer * layers * args.steps,
-        "setup_s": setup_s,
+        "config": {"workload": head_name, "E": head["E"], "H": head["H"], "I": head["I"], "top_k": head["top_k"],
+                   "T": head["T"], "layers_per_step": head["layers_per_step"], "global_batch": head["T"] * world,
+                   "parallelism": f"replicas x{world}", "l2": head["l2"],
+                   "graph": f"one CUDA graph of fe_moe_stack_forward over {head['layers_per_step']} layers, "
+                            "each with its own seeded weights, x and logits"},
+        "us_per_layer": head["us_per_layer"],
+        "roofline": head["roofline"],
+        "clocks": head["clocks"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "setup_s": head["setup_s"],
     }
+    if "parity" in head:
+        line["parity"] = head["parity"]
+    if extra:
+        line["workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import synth
         reps = args.cpu_reps
-        per = time_oracle(cfg, reps)
-        line["cpu_baseline"] = {"value": 1.0 / per, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"layer 0 of the stack, token 0, {reps} single-threaded oracle forwards"}
+        per = time_oracle(synth.WORKLOADS[head_name], reps) if not prefill else None
+        if per is not None:
+            line["cpu_baseline"] = {"value": 1.0 / per, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"layer 0 of the stack, token 0, {reps} single-threaded oracle forwards"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0
@@ -420,15 +526,15 @@ def run_gpu(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["fe", "reference"], default="fe")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--cpu-reps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD,
-                    choices=["decode_e128_t1", "decode_e128_t64_zipf", "decode_e512_t1", "decode_e512_t4",
-                             "prefill_e128_t4096"])
+    ap.add_argument("--no-check", action="store_true", help="skip the oracle check of the headline stack's output")
+    ap.add_argument("--workload", default="all", choices=["all", HEADLINE] + OTHERS,
+                    help="all: the headline workload plus the others under 'workloads'")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -60,6 +60,13 @@ _SIGS = {
     "fe_moe_device_bytes": (ctypes.c_size_t, [_P]),
     "fe_moe_last_error": (ctypes.c_char_p, []),
     "fe_moe_forward_noalloc": (_st, [_i32, _i32, _i32, _P, _P, _P, _P, _P, _P, _i32, _i32, _P, _P]),
+    "fe_moe_get_grouping": (_st, [_P, _P, _P, _P]),
+    "fe_moe_noalloc_get_status": (_st, [ctypes.POINTER(ctypes.c_uint32)]),
+    "fe_moe_noalloc_get_routing": (_st, [_i32, _i32, _i32, _P, _P, _P, _P, _P, _P, _P]),
+    "fe_moe_stack_create": (_st, [ctypes.POINTER(_P), _i32, ctypes.POINTER(_P)]),
+    "fe_moe_stack_forward": (_st, [_P, _P, _P, _i32, _i32, _P, _P]),
+    "fe_moe_stack_forward_host": (_st, [_P, _P, _P, _i32, _i32, _P, _i32, _P]),
+    "fe_moe_stack_destroy": (None, [_P]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -162,6 +169,15 @@ class MoELayer:
               "fe_moe_get_routing")
         return idx, w, offsets, sp
 
+    def grouping(self, T: int, top_k: int, stream=None):
+        """(counts int32 [E], pair_row int32 [T*top_k]) of the last forward, as device tensors."""
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        counts = torch.empty(self.E, dtype=torch.int32, device=dev)
+        pair_row = torch.empty(T * top_k, dtype=torch.int32, device=dev)
+        check(fe_moe_get_grouping(self.h, _dptr(counts), _dptr(pair_row), _stream_ptr(stream)), "fe_moe_get_grouping")
+        return counts, pair_row
+
     def status(self):
         bits = ctypes.c_uint32(0)
         st = fe_moe_get_status(self.h, ctypes.byref(bits))
@@ -188,6 +204,55 @@ class MoELayer:
             self.close()
         except Exception:
             pass
+
+
+class Stack:
+    """fe_moe_stack over MoELayer objects (kept alive here): n layers back to back on one stream."""
+
+    def __init__(self, layers):
+        self.layers = list(layers)
+        arr = (_P * len(self.layers))(*[m.h for m in self.layers])
+        h = _P()
+        check(fe_moe_stack_create(arr, len(self.layers), ctypes.byref(h)), "fe_moe_stack_create")
+        self.h = h
+        self.n = len(self.layers)
+        self.E, self.H = self.layers[0].E, self.layers[0].H
+
+    def forward(self, x_bf16, logits, top_k: int, y_bf16, stream=None):
+        """x device bf16 [n, T, H] (layer l reads x[l]), logits device float32 [n, T, E], y device bf16
+        [n, T, H] (layer l writes y[l]); pass y = a view of x shifted by one layer to chain them."""
+        T = logits.shape[1]
+        check(fe_moe_stack_forward(self.h, _dptr(x_bf16), _dptr(logits), T, top_k, _dptr(y_bf16),
+                                   _stream_ptr(stream)), "fe_moe_stack_forward")
+        return y_bf16
+
+    def forward_host(self, x_bf16_host, logits_host, top_k: int, y_bf16_host, chained=False, stream=None):
+        """Host buffers (numpy or CPU torch, ideally pinned), bf16 as int16/uint16 bits; logits [n, T, E].
+        chained=False: x, y [n, T, H]; chained=True: x [T, H] into layer 0, y [T, H] out of the last."""
+        def hp(a):
+            return a.ctypes.data if hasattr(a, "ctypes") else a.data_ptr()
+        T = logits_host.shape[1]
+        check(fe_moe_stack_forward_host(self.h, hp(x_bf16_host), hp(logits_host), T, top_k, hp(y_bf16_host),
+                                        1 if chained else 0, _stream_ptr(stream)), "fe_moe_stack_forward_host")
+        return y_bf16_host
+
+    def close(self):
+        if getattr(self, "h", None):
+            fe_moe_stack_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def noalloc_status():
+    """(status, bits) of the last fe_moe_forward_noalloc call on the current device."""
+    bits = ctypes.c_uint32(0)
+    st = fe_moe_noalloc_get_status(ctypes.byref(bits))
+    return st, bits.value
 
 
 def pack_host(W):

@@ -73,6 +73,14 @@ struct fe_moe_s {
     int last_path = 0, last_kernels = 0;
 };
 
+struct fe_moe_stack_s {
+    std::vector<fe_moe_s*> layers;
+    int device = 0, E = 0, H = 0, max_T = 0;
+    uint16_t* a_stage = nullptr;     // fe_moe_stack_forward_host: [n + 1][max_T][H] (inputs; chained: all)
+    uint16_t* b_stage = nullptr;     // [n][max_T][H] (outputs of independent layers)
+    float* logits_stage = nullptr;   // [n][max_T][E]
+};
+
 namespace {
 
 // Text of the last CUDA failure seen by this thread (fe_moe_last_error).
@@ -775,6 +783,105 @@ fe_status fe_moe_forward_host(fe_moe_t h, const uint16_t* x_host, const float* l
     return FE_OK;
 }
 
+fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack_t* out)
+{
+    if (!out) return FE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!layers || n_layers < 1) return FE_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        const fe_moe_s* h = layers[l];
+        if (!h || h->E != layers[0]->E || h->H != layers[0]->H || h->device != layers[0]->device)
+            return FE_ERR_INVALID_ARG;
+        if (!h->loaded) return FE_ERR_NOT_LOADED;
+        if (h->max_T < 1) return FE_ERR_CAPACITY;
+    }
+    fe_moe_stack_s* st = new (std::nothrow) fe_moe_stack_s();
+    if (!st) return FE_ERR_OOM;
+    st->layers.assign(layers, layers + n_layers);
+    st->device = layers[0]->device;
+    st->E = layers[0]->E;
+    st->H = layers[0]->H;
+    st->max_T = layers[0]->max_T;
+    for (int l = 1; l < n_layers; ++l) st->max_T = std::min(st->max_T, layers[l]->max_T);
+    DeviceGuard g(st->device);
+    cudaError_t e = g.ok ? cudaSuccess : cudaErrorInvalidDevice;
+    const size_t row = (size_t)st->max_T * st->H;
+    if (e == cudaSuccess) e = dmalloc(&st->a_stage, ((size_t)n_layers + 1) * row, nullptr);
+    if (e == cudaSuccess) e = dmalloc(&st->b_stage, (size_t)n_layers * row, nullptr);
+    if (e == cudaSuccess) e = dmalloc(&st->logits_stage, (size_t)n_layers * st->max_T * st->E, nullptr);
+    if (e != cudaSuccess) {
+        fe_moe_stack_destroy(st);
+        return record_cuda(e, "fe_moe_stack_create");
+    }
+    *out = st;
+    return FE_OK;
+}
+
+fe_status fe_moe_stack_forward(fe_moe_stack_t st, const void* x_bf16, const float* logits, int T, int top_k,
+                               void* y_bf16, fe_stream_t stream)
+{
+    if (!st || T < 0 || top_k < 1) return FE_ERR_INVALID_ARG;
+    if (T == 0) return FE_OK;
+    if (!x_bf16 || !logits || !y_bf16) return FE_ERR_INVALID_ARG;
+    const size_t row_bytes = sizeof(uint16_t) * (size_t)T * st->H;
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x_bf16), ya = reinterpret_cast<uintptr_t>(y_bf16);
+    if ((xa > ya ? xa - ya : ya - xa) < row_bytes) return FE_ERR_INVALID_ARG;   // y_l would overlap x_l
+    if ((xa & 3u) || (ya & 3u) || (reinterpret_cast<uintptr_t>(logits) & 3u)) return FE_ERR_INVALID_ARG;
+    // every layer's arguments are checked before the first launch
+    for (fe_moe_s* h : st->layers) {
+        if (top_k > h->E) return FE_ERR_INVALID_ARG;
+        if (!h->loaded) return FE_ERR_NOT_LOADED;
+        if (T > h->max_T || top_k > h->max_k) return FE_ERR_CAPACITY;
+        if (h->path == FE_PATH_TCGEN05 && !(tc_shape_ok(h) && h->tc_scales_ok && h->tc_x)) return FE_ERR_UNSUPPORTED;
+    }
+    const int n = (int)st->layers.size();
+    const size_t xe = (size_t)T * st->H;
+    for (int l = 0; l < n; ++l) {
+        const fe_status r = fe_moe_forward(st->layers[l], static_cast<const uint16_t*>(x_bf16) + l * xe,
+                                           logits + (size_t)l * T * st->E, T, top_k,
+                                           static_cast<uint16_t*>(y_bf16) + l * xe, stream);
+        if (r != FE_OK) return r;
+    }
+    return FE_OK;
+}
+
+fe_status fe_moe_stack_forward_host(fe_moe_stack_t st, const uint16_t* x_host, const float* logits_host, int T,
+                                    int top_k, uint16_t* y_host, int chained, fe_stream_t stream)
+{
+    if (!st || T < 0 || top_k < 1) return FE_ERR_INVALID_ARG;
+    if (T == 0) return FE_OK;
+    if (!x_host || !logits_host || !y_host) return FE_ERR_INVALID_ARG;
+    if (T > st->max_T) return FE_ERR_CAPACITY;
+    DeviceGuard g(st->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t n = st->layers.size();
+    const size_t row = sizeof(uint16_t) * (size_t)T * st->H;
+    const size_t xs = chained ? row : n * row;
+    FE_CUDA_TRY(cudaMemcpyAsync(st->a_stage, x_host, xs, cudaMemcpyHostToDevice, s));
+    FE_CUDA_TRY(cudaMemcpyAsync(st->logits_stage, logits_host, sizeof(float) * n * T * st->E, cudaMemcpyHostToDevice, s));
+    uint16_t* y_dev = chained ? st->a_stage + (size_t)T * st->H : st->b_stage;
+    const fe_status r = fe_moe_stack_forward(st, st->a_stage, st->logits_stage, T, top_k, y_dev, stream);
+    if (r != FE_OK) return r;
+    const uint16_t* y_src = chained ? st->a_stage + n * (size_t)T * st->H : st->b_stage;
+    FE_CUDA_TRY(cudaMemcpyAsync(y_host, y_src, xs, cudaMemcpyDeviceToHost, s));
+    FE_CUDA_TRY(cudaStreamSynchronize(s));
+    return FE_OK;
+}
+
+void fe_moe_stack_destroy(fe_moe_stack_t st)
+{
+    if (!st) return;
+    {
+        DeviceGuard g(st->device);
+        cudaDeviceSynchronize();
+        if (st->a_stage) cudaFree(st->a_stage);
+        if (st->b_stage) cudaFree(st->b_stage);
+        if (st->logits_stage) cudaFree(st->logits_stage);
+    }
+    delete st;
+}
+
 fe_status fe_moe_get_routing(fe_moe_t h, int32_t* idx, float* w, int32_t* offsets, int32_t* sorted_pair,
                              fe_stream_t stream)
 {
@@ -790,6 +897,20 @@ fe_status fe_moe_get_routing(fe_moe_t h, int32_t* idx, float* w, int32_t* offset
         FE_CUDA_TRY(cudaMemcpyAsync(offsets, h->offsets, sizeof(int32_t) * (h->E + 1), cudaMemcpyDeviceToDevice, s));
     if (sorted_pair && P)
         FE_CUDA_TRY(cudaMemcpyAsync(sorted_pair, h->sorted_pair, sizeof(int32_t) * P, cudaMemcpyDeviceToDevice, s));
+    return FE_OK;
+}
+
+fe_status fe_moe_get_grouping(fe_moe_t h, int32_t* counts, int32_t* pair_row, fe_stream_t stream)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    if (!h->idx) return FE_ERR_CAPACITY;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t P = (size_t)h->last_T * h->last_k;
+    if (counts) FE_CUDA_TRY(cudaMemcpyAsync(counts, h->counts, sizeof(int32_t) * h->E, cudaMemcpyDeviceToDevice, s));
+    if (pair_row && P)
+        FE_CUDA_TRY(cudaMemcpyAsync(pair_row, h->pair_row, sizeof(int32_t) * P, cudaMemcpyDeviceToDevice, s));
     return FE_OK;
 }
 
@@ -987,6 +1108,8 @@ fe_status fe_moe_forward_noalloc(int E, int H, int I, const uint8_t* gate_up_cod
     if (st0 != FE_OK) return st0;
     cudaStream_t s = (cudaStream_t)stream;
     const int P = T * top_k;
+    // the status word starts every call at zero (a memset node, no allocation)
+    FE_CUDA_TRY(cudaMemsetAsync(scr + L.status, 0, sizeof(uint32_t), s));
 
     fe::RouteParams rp{};
     rp.logits = router_logits; rp.T = T; rp.E = E; rp.k = top_k;
@@ -1027,6 +1150,51 @@ fe_status fe_moe_forward_noalloc(int E, int H, int I, const uint8_t* gate_up_cod
     fe::combine_kernel<false><<<cgrid, 256, 0, s>>>(reinterpret_cast<const float*>(scr + L.o), rp.w, rp.pair_row, H, top_k,
                                               static_cast<__nv_bfloat16*>(y_bf16));
     FE_CUDA_TRY(cudaGetLastError());
+    return FE_OK;
+}
+
+fe_status fe_moe_noalloc_get_status(uint32_t* bits)
+{
+    int dev = 0;
+    FE_CUDA_TRY(cudaGetDevice(&dev));
+    unsigned char* scr = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (dev < 0 || dev >= 64 || !g_noalloc_dev[dev].ready) return FE_ERR_INVALID_ARG;
+        scr = g_noalloc_dev[dev].scratch;
+    }
+    uint32_t v = 0;
+    FE_CUDA_TRY(cudaDeviceSynchronize());
+    FE_CUDA_TRY(cudaMemcpy(&v, scr, sizeof(v), cudaMemcpyDeviceToHost));   // the status word is at offset 0
+    FE_CUDA_TRY(cudaMemset(scr, 0, sizeof(v)));
+    if (bits) *bits = v;
+    return v ? FE_ERR_DEVICE_STATUS : FE_OK;
+}
+
+fe_status fe_moe_noalloc_get_routing(int E, int T, int top_k, int32_t* idx, float* w, int32_t* counts,
+                                     int32_t* offsets, int32_t* sorted_pair, int32_t* pair_row, fe_stream_t stream)
+{
+    if (E < 1 || E > 1024 || T < 0 || top_k < 1 || top_k > E) return FE_ERR_INVALID_ARG;
+    int dev = 0;
+    FE_CUDA_TRY(cudaGetDevice(&dev));
+    unsigned char* scr = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (dev < 0 || dev >= 64 || !g_noalloc_dev[dev].ready) return FE_ERR_INVALID_ARG;
+        scr = g_noalloc_dev[dev].scratch;
+    }
+    // the routing lists sit before act and o, at offsets that depend on E, T and top_k only
+    const NoAllocLayout L = noalloc_layout(E, 64, 64, T, top_k);
+    if (L.act > kNoAllocScratchBytes) return FE_ERR_CAPACITY;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t P = (size_t)T * top_k;
+    const cudaMemcpyKind d2d = cudaMemcpyDeviceToDevice;
+    if (idx && P) FE_CUDA_TRY(cudaMemcpyAsync(idx, scr + L.idx, 4 * P, d2d, s));
+    if (w && P) FE_CUDA_TRY(cudaMemcpyAsync(w, scr + L.w, 4 * P, d2d, s));
+    if (counts) FE_CUDA_TRY(cudaMemcpyAsync(counts, scr + L.counts, 4 * (size_t)E, d2d, s));
+    if (offsets) FE_CUDA_TRY(cudaMemcpyAsync(offsets, scr + L.offsets, 4 * ((size_t)E + 1), d2d, s));
+    if (sorted_pair && P) FE_CUDA_TRY(cudaMemcpyAsync(sorted_pair, scr + L.sorted_pair, 4 * P, d2d, s));
+    if (pair_row && P) FE_CUDA_TRY(cudaMemcpyAsync(pair_row, scr + L.pair_row, 4 * P, d2d, s));
     return FE_OK;
 }
 

@@ -88,10 +88,11 @@ FE_DEV void stage_inputs(const GemvParams& p, int e_pos0, int nt, uint32_t* xs, 
     if (tid < NT) {
         float m = 0.0f;
         for (int w = 0; w < nthreads / 32; ++w) m = fmaxf(m, red[w * NT + tid]);
-        // smallest s >= 0 with m * 2^-s < 2^15
+        // s with m * 2^-s in [2^14, 2^15): no fp16 overflow for large rows, full
+        // fp16 precision for small ones; s in [-100, 113], 0 for a zero, inf or
+        // nan maximum (inf/nan propagate as they are)
         int s = 0;
-        if (m >= 32768.0f) s = (int)((__float_as_uint(m) >> 23) & 0xff) - 127 - 14;
-        if (!(m == m) || m > 3.0e38f) s = 0;  // inf/nan propagate as they are
+        if (m > 0.0f && m <= 3.4e38f) s = max(-100, (int)((__float_as_uint(m) >> 23) & 0xff) - 127 - 14);
         shift[tid] = s;
     }
     __syncthreads();

@@ -182,13 +182,16 @@ FE_DEV void quad_mma2_b(const uint8_t* blk0, const uint8_t* blk1, int K, const u
     }
 }
 
-// Power-of-two shift s >= 0 with m * 2^-s < 2^15 (m = max |v| of a row), so
-// that a row staged as fp16 cannot overflow.
+// Power-of-two shift s of a row staged as fp16 (m = max |v| of the row): the
+// row is stored as v * 2^-s with m * 2^-s in [2^14, 2^15), so a large row
+// cannot overflow and a small one keeps fp16's full precision instead of
+// sinking into its subnormal range.  s is clamped to [-100, 113] (both 2^s and
+// 2^-s stay normal floats); a zero, infinite or NaN maximum gives s = 0.
 FE_DEV int fp16_shift(float m)
 {
-    int s = 0;
-    if (m >= 32768.0f && m <= 3.0e38f) s = (int)((__float_as_uint(m) >> 23) & 0xff) - 127 - 14;
-    return s;
+    if (!(m > 0.0f) || m > 3.4e38f) return 0;
+    const int s = (int)((__float_as_uint(m) >> 23) & 0xff) - 127 - 14;
+    return s < -100 ? -100 : s;
 }
 
 FE_DEV float pow2f(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }

@@ -73,19 +73,29 @@ typedef enum {
 #define FE_DEVICE_TC_TIMEOUT 0x10       /* a tensor-core tile gave up waiting for its MMAs */
 
 /* Create a handle for a layer of E experts, hidden size H and expert
- * intermediate size I on the current CUDA device.  group must be 32; H and I
+ * intermediate size I on the current CUDA device.  The layer's shape is the
+ * 128-expert MoE FFN of "FireEcho Engine" (section "Key Results": 30B total,
+ * ~3.3B active parameters per token; "Architecture": MoEFFN, packed MoE with
+ * fused dispatch); group is the number of consecutive k sharing one scale.  group must be 32; H and I
  * must be positive multiples of 32 (FE_ERR_INVALID_ARG otherwise) and of 64
  * (FE_ERR_UNSUPPORTED otherwise: the kernels read K in quads of 64); E in
  * [1, 1024].  Allocates the weight buffers (E * (H*2I + I*H) * 9/16 bytes) but
  * no workspace. */
 fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out);
 
-/* Allocate the forward workspace for up to max_T tokens and top_k <= max_top_k.
+/* Allocate the forward workspace for up to max_T tokens and top_k <= max_top_k
+ * ("FireEcho Engine", "Speed Optimization History" steps 6-7: buffers are
+ * made once, outside the decode loop, so that the graph-captured forward
+ * allocates nothing).
  * Synchronous, allocating, not capturable; call it before capturing forward in
  * a CUDA graph.  Calling it again with larger limits re-allocates. */
 fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k);
 
-/* Load packed weights in the format above (sizes follow from E, H, I):
+/* Load packed weights in the format above ("FireEcho Engine", "The Goliath
+ * Kernel: Why It's Fast": all experts packed into one contiguous
+ * [E, K/2, N] buffer; "Key Results": 4x compression of BF16; "Packed Marlin
+ * projections": gate and up projections packed into one matrix at load
+ * time).  Sizes follow from E, H, I:
  *   gate_up_codes  uint8 [E][H/2][2I],  gate_up_scales bf16 [E][H/32][2I],
  *   down_codes     uint8 [E][I/2][H],   down_scales    bf16 [E][I/32][H].
  * src_on_device = 1: the four pointers are device memory; 0: host memory.
@@ -99,7 +109,11 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uin
                              const uint8_t* down_codes, const uint16_t* down_scales, int src_on_device,
                              fe_stream_t stream);
 
-/* The layer: y = MoE(x).  x_bf16 device bf16 [T][H], router_logits device
+/* The layer: y = MoE(x) ("FireEcho Engine", "Speed Optimization History"
+ * steps 1-5 and "The Goliath Kernel: Why It's Fast": grouped dispatch with
+ * expert ids read from device memory, fused gate_up projection, FP4 decoded
+ * inside the matmul loop; "FastInfer", "Confirmed elementwise SwiGLU
+ * scheduling": SiLU(gate) * up).  x_bf16 device bf16 [T][H], router_logits device
  * float [T][E], y_bf16 device bf16 [T][H] (must not alias x).  T = 0 is a
  * no-op.  1 <= top_k <= min(E, max_top_k), T <= max_T.  Asynchronous on
  * stream: no host synchronisation and no allocation, so it can be captured in
@@ -108,18 +122,28 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uin
 fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k,
                          void* y_bf16, fe_stream_t stream);
 
-/* The layer on HOST buffers: copies x and the logits to the device, runs
+/* The layer on HOST buffers (no counterpart on the pages: the same layer as
+ * fe_moe_forward for a caller whose x and logits are in host memory): copies
+ * x and the logits to the device, runs
  * fe_moe_forward and copies y back, then waits for the stream.  Same argument
  * rules as fe_moe_forward (T <= max_T).  Synchronous. */
 fe_status fe_moe_forward_host(fe_moe_t h, const uint16_t* x_bf16_host, const float* router_logits_host, int T,
                               int top_k, uint16_t* y_bf16_host, fe_stream_t stream);
 
 /* Copy the routing of the last forward into caller device buffers (any may
- * be NULL): idx int32 [T][top_k], w float [T][top_k], offsets int32 [E+1]
+ * be NULL) -- the router and grouping of "FireEcho Engine", "Speed
+ * Optimization History" step 1 (grouped dispatch) and "The Goliath Kernel:
+ * Why It's Fast" (expert ids stay on the GPU): idx int32 [T][top_k], w float [T][top_k], offsets int32 [E+1]
  * (exclusive scan of the per-expert pair counts), sorted_pair int32
  * [T*top_k] (pair ids ordered by (expert, pair id)).  Enqueued on stream. */
 fe_status fe_moe_get_routing(fe_moe_t h, int32_t* idx, float* w, int32_t* offsets, int32_t* sorted_pair,
                              fe_stream_t stream);
+
+/* Copy the rest of the last forward's grouping into caller device buffers
+ * (either may be NULL): counts int32 [E] (pairs per expert) and pair_row
+ * int32 [T*top_k] (pair_row[p] = the grouped position of pair p, the inverse
+ * of sorted_pair, which the ordered combine reads).  Enqueued on stream. */
+fe_status fe_moe_get_grouping(fe_moe_t h, int32_t* counts, int32_t* pair_row, fe_stream_t stream);
 
 /* Wait for the device and return FE_ERR_DEVICE_STATUS if a kernel flagged a
  * problem since the last call (the bits go to *bits if non-NULL), FE_OK
@@ -192,14 +216,71 @@ fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, ui
  * each device, with that device current, looks up the array's device address
  * and sets kernel attributes (neither allocates); make that first call before
  * any stream capture.  Every call shares the array and leaves its contents
- * behind; each call writes every scratch word it reads, so nothing has to be
- * cleared between calls, but calls whose kernels overlap on the GPU (other
- * streams, other threads) race on the array and must be serialised by the
- * caller.  Same sizes and layouts as fe_moe_create + fe_moe_forward; no
- * allocation, no host synchronisation; argument errors as fe_moe_forward. */
+ * behind: each call clears the array's status word when it starts (an
+ * asynchronous memset on the stream, which allocates nothing) and writes
+ * every other scratch word before it reads it, but calls whose kernels
+ * overlap on the GPU (other streams, other threads) race on the array and
+ * must be serialised by the caller.  Same sizes and layouts as fe_moe_create
+ * + fe_moe_forward; no allocation, no host synchronisation; argument errors
+ * as fe_moe_forward.  Device-side problems (a NaN logit, an expert id out of
+ * range) are reported by fe_moe_noalloc_get_status, not fe_moe_get_status. */
 fe_status fe_moe_forward_noalloc(int E, int H, int I, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
                                  const uint8_t* down_codes, const uint16_t* down_scales, const void* x_bf16,
                                  const float* router_logits, int T, int top_k, void* y_bf16, fe_stream_t stream);
+
+/* Device-side problem bits (FE_DEVICE_BAD_EXPERT, FE_DEVICE_NAN_LOGIT) of the
+ * last fe_moe_forward_noalloc call on the current device.  Waits for the
+ * device, returns FE_ERR_DEVICE_STATUS if a bit is set (the bits go to *bits
+ * if non-NULL) and FE_OK otherwise, and clears the word.  The word is shared
+ * by every call on the device, like the rest of the array.  Allocates
+ * nothing; FE_ERR_INVALID_ARG before the first fe_moe_forward_noalloc call on
+ * the device. */
+fe_status fe_moe_noalloc_get_status(uint32_t* bits);
+
+/* Copy the routing and grouping of the last fe_moe_forward_noalloc call on
+ * the current device (which must have had these E, T and top_k) from the
+ * static array into caller device buffers, any of which may be NULL: idx int32
+ * [T][top_k], w float [T][top_k], counts int32 [E], offsets int32 [E+1],
+ * sorted_pair and pair_row int32 [T*top_k] (as fe_moe_get_routing and
+ * fe_moe_get_grouping).  Enqueued on stream; allocates nothing. */
+fe_status fe_moe_noalloc_get_routing(int E, int T, int top_k, int32_t* idx, float* w, int32_t* counts,
+                                     int32_t* offsets, int32_t* sorted_pair, int32_t* pair_row, fe_stream_t stream);
+
+/* ---- a stack of layers -------------------------------------------------------
+ * n layers run back to back on one stream, as in the 48-layer graph-captured
+ * decode forward of "FireEcho Engine" (section "Benchmark Results", row L6,
+ * and "Speed Optimization History" step 7). */
+typedef struct fe_moe_stack_s* fe_moe_stack_t;
+
+/* Build a stack over n_layers >= 1 handles, which it does not own (they must
+ * outlive the stack): all on one device, with the same E and H, each reserved
+ * and loaded.  Allocates staging for fe_moe_stack_forward_host: x and y of
+ * every layer ([n_layers (+1)][max_T][H] bf16, max_T the smallest
+ * reservation among the layers) and the logits of every layer. */
+fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack_t* out);
+
+/* Layer l = 0 .. n_layers-1, in order on stream: y_l = layer[l](x_l) with
+ * x_l = x_bf16 + l*T*H, logits_l = logits + l*T*E and y_l = y_bf16 + l*T*H
+ * (device memory; bf16 [T][H], float [T][E]).  y_l must not overlap x_l.
+ * Passing y_bf16 = x_bf16 + T*H chains the layers (layer l + 1 reads what
+ * layer l wrote, stream order making it safe); separate buffers make them
+ * independent.  Each layer runs as fe_moe_forward on its own handle; every
+ * layer's arguments are checked before the first launch.  Asynchronous, no
+ * allocation, no host synchronisation: capturable in one CUDA graph. */
+fe_status fe_moe_stack_forward(fe_moe_stack_t s, const void* x_bf16, const float* logits, int T, int top_k,
+                               void* y_bf16, fe_stream_t stream);
+
+/* The stack on HOST buffers: copies the inputs and the logits of every layer
+ * [n_layers][T][E] to the device (one copy each), runs fe_moe_stack_forward,
+ * copies the outputs back and waits for the stream.  chained = 0: x
+ * [n_layers][T][H] in, y [n_layers][T][H] out (independent layers); chained
+ * = 1: x [T][H] is layer 0's input, each layer feeds the next, y [T][H] is the
+ * last layer's output.  Synchronous. */
+fe_status fe_moe_stack_forward_host(fe_moe_stack_t s, const uint16_t* x_bf16_host, const float* logits_host, int T,
+                                    int top_k, uint16_t* y_bf16_host, int chained, fe_stream_t stream);
+
+/* Free the stack's buffers (not the layers).  Waits for the device first. */
+void fe_moe_stack_destroy(fe_moe_stack_t s);
 
 /* Text of the last CUDA failure behind an FE_ERR_CUDA / FE_ERR_OOM returned to
  * this thread ("" if none); static thread-local storage. */

@@ -98,12 +98,8 @@ def _experts(E: int, experts) -> np.ndarray:
     return ex
 
 
-def weights_gate_up(seed: int, E: int, H: int, I: int, experts=None) -> np.ndarray:
-    """Unquantised fused gate_up weights, float32 [n_experts, H, 2I].
-
-    Columns [0, I) are W_gate[e] (tensor 0), columns [I, 2I) are W_up[e]
-    (tensor 1); element (e, k, n) of either has flat index (e*H + k)*I + n.
-    """
+def _weights_gate_up_np(seed: int, E: int, H: int, I: int, experts=None) -> np.ndarray:
+    """The numpy definition of weights_gate_up (see there)."""
     ex = _experts(E, experts)
     out = np.empty((ex.size, H, 2 * I), dtype=np.float32)
     kn = (np.arange(H, dtype=np.uint64)[:, None] * np.uint64(I)
@@ -115,8 +111,8 @@ def weights_gate_up(seed: int, E: int, H: int, I: int, experts=None) -> np.ndarr
     return out
 
 
-def weights_down(seed: int, E: int, I: int, H: int, experts=None) -> np.ndarray:
-    """Unquantised down weights, float32 [n_experts, I, H]; flat index (e*I + k)*H + n."""
+def _weights_down_np(seed: int, E: int, I: int, H: int, experts=None) -> np.ndarray:
+    """The numpy definition of weights_down (see there)."""
     ex = _experts(E, experts)
     out = np.empty((ex.size, I, H), dtype=np.float32)
     kn = (np.arange(I, dtype=np.uint64)[:, None] * np.uint64(H)
@@ -127,15 +123,45 @@ def weights_down(seed: int, E: int, I: int, H: int, experts=None) -> np.ndarray:
     return out
 
 
+def weights_gate_up(seed: int, E: int, H: int, I: int, experts=None) -> np.ndarray:
+    """Unquantised fused gate_up weights, float32 [n_experts, H, 2I].
+
+    Columns [0, I) are W_gate[e] (tensor 0), columns [I, 2I) are W_up[e]
+    (tensor 1); element (e, k, n) of either has flat index (e*H + k)*I + n.
+    Drawn by the host C copy of the generator when it is built (identical
+    values, pinned against the numpy definition), else by numpy.
+    """
+    ex = _experts(E, experts)
+    lib = _host_lib()
+    if lib is None:
+        return _weights_gate_up_np(seed, E, H, I, experts)
+    out = np.empty((ex.size, H, 2 * I), dtype=np.float32)
+    exa = np.ascontiguousarray(ex, dtype=np.int64)
+    lib.synth_host_gate_up(out.ctypes.data, seed, H, I, exa.ctypes.data, ex.size)
+    return out
+
+
+def weights_down(seed: int, E: int, I: int, H: int, experts=None) -> np.ndarray:
+    """Unquantised down weights, float32 [n_experts, I, H]; flat index (e*I + k)*H + n."""
+    ex = _experts(E, experts)
+    lib = _host_lib()
+    if lib is None:
+        return _weights_down_np(seed, E, I, H, experts)
+    out = np.empty((ex.size, I, H), dtype=np.float32)
+    exa = np.ascontiguousarray(ex, dtype=np.int64)
+    lib.synth_host_down(out.ctypes.data, seed, I, H, exa.ctypes.data, ex.size)
+    return out
+
+
 def activations_bf16(seed: int, T: int, H: int) -> np.ndarray:
     """x as bfloat16 bit patterns, uint16 [T, H]."""
-    z = normal_f32(seed, TID_X, np.arange(T * H, dtype=np.uint64)).reshape(T, H)
+    z = normal_range_f32(seed, TID_X, 0, T * H).reshape(T, H)
     return bf16_bits_rne(z)
 
 
 def router_logits(seed: int, T: int, E: int, zipf_s: float | None = None) -> np.ndarray:
     """Router logits float32 [T, E]; optional Zipf(s) per-expert bias -s*ln(e+1)."""
-    z = normal_f32(seed, TID_LOGITS, np.arange(T * E, dtype=np.uint64)).reshape(T, E)
+    z = normal_range_f32(seed, TID_LOGITS, 0, T * E).reshape(T, E)
     if zipf_s is not None:
         bias = np.array([-zipf_s * math.log(e + 1) for e in range(E)], dtype=np.float64)
         z = (z + bias.astype(np.float32)[None, :]).astype(np.float32)
@@ -157,6 +183,58 @@ WORKLOADS = {
 }
 STACK_LAYERS = 48
 STACK_SEED0 = 1000
+
+
+# -- host C copy of the generator (synth_host.c, built into libfe_synth_host.so) ----
+
+_HOST_SRC = None
+_HOST_LIB = None
+_HOST_TRIED = False
+
+
+def build_host(force: bool = False) -> str:
+    """Compile synth_host.c with gcc (OpenMP, no FMA contraction, no fast-math)."""
+    import os
+    import subprocess
+    here = os.path.dirname(os.path.abspath(__file__))
+    src = os.path.join(here, "synth_host.c")
+    out = os.path.join(here, "libfe_synth_host.so")
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+                               "-ffp-contract=off", "-o", tmp, src])
+        os.replace(tmp, out)
+    return out
+
+
+def _host_lib():
+    """The host C generator, built on first use; None if it cannot be built."""
+    global _HOST_LIB, _HOST_TRIED
+    if _HOST_LIB is None and not _HOST_TRIED:
+        _HOST_TRIED = True
+        try:
+            import ctypes
+            lib = ctypes.CDLL(build_host())
+            P, u64, i64 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64
+            lib.synth_host_gate_up.argtypes = [P, u64, i64, i64, P, i64]
+            lib.synth_host_down.argtypes = [P, u64, i64, i64, P, i64]
+            lib.synth_host_normal.argtypes = [P, u64, u64, u64, i64]
+            for f in (lib.synth_host_gate_up, lib.synth_host_down, lib.synth_host_normal):
+                f.restype = ctypes.c_int
+            _HOST_LIB = lib
+        except (OSError, FileNotFoundError, Exception):   # no compiler: numpy definition only
+            _HOST_LIB = None
+    return _HOST_LIB
+
+
+def normal_range_f32(seed: int, tid: int, first: int, count: int) -> np.ndarray:
+    """normal_f32(seed, tid, first .. first + count - 1), by the C copy when built."""
+    lib = _host_lib()
+    if lib is None:
+        return normal_f32(seed, tid, np.arange(first, first + count, dtype=np.uint64))
+    out = np.empty(count, dtype=np.float32)
+    lib.synth_host_normal(out.ctypes.data, seed, tid, first, count)
+    return out
 
 
 # -- device copy of the generator (synth.cu, built into libfe_synth.so) ----------

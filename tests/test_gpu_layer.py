@@ -22,22 +22,67 @@ def torch_cuda():
     return torch
 
 
-def check_routing(orc, logits, k, E, idx, w, off, sp):
+def check_routing(orc, logits, k, E, idx, w, off, sp, counts=None, pair_row=None):
     idx_ref, w_ref = orc.route(logits, k)
-    counts, off_ref, sp_ref, _ = orc.group(idx_ref, E)
+    counts_ref, off_ref, sp_ref, pr_ref = orc.group(idx_ref, E)
     assert np.array_equal(idx, idx_ref), "router indices differ"
     np.testing.assert_allclose(w, w_ref, rtol=1e-6, atol=1e-7)
     assert np.array_equal(off, off_ref), "expert offsets differ"
     assert np.array_equal(sp, sp_ref), "grouped pair order differs"
+    if counts is not None:
+        assert np.array_equal(counts, counts_ref), "per-expert pair counts differ"
+    if pair_row is not None:
+        assert np.array_equal(pair_row, pr_ref), "inverse permutation (pair -> grouped row) differs"
 
 
-def run_and_check(gl, osd, x, lg, k, sample=None, what=""):
+def run_and_check(gl, osd, x, lg, k, sample=None, what="", y_ref=None):
     orc = oracle.default()
     y, idx, w, off, sp = gl.forward(x, lg, k)
-    check_routing(orc, lg, k, gl.E, idx, w, off, sp)
+    check_routing(orc, lg, k, gl.E, idx, w, off, sp, *gl.last_grouping)
     rows = np.arange(x.shape[0]) if sample is None else np.asarray(sample)
-    y_ref, _ = osd.forward(x[rows], lg[rows], k)
+    if y_ref is None:
+        y_ref, _ = osd.forward(x[rows], lg[rows], k)
     return harness.assert_output_close(y[rows], y_ref, what)
+
+
+def covering_rows(logits, k, E, tile=256, group=32, at_least=256, seed=0):
+    """Token rows whose pairs touch, for every expert, its first and last
+    grouped row and every 32-row epilogue group of every 256-row tile (so a
+    second tile of an expert with more than 256 pairs is covered), topped up
+    with random rows to at least `at_least`.  Chosen from the oracle's routing."""
+    orc = oracle.default()
+    idx, _ = orc.route(logits, k)
+    counts, off, sp, _ = orc.group(idx, E)
+    chosen = set()
+    covered = set()
+    pos_cell = {}
+    for e in range(E):
+        o, c = int(off[e]), int(counts[e])
+        for r in range(c):
+            pos_cell[o + r] = (e, r // tile, (r % tile) // group)
+    # cells a token covers, through the inverse permutation
+    _, _, _, pr = orc.group(idx, E)
+    def cells_of(tok):
+        return {pos_cell[int(pr[tok * k + j])] for j in range(k)}
+    for e in range(E):
+        o, c = int(off[e]), int(counts[e])
+        if c == 0:
+            continue
+        for pos in (o, o + c - 1):
+            t = int(sp[pos]) // k
+            chosen.add(t)
+            covered |= cells_of(t)
+    for pos in sorted(pos_cell):
+        if pos_cell[pos] not in covered:
+            t = int(sp[pos]) // k
+            chosen.add(t)
+            covered |= cells_of(t)
+    rng = np.random.default_rng(seed)
+    T = logits.shape[0]
+    while len(chosen) < min(at_least, T):
+        chosen.add(int(rng.integers(0, T)))
+    assert covered == set(pos_cell.values())
+    return np.array(sorted(chosen))
 
 
 def test_device_generator_matches_host(torch_cuda):
@@ -150,7 +195,7 @@ def test_decode_e128_t64_zipf(torch_cuda):
     idx, _ = oracle.default().route(lg, k)
     counts = np.bincount(idx.reshape(-1), minlength=E)
     assert (counts == 0).sum() > 0 and counts.max() > 32   # skewed, some experts empty
-    run_and_check(gl, osd, x, lg, k, sample=np.arange(0, 64, 3), what="t64 zipf")
+    run_and_check(gl, osd, x, lg, k, what="t64 zipf (all 64 rows)")
 
 
 @pytest.mark.parametrize("seed,T", [(4, 1), (5, 1), (4, 4), (5, 4)])
@@ -183,14 +228,27 @@ def _cached_oracle(E, H, I, seed):
     return _ORACLES[key]
 
 
+_PREFILL_REF = {}
+
+
 @pytest.mark.parametrize("path", ["gemv", "tc"])
-def test_prefill_t4096_sampled(torch_cuda, path):
+def test_prefill_t4096_covering_rows(torch_cuda, path):
+    """T=4096: routing and grouping compared on all 4096 tokens; y on a row set
+    that touches every expert's first and last grouped row and every 32-row
+    epilogue group of every 256-row tile (several hundred rows)."""
     import fp4_expert_gemv_b200 as fe
     cfg, seed, x, lg = harness.workload_inputs("prefill_e128_t4096")
     E, H, I, k, T = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"], cfg["T"]
     gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=k, path=PATHS[path])
-    osd = harness.OracleSide(E, H, I, seed)
-    run_and_check(gl, osd, x, lg, k, sample=[0, 1, 2047, 4095], what="prefill sampled")
+    if "rows" not in _PREFILL_REF:
+        rows = covering_rows(lg, k, E)
+        assert len(rows) >= 256
+        osd = harness.OracleSide(E, H, I, seed)
+        _PREFILL_REF["rows"] = rows
+        _PREFILL_REF["y"] = osd.forward(x[rows], lg[rows], k)[0]
+    rows = _PREFILL_REF["rows"]
+    run_and_check(gl, None, x, lg, k, sample=rows, y_ref=_PREFILL_REF["y"],
+                  what=f"prefill, {len(rows)} covering rows, path {path}")
     if path == "tc":
         assert gl.layer.last_forward_info()[0] == fe.PATH_TCGEN05
     _LAYERS.clear()
@@ -316,14 +374,20 @@ def test_fused_routing_cases(torch_cuda, E, k, T):
         assert gl.layer.last_forward_info()[0] == fe.PATH_FUSED_DECODE, what
 
 
-def test_large_activations_use_power_of_two_shift(torch_cuda):
+@pytest.mark.parametrize("path", ["auto", "gemv", "tc"])
+@pytest.mark.parametrize("scale", [3e5, 1e-4, 1e-8])
+def test_activation_magnitudes_use_power_of_two_shift(torch_cuda, scale, path):
+    """x far from unit scale: rows are staged in fp16 with a power-of-two shift
+    that puts each row's maximum in [2^14, 2^15), so |x| ~ 1e6 does not
+    overflow and |x| ~ 1e-8 (act ~ 1e-17) keeps fp16's precision."""
     E, H, I, seed = 8, 256, 128, 0
-    gl = harness.GpuLayer(E, H, I, seed, max_T=4, max_k=2, source="host")
+    T = 40 if path == "tc" else 4
+    gl = harness.GpuLayer(E, H, I, seed, max_T=T, max_k=2, source="host", path=PATHS[path])
     osd = harness.OracleSide(E, H, I, seed)
-    x = synth.activations_bf16(60, 4, H)
-    big = synth.bf16_bits_rne(synth.bf16_bits_to_f32(x) * np.float32(3e5))
-    lg = synth.router_logits(60, 4, E)
-    run_and_check(gl, osd, big, lg, 2, what="|x| up to ~1e6")
+    x = synth.activations_bf16(60, T, H)
+    xs = synth.bf16_bits_rne(synth.bf16_bits_to_f32(x) * np.float32(scale))
+    lg = synth.router_logits(60, T, E)
+    run_and_check(gl, osd, xs, lg, 2, what=f"|x| ~ {scale:g}, path {path}")
 
 
 def test_nan_logit_sets_status(torch_cuda):

@@ -60,3 +60,24 @@ def test_zipf_bias_skews_routing():
     counts = np.bincount(top.reshape(-1), minlength=cfg["E"])
     assert (counts == 0).sum() > 20          # some experts receive no token
     assert counts.max() >= 48                # the hottest expert takes most tokens
+
+
+def test_host_c_generator_equals_numpy_definition():
+    """The C copy of the generator (used to draw the oracle's weights quickly)
+    gives the numpy definition's values bit for bit."""
+    assert synth._host_lib() is not None, "gcc build of synth_host.c failed"
+    E, H, I = 7, 96, 64
+    ex = [6, 0, 3]
+    assert np.array_equal(synth.weights_gate_up(21, E, H, I, experts=ex).view(np.uint32),
+                          synth._weights_gate_up_np(21, E, H, I, experts=ex).view(np.uint32))
+    assert np.array_equal(synth.weights_down(21, E, I, H, experts=ex).view(np.uint32),
+                          synth._weights_down_np(21, E, I, H, experts=ex).view(np.uint32))
+    got = synth.normal_range_f32(5, synth.TID_LOGITS, 1000, 4096)
+    ref = synth.normal_f32(5, synth.TID_LOGITS, np.arange(1000, 5096, dtype=np.uint64))
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # a full-size expert at the 30B-like shape, spot-checked against the definition
+    W = synth.weights_gate_up(1000, 128, 2048, 768, experts=[77])
+    rows = np.array([0, 1, 1023, 2047], dtype=np.uint64)
+    flat = np.uint64(77 * 2048 * 768) + rows[:, None] * np.uint64(768) + np.arange(768, dtype=np.uint64)[None, :]
+    assert np.array_equal(W[0, rows.astype(np.int64), 768:],
+                          synth.normal_f32(1000, synth.TID_UP, flat) * synth.WEIGHT_STD)
