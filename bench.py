@@ -49,7 +49,7 @@ NOMINAL_FP4_TFLOPS = 9000.0
 L2_BYTES = 126e6
 PATH_NAMES = {1: "moderate-T path: routing + streaming mma.sync projections (sg_kernel) + ordered combine",
               2: "large-T path: routing + tensor-core tiles (tc_gemm_kernel) + ordered combine",
-              3: "decode_kernel (whole layer in one launch)"}
+              3: "single-launch decode; a stack at T=1 runs as one persistent launch (stack_decode_kernel)"}
 CSRC = os.path.join(ROOT, "fp4_expert_gemv_b200", "csrc")
 
 # DRAM bytes (read + write) per launch of a workload's dominant kernel, read
@@ -353,6 +353,7 @@ def run_workload(name, args, device, world, rank, headline=False):
         stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
     torch.cuda.synchronize()
     path, kernels_per_layer = handles[0].last_forward_info()
+    launches_per_step = stack.last_launches()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
@@ -389,6 +390,32 @@ def run_workload(name, args, device, world, rank, headline=False):
     ms = max_over_ranks(ms_local, world, device)
     tokens_step = sum_over_ranks(layers * T, world, device)
     value = tokens_step / (ms / 1e3)
+
+    # the same stack with one launch per layer (cross-layer streaming off; it applies
+    # at T = 1): each layer then starts its weight stream when its own launch starts,
+    # as a layer whose routing is only known once its own logits exist
+    no_prefetch = None
+    if T == 1:
+        stack.set_prefetch(False)
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=s):
+            stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
+        for _ in range(args.warmup):
+            g2.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(cur)
+        for _ in range(args.steps):
+            g2.replay()
+        e1.record(cur)
+        torch.cuda.synchronize()
+        ms2_local = e0.elapsed_time(e1) / args.steps
+        ms2 = max_over_ranks(ms2_local, world, device)
+        no_prefetch = {"ms_per_step": ms2, "us_per_layer": ms2_local * 1e3 / layers,
+                       "value": tokens_step / (ms2 / 1e3), "unit": "tokens/s"}
+        del g2
+        stack.set_prefetch(True)
 
     # parity of the timed graph's outputs: layers 0 and 47 against the oracle
     parity = None
@@ -430,6 +457,10 @@ def run_workload(name, args, device, world, rank, headline=False):
                     "frac_of_nominal_fp4_9pflops": tf / NOMINAL_FP4_TFLOPS}
     else:
         achieved = bytes_step / (ms_local / 1e3) / 1e9
+        if no_prefetch is not None:
+            a2 = bytes_step / (no_prefetch["ms_per_step"] / 1e3) / 1e9
+            no_prefetch["hbm_gbs"] = a2
+            no_prefetch["frac"] = a2 / float(peaks["hbm_gbs"])
         roofline = {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                     "frac": achieved / float(peaks["hbm_gbs"]), "traffic": traffic,
                     "kernel": PATH_NAMES.get(path, str(path)), "peak_kind": f"{peak_kind} HBM copy",
@@ -448,8 +479,8 @@ def run_workload(name, args, device, world, rank, headline=False):
                 "ms_per_step": e2e_ms,
                 "call": "fe_moe_stack_forward_host on pinned host buffers (every layer's x and logits in, y out; "
                         "synchronous)"},
-        "gpu_launches": kernels_per_layer * layers * args.steps,
-        "kernels_per_layer": kernels_per_layer,
+        "gpu_launches": launches_per_step * args.steps,
+        "launches_per_step": launches_per_step,
         "setup_s": setup_s,
         "l2": (f"inputs larger than L2: each step streams {layers} layers' routed experts ({bytes_step / 1e9:.2f} GB)"
                if bytes_step > L2_BYTES else
@@ -457,6 +488,8 @@ def run_workload(name, args, device, world, rank, headline=False):
     }
     if parity is not None:
         res["parity"] = parity
+    if no_prefetch is not None:
+        res["one_launch_per_layer"] = no_prefetch
     del g
     stack.close()
     for m in handles:
@@ -507,6 +540,8 @@ def run_gpu(args):
     }
     if "parity" in head:
         line["parity"] = head["parity"]
+    if "one_launch_per_layer" in head:
+        line["one_launch_per_layer"] = head["one_launch_per_layer"]
     if extra:
         line["workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

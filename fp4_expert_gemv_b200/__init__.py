@@ -67,6 +67,9 @@ _SIGS = {
     "fe_moe_stack_forward": (_st, [_P, _P, _P, _i32, _i32, _P, _P]),
     "fe_moe_stack_forward_host": (_st, [_P, _P, _P, _i32, _i32, _P, _i32, _P]),
     "fe_moe_stack_destroy": (None, [_P]),
+    "fe_moe_stack_set_prefetch": (_st, [_P, _i32]),
+    "fe_moe_stack_last_launches": (_i32, [_P]),
+    "fe_moe_set_exchange_test": (_st, [_P, _i32, ctypes.c_uint64]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -235,6 +238,13 @@ class Stack:
         check(fe_moe_stack_forward_host(self.h, hp(x_bf16_host), hp(logits_host), T, top_k, hp(y_bf16_host),
                                         1 if chained else 0, _stream_ptr(stream)), "fe_moe_stack_forward_host")
         return y_bf16_host
+
+    def set_prefetch(self, on: bool):
+        """Cross-layer streaming (one persistent launch at T=1) on or off."""
+        check(fe_moe_stack_set_prefetch(self.h, 1 if on else 0), "fe_moe_stack_set_prefetch")
+
+    def last_launches(self) -> int:
+        return fe_moe_stack_last_launches(self.h)
 
     def close(self):
         if getattr(self, "h", None):

@@ -19,6 +19,7 @@
 #include "pack.cuh"
 #include "route.cuh"
 #include "route_large.cuh"
+#include "stack_decode.cuh"
 #include "stream.cuh"
 #include "tcgen05.cuh"
 
@@ -36,6 +37,7 @@ struct fe_moe_s {
     // gate block and its up block, down blocks
     uint8_t* gu_blocks = nullptr;   // [E][I/16] x 18H bytes
     uint8_t* dn_blocks = nullptr;   // [E][H/16] x 9I bytes
+    uint8_t* dn_rows = nullptr;     // [E][I/32] x 18H bytes: W_dn in row groups (single-launch decode)
     bool loaded = false;
     // workspace
     int max_T = 0, max_k = 0;
@@ -50,9 +52,10 @@ struct fe_moe_s {
     int32_t* max_count = nullptr;
     float* act = nullptr;
     float* o = nullptr;
-    unsigned long long* dec_act = nullptr;  // fused decode: tagged act words by pair id
-    int32_t* plan = nullptr;                // fused decode: work split per nd
+    unsigned long long* dec_part = nullptr; // fused decode: [SMs][kDecMaxT][H] tagged per-CTA partial outputs
     unsigned long long* dec_epoch = nullptr;  // fused decode: per-CTA launch counts, then the arrival counter
+    uint32_t dec_plan[fe::kDecMaxT + 1][fe::kDecMaxPairs + 1] = {};   // weight bytes per (T, k); 0: not fused
+    bool dec_planned[fe::kDecMaxT + 1][fe::kDecMaxPairs + 1] = {};
     int32_t* sg_table = nullptr;            // streaming kernels: [2][SMs][4] work split
     unsigned long long* trace = nullptr;    // optional phase stamps (caller's buffer)
     // tensor-core path (tcgen05.cuh)
@@ -71,6 +74,8 @@ struct fe_moe_s {
     size_t weight_bytes = 0, work_bytes = 0;
     int last_T = 0, last_k = 0;
     int last_path = 0, last_kernels = 0;
+    int test_extra_arrivals = 0;            // fe_moe_set_exchange_test
+    unsigned long long exchange_timeout_ns = 200ull * 1000 * 1000;
 };
 
 struct fe_moe_stack_s {
@@ -79,6 +84,16 @@ struct fe_moe_stack_s {
     uint16_t* a_stage = nullptr;     // fe_moe_stack_forward_host: [n + 1][max_T][H] (inputs; chained: all)
     uint16_t* b_stage = nullptr;     // [n][max_T][H] (outputs of independent layers)
     float* logits_stage = nullptr;   // [n][max_T][E]
+    bool prefetch = true;            // one persistent launch streams the layers' weights back to back
+    // persistent launch (stack_decode.cuh): layer table, tagged partial outputs, counters
+    bool persistent_ok = false;      // shapes, sizes and occupancy allow it
+    uint32_t stk_smem = 0;
+    fe::StackLayer* d_layers = nullptr;        // [n] on the device
+    std::vector<fe::StackLayer> h_layers;      // the same on the host: the handles' buffers at creation
+    unsigned long long* part = nullptr;        // [3][SMs][H]
+    unsigned long long* ctr = nullptr;         // [SMs + 2]
+    int sm_count = 0;
+    int last_launches = 0;
 };
 
 namespace {
@@ -126,17 +141,16 @@ void free_workspace(fe_moe_s* h)
 {
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
-                    h->dec_act, h->dec_epoch, h->sg_table, h->plan, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
+                    h->dec_part, h->dec_epoch, h->sg_table, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
                     h->tc_tiles, h->tc_ntiles, h->grp_bh};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
     h->pair_row = nullptr; h->active = nullptr; h->n_active = nullptr; h->max_count = nullptr; h->act = nullptr;
     h->o = nullptr; h->status = nullptr; h->x_stage = nullptr; h->logits_stage = nullptr; h->y_stage = nullptr;
-    h->dec_act = nullptr;
+    h->dec_part = nullptr;
     h->dec_epoch = nullptr;
     h->sg_table = nullptr;
-    h->plan = nullptr;
     h->tc_x = nullptr; h->tc_xshift = nullptr; h->tc_act = nullptr; h->tc_ashift = nullptr;
     h->tc_tiles = nullptr; h->tc_ntiles = nullptr;
     h->grp_bh = nullptr;
@@ -163,53 +177,38 @@ int roundup32(int v) { return (v + 31) / 32 * 32; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Largest per-CTA weight bytes of the fused decode split over every possible
-// number of distinct routed experts, or 0 if T, top_k or the shape exceed the
-// fused kernel.
-size_t decode_weight_bytes(const fe_moe_s* h, int T, int k)
+// Shared-memory bytes the fused decode kernel reserves for weights at (T, k),
+// or 0 if the call is outside what it takes: T <= 8 tokens, T*k <= 16 pairs,
+// E <= 512, H <= 2048, at most kDecMaxUnits units per CTA for any number of
+// distinct routed experts, the whole plan within the device's shared memory,
+// and the kernel resident on every SM at once (its CTAs wait for each other).
+// Computed once per (T, k) and kept in the handle.
+uint32_t decode_weight_bytes(fe_moe_s* h, int T, int k)
 {
-    const int P = T * k;
-    if (P > fe::kDecMaxPairs || h->sm_count <= 0 || h->I > 1024 || h->E > fe::kDecMaxE) return 0;
-    size_t worst = 0;
-    const int nd_max = std::min(h->E, P);
-    std::vector<int> gf, df;
-    for (int nd = 1; nd <= nd_max; ++nd) {
-        fe::decode_split(nd, h->H, h->I, h->sm_count, gf, df);
-        for (int c = 0; c < h->sm_count; ++c) {
-            const int ngu = gf[c + 1] - gf[c], ndn = df[c + 1] - df[c];
-            if (ngu + ndn > fe::kDecMaxItems) return 0;
-            const size_t bytes = (size_t)ngu * 2 * fe::block_bytes(h->H) + (size_t)ndn * nd * fe::block_bytes(h->I);
-            worst = std::max(worst, bytes);
-        }
+    if (T < 1 || T > fe::kDecMaxT || k < 1 || k > fe::kDecMaxPairs || T * k > fe::kDecMaxPairs) return 0;
+    if (h->dec_planned[T][k]) return h->dec_plan[T][k];
+    uint32_t wb = 0;
+    const int nd_max = std::min(h->E, T * k);
+    const int U = fe::dec_units(nd_max, h->I);
+    const int units = (U + h->sm_count - 1) / h->sm_count;
+    if (h->E <= fe::kDecMaxE && h->H <= fe::kDecMaxH && h->I <= 1024 && h->sm_count > 0 &&
+        h->sm_count <= fe::kDecMaxCtas && units <= fe::kDecMaxUnits &&
+        h->dec_part != nullptr) {
+        const uint32_t w = ((uint32_t)units * fe::dec_unit_bytes(h->H) + 127u) / 128u * 128u;
+        const size_t total = fe::decode_smem_layout(w, T, h->H).total;
+        int per_sm = 0;
+        if (total <= (size_t)h->smem_optin &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fe::decode_kernel, fe::kDecThreads, total) ==
+                cudaSuccess &&
+            per_sm >= 1)
+            wb = w;
     }
-    return (worst + 127) / 128 * 128;
+    h->dec_plan[T][k] = wb;
+    h->dec_planned[T][k] = true;
+    return wb;
 }
 
-// Work-split table of the fused kernel: [nd][gate_up | down][CTA] first units.
-cudaError_t build_plan_table(fe_moe_s* h)
-{
-    const int cols = h->sm_count + 1;
-    std::vector<int32_t> tab((size_t)(fe::kDecMaxPairs + 1) * 2 * cols, 0);
-    std::vector<int> gf, df;
-    for (int nd = 1; nd <= fe::kDecMaxPairs; ++nd) {
-        fe::decode_split(nd, h->H, h->I, h->sm_count, gf, df);
-        for (int c = 0; c < cols; ++c) {
-            tab[((size_t)nd * 2 + 0) * cols + c] = gf[c];
-            tab[((size_t)nd * 2 + 1) * cols + c] = df[c];
-        }
-    }
-    cudaError_t e = cudaMalloc(&h->plan, tab.size() * sizeof(int32_t));
-    if (e != cudaSuccess) return e;
-    h->work_bytes += tab.size() * sizeof(int32_t);
-    return cudaMemcpy(h->plan, tab.data(), tab.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
-}
-
-size_t decode_smem_total(const fe_moe_s* h, size_t wbytes, int T, int k)
-{
-    return fe::decode_smem_layout((uint32_t)wbytes, T, k, h->H, h->I, h->E).total;
-}
-
-fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, int k, void* y, size_t wbytes,
+fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, int k, void* y, uint32_t wbytes,
                       cudaStream_t s)
 {
     fe::DecodeParams dp{};
@@ -217,21 +216,22 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     dp.logits = logits;
     dp.y = static_cast<uint16_t*>(y);
     dp.T = T; dp.E = h->E; dp.H = h->H; dp.I = h->I; dp.k = k;
-    dp.gu_blocks = h->gu_blocks; dp.dn_blocks = h->dn_blocks;
-    dp.plan = h->plan;
+    dp.gu_blocks = h->gu_blocks; dp.dn_rows = h->dn_rows;
     dp.idx = h->idx; dp.w = h->w; dp.counts = h->counts; dp.offsets = h->offsets;
     dp.sorted_pair = h->sorted_pair; dp.pair_row = h->pair_row;
-    dp.act = h->dec_act;
+    dp.part = h->dec_part;
     dp.epoch = h->dec_epoch;
     dp.trace = h->trace;
     dp.status = h->status;
     dp.timeout_ns = 200ull * 1000 * 1000;
-    dp.weight_bytes = (uint32_t)wbytes;
+    dp.exchange_timeout_ns = h->exchange_timeout_ns;
+    dp.extra_arrivals = h->test_extra_arrivals;
+    dp.weight_bytes = wbytes;
     dp.bulk_inputs = aligned16(x);   // 2*T*H bytes: a multiple of 16 (H % 64 == 0)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(h->sm_count);
     cfg.blockDim = dim3(fe::kDecThreads);
-    cfg.dynamicSmemBytes = decode_smem_total(h, wbytes, T, k);
+    cfg.dynamicSmemBytes = fe::decode_smem_layout(wbytes, T, h->H).total;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -568,6 +568,7 @@ fe_status fe_moe_create(int E, int H, int I, int group, fe_moe_t* out)
     // codes (K/2 bytes per column) + scales (K/32 bf16 per column), same bytes as the packed format
     if (e == cudaSuccess) e = dmalloc(&h->gu_blocks, (size_t)E * (I / 16) * 2 * fe::block_bytes(H), &acc);
     if (e == cudaSuccess) e = dmalloc(&h->dn_blocks, (size_t)E * (H / 16) * fe::block_bytes(I), &acc);
+    if (e == cudaSuccess) e = dmalloc(&h->dn_rows, (size_t)E * (I / 32) * 18 * (size_t)H, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->status, 1, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(uint32_t));
     if (e != cudaSuccess) {
@@ -607,8 +608,9 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = dmalloc(&h->x_stage, (size_t)max_T * h->H, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->logits_stage, (size_t)max_T * h->E, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->y_stage, (size_t)max_T * h->H, &acc);
-    if (e == cudaSuccess) e = dmalloc(&h->dec_act, (size_t)fe::kDecMaxPairs * h->I, &acc);
-    if (e == cudaSuccess) e = cudaMemset(h->dec_act, 0, sizeof(unsigned long long) * fe::kDecMaxPairs * h->I);
+    if (e == cudaSuccess) e = dmalloc(&h->dec_part, (size_t)h->sm_count * fe::kDecMaxT * h->H, &acc);
+    if (e == cudaSuccess)
+        e = cudaMemset(h->dec_part, 0, sizeof(unsigned long long) * (size_t)h->sm_count * fe::kDecMaxT * h->H);
     if (e == cudaSuccess) e = dmalloc(&h->dec_epoch, (size_t)h->sm_count + 1, &acc);
     if (e == cudaSuccess) e = dmalloc(&h->sg_table, 8 * (size_t)h->sm_count, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned long long) * ((size_t)h->sm_count + 1));
@@ -624,7 +626,8 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
         if (e == cudaSuccess) e = dmalloc(&h->tc_ntiles, 1, &acc);
     }
     h->work_bytes = 0;
-    if (e == cudaSuccess) e = build_plan_table(h);
+    for (auto& row : h->dec_planned)
+        for (bool& b : row) b = false;
     if (e != cudaSuccess) {
         keep_status = h->status;
         h->status = nullptr;
@@ -676,6 +679,10 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
     rp.src_codes = sdc; rp.src_scales = sds; rp.dst = h->dn_blocks;
     rp.K = I; rp.N = H; rp.gate_up = 0;
     fe::relayout_kernel<<<1184, 256, 0, s>>>(rp);
+    fe::RowRelayoutParams rr{};
+    rr.src_codes = sdc; rr.src_scales = sds; rr.dst = h->dn_rows;
+    rr.E = E; rr.I = I; rr.H = H;
+    fe::relayout_rows_kernel<<<1184, 256, 0, s>>>(rr);
     FE_CUDA_TRY(cudaGetLastError());
     // the tensor-core path needs every scale in the range where code x scale is an
     // exact f16; checked once here (this waits for the stream)
@@ -697,8 +704,13 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
     return FE_OK;
 }
 
-fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k, void* y_bf16,
-                         fe_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// The body of fe_moe_forward (also run by the stack for each of its layers).
+fe_status forward_impl(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k, void* y_bf16,
+                       fe_stream_t stream)
 {
     if (!h || T < 0 || top_k < 1 || top_k > h->E) return FE_ERR_INVALID_ARG;
     if (T == 0) return FE_OK;
@@ -716,8 +728,8 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     const int P = T * top_k;
 
     if (h->path == FE_PATH_AUTO || h->path == FE_PATH_FUSED_DECODE) {
-        const size_t wbytes = decode_weight_bytes(h, T, top_k);
-        if (wbytes > 0 && decode_smem_total(h, wbytes, T, top_k) <= (size_t)h->smem_optin) {
+        const uint32_t wbytes = decode_weight_bytes(h, T, top_k);
+        if (wbytes > 0) {
             fe_status st = decode_path(h, x_bf16, router_logits, T, top_k, y_bf16, wbytes, s);
             if (st == FE_OK) {
                 h->last_T = T;
@@ -760,6 +772,16 @@ fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_log
     const bool large_route = T >= kRouteLargeTokens && fe::route_large_ok(h->E, top_k);
     h->last_kernels = (large_route ? 4 : 1) + (use_tc ? 6 : 2) + 1;   // routing, projections, combine
     return FE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k, void* y_bf16,
+                         fe_stream_t stream)
+{
+    return forward_impl(h, x_bf16, router_logits, T, top_k, y_bf16, stream);
 }
 
 fe_status fe_moe_forward_host(fe_moe_t h, const uint16_t* x_host, const float* logits_host, int T, int top_k,
@@ -809,6 +831,43 @@ fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack
     if (e == cudaSuccess) e = dmalloc(&st->a_stage, ((size_t)n_layers + 1) * row, nullptr);
     if (e == cudaSuccess) e = dmalloc(&st->b_stage, (size_t)n_layers * row, nullptr);
     if (e == cudaSuccess) e = dmalloc(&st->logits_stage, (size_t)n_layers * st->max_T * st->E, nullptr);
+    // the persistent launch for one token: every layer of one shape, small enough, the
+    // kernel resident on every SM
+    st->sm_count = layers[0]->sm_count;
+    bool same = true;
+    for (int l = 1; l < n_layers; ++l) same &= layers[l]->I == layers[0]->I;
+    const int H = st->H, I = layers[0]->I;
+    if (e == cudaSuccess && same && n_layers <= fe::kStkMaxLayers && st->E <= fe::kDecMaxE && H <= fe::kDecMaxH &&
+        I <= 1024 && st->sm_count <= fe::kDecMaxCtas) {
+        const uint32_t smem = fe::stack_smem_layout(H).total;
+        int per_sm = 0;
+        if (smem <= (uint32_t)layers[0]->smem_optin &&
+            cudaFuncSetAttribute(fe::stack_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+                cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fe::stack_decode_kernel, fe::kStkThreads, smem) ==
+                cudaSuccess &&
+            per_sm >= 1) {
+            st->stk_smem = smem;
+            st->h_layers.resize(n_layers);
+            for (int l = 0; l < n_layers; ++l) {
+                fe_moe_s* h = layers[l];
+                st->h_layers[l] = fe::StackLayer{h->gu_blocks, h->dn_rows, h->idx, h->w, h->counts, h->offsets,
+                                                 h->sorted_pair, h->pair_row};
+            }
+            const size_t pbytes = sizeof(unsigned long long) * fe::kStkBufs * (size_t)st->sm_count * H;
+            e = cudaMalloc(reinterpret_cast<void**>(&st->part), pbytes);
+            if (e == cudaSuccess) e = cudaMemset(st->part, 0, pbytes);
+            if (e == cudaSuccess) e = dmalloc(&st->ctr, (size_t)st->sm_count + 2, nullptr);
+            if (e == cudaSuccess) e = cudaMemset(st->ctr, 0, sizeof(unsigned long long) * ((size_t)st->sm_count + 2));
+            if (e == cudaSuccess) e = dmalloc(&st->d_layers, (size_t)n_layers, nullptr);
+            if (e == cudaSuccess)
+                e = cudaMemcpy(st->d_layers, st->h_layers.data(), sizeof(fe::StackLayer) * n_layers,
+                               cudaMemcpyHostToDevice);
+            st->persistent_ok = e == cudaSuccess;
+        } else {
+            cudaGetLastError();   // a refused attribute leaves no error behind
+        }
+    }
     if (e != cudaSuccess) {
         fe_moe_stack_destroy(st);
         return record_cuda(e, "fe_moe_stack_create");
@@ -816,6 +875,77 @@ fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack
     *out = st;
     return FE_OK;
 }
+
+}  // extern "C"
+
+namespace {
+
+// Whether fe_moe_stack_forward can run the whole stack as one persistent launch:
+// one token, every layer on the single-launch decode kernel's shapes, the
+// layers' buffers unchanged since the stack was made, and x / y either chained
+// (y = x + H) or disjoint.  Returns 1 (independent), 2 (chained) or 0.
+int stack_persistent_mode(fe_moe_stack_s* st, const void* x, void* y, int T, int top_k)
+{
+    if (!st->persistent_ok || !st->prefetch || T != 1 || top_k > fe::kStkMaxK) return 0;
+    const int n = (int)st->layers.size();
+    for (int l = 0; l < n; ++l) {
+        fe_moe_s* h = st->layers[l];
+        if (h->path != FE_PATH_AUTO && h->path != FE_PATH_FUSED_DECODE) return 0;
+        if (decode_weight_bytes(h, 1, top_k) == 0) return 0;
+        const fe::StackLayer& s = st->h_layers[l];
+        if (s.gu_blocks != h->gu_blocks || s.dn_rows != h->dn_rows || s.idx != h->idx || s.w != h->w ||
+            s.counts != h->counts || s.offsets != h->offsets || s.sorted_pair != h->sorted_pair ||
+            s.pair_row != h->pair_row)
+            return 0;
+    }
+    const size_t bytes = sizeof(uint16_t) * (size_t)n * st->H;
+    const char* xb = static_cast<const char*>(x);
+    const char* yb = static_cast<const char*>(y);
+    if (yb == xb + sizeof(uint16_t) * st->H) return 2;
+    if (yb + bytes <= xb || xb + bytes <= yb) return 1;
+    return 0;
+}
+
+fe_status stack_persistent_launch(fe_moe_stack_s* st, const void* x, const float* logits, int top_k, void* y,
+                                  int mode, cudaStream_t s)
+{
+    fe_moe_s* h0 = st->layers[0];
+    fe::StackParams sp{};
+    sp.layers = st->d_layers;
+    sp.L = (int)st->layers.size();
+    sp.E = st->E; sp.H = st->H; sp.I = h0->I; sp.k = top_k;
+    sp.x = static_cast<const uint16_t*>(x);
+    sp.logits = logits;
+    sp.y = static_cast<uint16_t*>(y);
+    sp.chained = mode == 2;
+    sp.part = st->part;
+    sp.ctr = st->ctr;
+    sp.status = h0->status;
+    sp.timeout_ns = 200ull * 1000 * 1000;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(st->sm_count);
+    cfg.blockDim = dim3(fe::kStkThreads);
+    cfg.dynamicSmemBytes = st->stk_smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    FE_CUDA_TRY(cudaLaunchKernelEx(&cfg, fe::stack_decode_kernel, sp));
+    for (fe_moe_s* h : st->layers) {
+        h->last_T = 1;
+        h->last_k = top_k;
+        h->last_path = FE_PATH_FUSED_DECODE;
+        h->last_kernels = 0;
+    }
+    st->last_launches = 1;
+    return FE_OK;
+}
+
+}  // namespace
+
+extern "C" {
 
 fe_status fe_moe_stack_forward(fe_moe_stack_t st, const void* x_bf16, const float* logits, int T, int top_k,
                                void* y_bf16, fe_stream_t stream)
@@ -836,12 +966,21 @@ fe_status fe_moe_stack_forward(fe_moe_stack_t st, const void* x_bf16, const floa
     }
     const int n = (int)st->layers.size();
     const size_t xe = (size_t)T * st->H;
-    for (int l = 0; l < n; ++l) {
-        const fe_status r = fe_moe_forward(st->layers[l], static_cast<const uint16_t*>(x_bf16) + l * xe,
-                                           logits + (size_t)l * T * st->E, T, top_k,
-                                           static_cast<uint16_t*>(y_bf16) + l * xe, stream);
-        if (r != FE_OK) return r;
+    const int mode = stack_persistent_mode(st, x_bf16, y_bf16, T, top_k);
+    if (mode > 0) {
+        DeviceGuard g(st->device);
+        if (!g.ok) return FE_ERR_CUDA;
+        return stack_persistent_launch(st, x_bf16, logits, top_k, y_bf16, mode, (cudaStream_t)stream);
     }
+    int launches = 0;
+    for (int l = 0; l < n; ++l) {
+        const fe_status r = forward_impl(st->layers[l], static_cast<const uint16_t*>(x_bf16) + l * xe,
+                                         logits + (size_t)l * T * st->E, T, top_k,
+                                         static_cast<uint16_t*>(y_bf16) + l * xe, stream);
+        if (r != FE_OK) return r;
+        launches += st->layers[l]->last_kernels;
+    }
+    st->last_launches = launches;
     return FE_OK;
 }
 
@@ -869,12 +1008,24 @@ fe_status fe_moe_stack_forward_host(fe_moe_stack_t st, const uint16_t* x_host, c
     return FE_OK;
 }
 
+fe_status fe_moe_stack_set_prefetch(fe_moe_stack_t st, int on)
+{
+    if (!st) return FE_ERR_INVALID_ARG;
+    st->prefetch = on != 0;
+    return FE_OK;
+}
+
+int fe_moe_stack_last_launches(fe_moe_stack_t st) { return st ? st->last_launches : -1; }
+
 void fe_moe_stack_destroy(fe_moe_stack_t st)
 {
     if (!st) return;
     {
         DeviceGuard g(st->device);
         cudaDeviceSynchronize();
+        if (st->part) cudaFree(st->part);
+        if (st->ctr) cudaFree(st->ctr);
+        if (st->d_layers) cudaFree(st->d_layers);
         if (st->a_stage) cudaFree(st->a_stage);
         if (st->b_stage) cudaFree(st->b_stage);
         if (st->logits_stage) cudaFree(st->logits_stage);
@@ -934,6 +1085,14 @@ fe_status fe_moe_set_path(fe_moe_t h, int path)
     return FE_OK;
 }
 
+fe_status fe_moe_set_exchange_test(fe_moe_t h, int unreachable, unsigned long long wait_ns)
+{
+    if (!h || wait_ns == 0) return FE_ERR_INVALID_ARG;
+    h->test_extra_arrivals = unreachable ? 1 : 0;
+    h->exchange_timeout_ns = unreachable ? wait_ns : 200ull * 1000 * 1000;
+    return FE_OK;
+}
+
 fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf)
 {
     if (!h) return FE_ERR_INVALID_ARG;
@@ -956,7 +1115,7 @@ void fe_moe_destroy(fe_moe_t h)
         DeviceGuard g(h->device);
         cudaDeviceSynchronize();
         free_workspace(h);
-        void* ptrs[] = {h->gu_blocks, h->dn_blocks};
+        void* ptrs[] = {h->gu_blocks, h->dn_blocks, h->dn_rows};
         for (void* p : ptrs)
             if (p) cudaFree(p);
     }

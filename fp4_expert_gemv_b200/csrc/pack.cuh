@@ -135,4 +135,66 @@ __global__ void relayout_kernel(RelayoutParams p)
     }
 }
 
+// Re-layout of the down matrices into row groups for the single-launch decode
+// kernel, which multiplies 16 act values of one expert (the act columns a CTA
+// computed) by the 16 matching rows of W_dn for every output column h.  Per
+// expert, per group of 32 rows i (one scale group along K = I), one
+// contiguous run of 18H bytes:
+//   [codes of rows 32g .. 32g+15][scales of group g][codes of rows 32g+16 .. 32g+31]
+// so a unit of 16 rows is one contiguous 10H-byte copy (its codes and the
+// group's scales, in either order) and two units of one group are one 18H copy.
+// Codes of 16 rows x H columns, in the order of the mma.m16n8k16 A fragment
+// whose 16 rows are 16 output columns h and whose K is the 16 rows i: byte
+// 16L + 4s + j of quad q (512 bytes) belongs to column tile t = 4q + s (16
+// columns), lane L = 4g + c, and holds the source byte of row pair c + 4(j>>1)
+// (rows 2c, 2c+1, or 2c+8, 2c+9 of the 16) at column 16t + g + 8(j&1).
+// Scales: word g of column tile t (8 words per tile) holds the bf16 scales of
+// columns 16t + g (low half) and 16t + g + 8 (high half).
+struct RowRelayoutParams {
+    const uint8_t* src_codes;    // [E][I/2][H]
+    const uint16_t* src_scales;  // [E][I/32][H]
+    uint8_t* dst;                // [E][I/32] groups of 18H bytes
+    int64_t E, I, H;
+};
+
+// One thread per destination 4-byte word.
+__global__ void relayout_rows_kernel(RowRelayoutParams p)
+{
+    const int64_t H = p.H, G = p.I / 32;
+    const int64_t half_words = 2 * H;           // 8H bytes of codes
+    const int64_t scale_words = H / 2;          // 2H bytes of scales
+    const int64_t per_group = 2 * half_words + scale_words;
+    const int64_t total = p.E * G * per_group;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t w = i % per_group, eg = i / per_group;   // eg = e * G + g
+        const int64_t e = eg / G, g = eg % G;
+        uint8_t* dst = p.dst + eg * 18 * H;
+        if (w < half_words || w >= half_words + scale_words) {
+            const int half = w < half_words ? 0 : 1;
+            const int64_t wc = half == 0 ? w : w - half_words - scale_words;
+            const int64_t q = wc / 128, r = wc % 128;
+            const int L = (int)(r / 4), sidx = (int)(r % 4);
+            const int gg = L >> 2, c = L & 3;
+            const int64_t tile = 4 * q + sidx;
+            const int64_t row_pair0 = (32 * g + 16 * half) / 2;   // first byte row of the 16 rows
+            uint32_t v = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t krow = row_pair0 + c + 4 * (j >> 1);
+                const int64_t col = 16 * tile + gg + 8 * (j & 1);
+                v |= (uint32_t)p.src_codes[(e * (p.I / 2) + krow) * H + col] << (8 * j);
+            }
+            const int64_t base = half == 0 ? 0 : 10 * H;
+            *reinterpret_cast<uint32_t*>(dst + base + 512 * q + 16 * L + 4 * sidx) = v;
+        } else {
+            const int64_t ws = w - half_words;     // scale word: tile ws / 8, g' = ws % 8
+            const int64_t tile = ws / 8, gg = ws % 8;
+            const uint16_t* srow = p.src_scales + (e * G + g) * H;
+            const uint32_t lo = srow[16 * tile + gg], hi = srow[16 * tile + gg + 8];
+            *reinterpret_cast<uint32_t*>(dst + 8 * H + 4 * ws) = lo | (hi << 16);
+        }
+    }
+}
+
 }  // namespace fe

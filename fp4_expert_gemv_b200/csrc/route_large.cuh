@@ -19,7 +19,7 @@
 #pragma once
 
 #include "common.cuh"
-#include "decode.cuh"   // warp_route, warp_softmax
+#include "warp_route.cuh"
 #include "route.cuh"    // RouteParams
 
 namespace fe {

@@ -92,18 +92,21 @@ FE_DEV uint32_t sg_smem(const void* p) { return (uint32_t)__cvta_generic_to_shar
 
 FE_DEV void sg_bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kSgComputeWarps) : "memory"); }
 
+// Bounded wait for phase `parity` (test_wait polling: no suspension past the
+// completion, which try_wait was seen to add).
 FE_DEV bool sg_wait(uint32_t bar, uint32_t parity, unsigned long long timeout_ns)
 {
     uint32_t ok = 0;
-    const unsigned long long t0 = globaltimer_ns();
-    for (;;) {
+    unsigned long long t0 = 0;
+    for (int it = 0;; ++it) {
         asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
             : "r"(bar), "r"(parity)
             : "memory");
         if (ok) return true;
-        if (globaltimer_ns() - t0 > timeout_ns) return false;
+        if (it == 0) t0 = globaltimer_ns();
+        else if ((it & 15) == 0 && globaltimer_ns() - t0 > timeout_ns) return false;
     }
 }
 

@@ -68,7 +68,7 @@ typedef enum {
 /* Device-side problem bits, reported through fe_moe_get_status. */
 #define FE_DEVICE_BAD_EXPERT 0x1   /* an expert id outside [0, E) reached a kernel */
 #define FE_DEVICE_NAN_LOGIT 0x2    /* a NaN router logit (treated as -inf) */
-#define FE_DEVICE_EXCHANGE_TIMEOUT 0x4  /* single-launch decode: act from other CTAs never arrived */
+#define FE_DEVICE_EXCHANGE_TIMEOUT 0x4  /* single-launch decode: other CTAs' partial outputs never arrived */
 #define FE_DEVICE_LOAD_TIMEOUT 0x8      /* a weight copy into shared memory never completed */
 #define FE_DEVICE_TC_TIMEOUT 0x10       /* a tensor-core tile gave up waiting for its MMAs */
 
@@ -156,7 +156,8 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
                                    streaming kernels, or one CTA per unit when their ring does not fit */
 #define FE_PATH_TCGEN05 2       /* routing + tcgen05 tensor-core tiles + combine (large T; I % 128 == 0,
                                    H % 256 == 0, scales in the exact-f16 range) */
-#define FE_PATH_FUSED_DECODE 3  /* one cooperative kernel for the whole layer (T * top_k <= 16) */
+#define FE_PATH_FUSED_DECODE 3  /* one kernel for the whole layer (T <= 8, T * top_k <= 16), its CTAs all
+                                   resident at once (checked from the occupancy; otherwise not taken) */
 
 /* Force a compute path (FE_PATH_*); FE_ERR_UNSUPPORTED from forward if the
  * forced path cannot run the call.  For tests and measurements. */
@@ -167,19 +168,26 @@ fe_status fe_moe_set_path(fe_moe_t h, int path);
 fe_status fe_moe_last_forward_info(fe_moe_t h, int* path, int* kernels);
 
 /* Diagnostics: when device_buf (device memory, [number of SMs][64] uint64)
- * is set, every CTA of the fused decode kernel writes stamps of its phases
- * there: slot i (0..31) holds %globaltimer in ns and slot 32 + i the SM's
- * clock64 at the same point (0 start, 8 previous grid done, 10 routed,
- * 12 routing shared, 9 grouped, 15 barriers armed, 1 loads issued, 2 x
- * staged, 11 / 13 first / last gate_up unit landed, 16-19 first gate_up
- * unit: mma done, partials shared, reduced, done, 3 gate_up done, 14 down
- * weights landed, 4 act read back, 6 first down unit landed, 20 / 7 / 21
- * first down unit: mma done, partials shared, reduced, 5 end).  Slots a
- * CTA does not reach keep their old contents.  The streaming kernels of the
- * moderate-T path write [2][number of SMs][8] instead (gate_up, then down;
- * per CTA clock64 at start, range known, first unit landed, end; its unit
- * count; %globaltimer at start and end).  NULL switches it off. */
+ * is set, every CTA of the single-launch decode kernel writes stamps of its
+ * phases there: slot i (0..31) holds %globaltimer in ns and slot 32 + i the
+ * SM's clock64 at the same point (0 start, 8 previous grid done, 10 routed,
+ * 9 grouped, 1 copies issued, 2 x staged, 11 / 13 first / last unit's
+ * gate_up bytes landed, 3 units done, 26 every CTA arrived (CTAs that sum an
+ * output slice), 5 end).  Slots a CTA does not reach keep their old
+ * contents.  The streaming kernels of the moderate-T path write
+ * [2][number of SMs][8] instead (gate_up, then down; per CTA clock64 at
+ * start, range known, first unit landed, end; its unit count; %globaltimer
+ * at start and end).  NULL switches it off. */
 fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf);
+
+/* For tests of the failure path: with unreachable = 1 the single-launch
+ * decode kernel's CTAs that sum an output slice wait for one arrival more than
+ * the launch has (it never comes) for at most wait_ns nanoseconds, then set
+ * FE_DEVICE_EXCHANGE_TIMEOUT and leave their slice of y unwritten; every wait
+ * on the CTA's own copies keeps its full bound, so no copy is in flight when a
+ * CTA returns.  unreachable = 0 restores the normal wait (bounded at 200 ms).
+ * No counterpart on the pages. */
+fe_status fe_moe_set_exchange_test(fe_moe_t h, int unreachable, unsigned long long wait_ns);
 
 /* Human-readable text of a status code (static storage). */
 const char* fe_moe_status_string(fe_status s);
@@ -253,8 +261,10 @@ fe_status fe_moe_noalloc_get_routing(int E, int T, int top_k, int32_t* idx, floa
 typedef struct fe_moe_stack_s* fe_moe_stack_t;
 
 /* Build a stack over n_layers >= 1 handles, which it does not own (they must
- * outlive the stack): all on one device, with the same E and H, each reserved
- * and loaded.  Allocates staging for fe_moe_stack_forward_host: x and y of
+ * outlive the stack and keep the reservation they had when it was made; a
+ * layer reserved again afterwards makes the stack fall back to one launch per
+ * layer): all on one device, with the same E and H, each reserved and
+ * loaded.  Allocates staging for fe_moe_stack_forward_host: x and y of
  * every layer ([n_layers (+1)][max_T][H] bf16, max_T the smallest
  * reservation among the layers) and the logits of every layer. */
 fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack_t* out);
@@ -278,6 +288,26 @@ fe_status fe_moe_stack_forward(fe_moe_stack_t s, const void* x_bf16, const float
  * last layer's output.  Synchronous. */
 fe_status fe_moe_stack_forward_host(fe_moe_stack_t s, const uint16_t* x_bf16_host, const float* logits_host, int T,
                                     int top_k, uint16_t* y_bf16_host, int chained, fe_stream_t stream);
+
+/* Cross-layer streaming on (1, the default) or off (0).  On: a call at T = 1
+ * whose layers all take the single-launch decode kernel (same shape, x and y
+ * chained as y = x + H or not overlapping) runs the whole stack as ONE
+ * persistent launch, one CTA per SM: every layer is routed up front (the stack
+ * takes every layer's logits at once), each CTA streams its share of the
+ * layers' weights through a ring of shared-memory slots without stopping at
+ * layer boundaries, so the next layer's weights arrive while the current one
+ * finishes ("FireEcho Engine", "Benchmark Results": row L2, the next layer
+ * fetched ahead of use, and row L6, the 48-layer forward as one graph).
+ * Device-side problems of that launch are reported through the first layer's
+ * handle (fe_moe_get_status).  Off, or any other call: one fe_moe_forward per
+ * layer.  Both are bit-reproducible run to run; they differ from each other in
+ * how the per-CTA partial outputs are grouped before the fixed-order sum, so
+ * their outputs agree to within rounding, not bit for bit. */
+fe_status fe_moe_stack_set_prefetch(fe_moe_stack_t s, int on);
+
+/* Kernels the last fe_moe_stack_forward enqueued (1 for the persistent
+ * launch); -1 for a NULL stack. */
+int fe_moe_stack_last_launches(fe_moe_stack_t s);
 
 /* Free the stack's buffers (not the layers).  Waits for the device first. */
 void fe_moe_stack_destroy(fe_moe_stack_t s);

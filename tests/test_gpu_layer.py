@@ -313,8 +313,8 @@ def test_edge_cases(torch_cuda, path):
     lg_hot[:, 5] += 100.0
     run_and_check(gl, osd, x, lg_hot, 1, what="all tokens to one expert")
     run_and_check(gl, osd, x, lg_hot, 2, what="one hot expert, k=2")
-    # 12 tokens on one expert through the single-launch kernel: two 8-token blocks
-    run_and_check(gl, osd, x[:12], lg_hot[:12], 1, what="one hot expert, T=12, k=1")
+    # 8 tokens on one expert through the single-launch kernel: a full 8-column block
+    run_and_check(gl, osd, x[:8], lg_hot[:8], 1, what="one hot expert, T=8, k=1")
     if path == "auto":
         assert gl.layer.last_forward_info()[0] == fe.PATH_FUSED_DECODE
     # ties: equal logits everywhere, and pairwise ties
@@ -501,3 +501,23 @@ def test_argument_errors(torch_cuda):
         assert fe.fe_moe_forward(h2, 16, 16, 1, 2, 32, None) == fe.FE_ERR_UNSUPPORTED
     finally:
         fe.fe_moe_destroy(h2)
+
+
+def test_exchange_timeout_reports_and_recovers(torch_cuda):
+    """The single-launch kernel's wait for the other CTAs runs out (it waits for
+    an arrival that never comes, bounded at 20 us): the status reports
+    FE_DEVICE_EXCHANGE_TIMEOUT and the next normal forward is oracle-correct."""
+    import fp4_expert_gemv_b200 as fe
+    cfg, seed, x, lg = harness.workload_inputs("decode_e128_t1")
+    E, H, I, k = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"]
+    gl = harness.GpuLayer(E, H, I, seed, max_T=1, max_k=k)
+    osd = harness.OracleSide(E, H, I, seed)
+    fe.check(fe.fe_moe_set_exchange_test(gl.layer.h, 1, 20000))
+    gl.forward(x, lg, k)
+    assert gl.layer.last_forward_info()[0] == fe.PATH_FUSED_DECODE
+    st, bits = gl.layer.status()
+    assert st == fe.FE_ERR_DEVICE_STATUS and bits & fe.FE_DEVICE_EXCHANGE_TIMEOUT
+    fe.check(fe.fe_moe_set_exchange_test(gl.layer.h, 0, 1))
+    run_and_check(gl, osd, x, lg, k, what="decode after a timed-out exchange")
+    st, bits = gl.layer.status()
+    assert st == fe.FE_OK and bits == 0

@@ -52,6 +52,18 @@ def test_stack_graph_layers_0_and_last_match_oracle(torch_cuda, name):
     torch.cuda.synchronize()
     y = y_dev.view(torch.int16).cpu().numpy()
     assert np.array_equal(y, y_direct), "graph replay differs from the direct stack forward"
+    if T == 1:
+        # one launch per layer instead of the persistent launch: the same layer, the
+        # cross-CTA sums grouped differently (the persistent split rotates per layer)
+        stack.set_prefetch(False)
+        with torch.cuda.stream(s):
+            stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
+        torch.cuda.synchronize()
+        y_per = y_dev.view(torch.int16).cpu().numpy().view(np.uint16)
+        for l in range(layers):
+            harness.assert_output_close(y.view(np.uint16)[l], harness.bf16_to_f64(y_per[l]),
+                                        f"{name}: persistent against per-layer launches, layer {l}")
+        stack.set_prefetch(True)
     y = y.view(np.uint16)
     rows = np.arange(T) if T <= 8 else np.unique(np.linspace(0, T - 1, 24).astype(np.int64))
     for l in (0, layers - 1):
@@ -107,4 +119,70 @@ def test_stack_chaining_and_host_forms(torch_cuda):
     # y overlapping x of the same layer is refused before anything runs
     assert fe.fe_moe_stack_forward(stack.h, x_dev.data_ptr(), lg_dev.data_ptr(), T, k, x_dev.data_ptr() + 2,
                                    None) == fe.FE_ERR_INVALID_ARG
+    stack.close()
+
+
+@pytest.mark.parametrize("E,H,I,k", [(8, 256, 128, 2), (128, 2048, 768, 8)])
+def test_persistent_stack_one_token(torch_cuda, E, H, I, k):
+    """At T = 1 the stack runs as one persistent launch (every layer routed up
+    front, the weights streamed through a shared-memory ring across layer
+    boundaries).  Independent and chained layers, against the oracle layer by
+    layer (chained: the first two layers, whose inputs are still far from
+    zero), and against one launch per layer."""
+    torch = torch_cuda
+    import fp4_expert_gemv_b200 as fe
+    n = 6
+    layers = []
+    for l in range(n):
+        if H <= 256:
+            gl = harness.GpuLayer(E, H, I, 500 + l, max_T=1, max_k=k, source="host")
+        else:
+            gl = harness.GpuLayer(E, H, I, 500 + l, max_T=1, max_k=k)
+        layers.append(gl.layer)
+    stack = fe.Stack(layers)
+    xs = np.stack([synth.activations_bf16(510 + l, 1, H) for l in range(n)])
+    lg = np.ascontiguousarray(np.stack([synth.router_logits(520 + l, 1, E) for l in range(n)]), dtype=np.float32)
+    lg_dev = torch.from_numpy(lg).cuda()
+    x_dev = torch.from_numpy(xs.view(np.int16)).cuda()
+    # independent layers: one launch
+    y1 = torch.empty_like(x_dev)
+    for _ in range(3):   # repeated launches: tags and counters of later launches
+        stack.forward(x_dev.view(torch.bfloat16), lg_dev, k, y1.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert stack.last_launches() == 1
+    ya = y1.cpu().numpy().view(np.uint16)
+    for l in range(n):
+        osd = harness.OracleSide(E, H, I, 500 + l)
+        harness.assert_output_close(ya[l], osd.forward(xs[l], lg[l], k)[0], f"persistent, layer {l}")
+    # the same with one launch per layer
+    stack.set_prefetch(False)
+    y2 = torch.empty_like(x_dev)
+    stack.forward(x_dev.view(torch.bfloat16), lg_dev, k, y2.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert stack.last_launches() == n
+    yb = y2.cpu().numpy().view(np.uint16)
+    for l in range(n):
+        harness.assert_output_close(ya[l], harness.bf16_to_f64(yb[l]), f"persistent against per-layer, layer {l}")
+    stack.set_prefetch(True)
+    # chained: y = x shifted by one layer
+    buf = torch.zeros((n + 1, 1, H), dtype=torch.int16, device="cuda")
+    buf[0].copy_(x_dev[0])
+    for _ in range(2):
+        stack.forward(buf[0:].view(torch.bfloat16), lg_dev, k, buf[1:].view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert stack.last_launches() == 1
+    yc = buf.cpu().numpy().view(np.uint16)
+    chain = harness.oracle_chain(500, 2, xs[0][0], lg[:2, 0, :], k, E, H, I)
+    for l in range(2):
+        harness.assert_output_close(yc[l + 1], chain[l][0].reshape(1, H), f"persistent chained, layer {l}")
+    # and against one launch per layer, chained the same way
+    stack.set_prefetch(False)
+    buf2 = torch.zeros_like(buf)
+    buf2[0].copy_(x_dev[0])
+    stack.forward(buf2[0:].view(torch.bfloat16), lg_dev, k, buf2[1:].view(torch.bfloat16))
+    torch.cuda.synchronize()
+    yd = buf2.cpu().numpy().view(np.uint16)
+    harness.assert_output_close(yc[1], harness.bf16_to_f64(yd[1]), "chained, layer 0 against per-layer")
+    st, bits = layers[0].status()
+    assert st == fe.FE_OK and bits == 0
     stack.close()
