@@ -57,6 +57,18 @@ FE_DEV bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long timeout_
     }
 }
 
+// 16 bytes global -> shared by this thread, cached in L2 only (never a stale L1
+// line of data another SM wrote); complete after cp_async_wait_all.
+FE_DEV void cp_async16_cg(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+FE_DEV void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 FE_DEV void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -82,6 +94,13 @@ FE_DEV unsigned long long ld_relaxed_u64(const unsigned long long* p)
 {
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+FE_DEV ulonglong2 ld_relaxed_u64x2(const unsigned long long* p)
+{
+    ulonglong2 v;
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
     return v;
 }
 

@@ -91,7 +91,7 @@ struct fe_moe_stack_s {
     fe::StackLayer* d_layers = nullptr;        // [n] on the device
     std::vector<fe::StackLayer> h_layers;      // the same on the host: the handles' buffers at creation
     unsigned long long* part = nullptr;        // [3][SMs][H]
-    unsigned long long* ctr = nullptr;         // [SMs + 2]
+    unsigned long long* ctr = nullptr;         // [SMs + 2 kStkBufs]
     int sm_count = 0;
     int last_launches = 0;
 };
@@ -857,8 +857,8 @@ fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack
             const size_t pbytes = sizeof(unsigned long long) * fe::kStkBufs * (size_t)st->sm_count * H;
             e = cudaMalloc(reinterpret_cast<void**>(&st->part), pbytes);
             if (e == cudaSuccess) e = cudaMemset(st->part, 0, pbytes);
-            if (e == cudaSuccess) e = dmalloc(&st->ctr, (size_t)st->sm_count + 2, nullptr);
-            if (e == cudaSuccess) e = cudaMemset(st->ctr, 0, sizeof(unsigned long long) * ((size_t)st->sm_count + 2));
+            if (e == cudaSuccess) e = dmalloc(&st->ctr, (size_t)st->sm_count + 2 * fe::kStkBufs, nullptr);
+            if (e == cudaSuccess) e = cudaMemset(st->ctr, 0, sizeof(unsigned long long) * ((size_t)st->sm_count + 2 * fe::kStkBufs));
             if (e == cudaSuccess) e = dmalloc(&st->d_layers, (size_t)n_layers, nullptr);
             if (e == cudaSuccess)
                 e = cudaMemcpy(st->d_layers, st->h_layers.data(), sizeof(fe::StackLayer) * n_layers,
@@ -922,6 +922,7 @@ fe_status stack_persistent_launch(fe_moe_stack_s* st, const void* x, const float
     sp.ctr = st->ctr;
     sp.status = h0->status;
     sp.timeout_ns = 200ull * 1000 * 1000;
+    sp.trace = h0->trace;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(st->sm_count);
     cfg.blockDim = dim3(fe::kStkThreads);

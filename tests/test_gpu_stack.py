@@ -42,6 +42,8 @@ def test_stack_graph_layers_0_and_last_match_oracle(torch_cuda, name):
     with torch.cuda.stream(s):
         stack.forward(x_dev, lg_dev, k, y_dev, stream=s)
     torch.cuda.synchronize()
+    if T == 1:
+        assert stack.last_launches() == 1, "the one-token stack should run as one persistent launch"
     y_direct = y_dev.view(torch.int16).cpu().numpy().copy()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
@@ -184,5 +186,5 @@ def test_persistent_stack_one_token(torch_cuda, E, H, I, k):
     yd = buf2.cpu().numpy().view(np.uint16)
     harness.assert_output_close(yc[1], harness.bf16_to_f64(yd[1]), "chained, layer 0 against per-layer")
     st, bits = layers[0].status()
-    assert st == fe.FE_OK and bits == 0
+    assert st == fe.FE_OK and bits == 0, f"device status bits {bits:#x}"
     stack.close()
