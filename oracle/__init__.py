@@ -92,6 +92,8 @@ class Oracle:
         lib.orc_route.restype = i32
         lib.orc_group.argtypes = [P, i32, i32, i32, P, P, P, P]
         lib.orc_group.restype = i32
+        lib.orc_router_logits.argtypes = [P, P, i32, i32, i32, P]
+        lib.orc_router_logits.restype = i32
         lib.orc_moe_forward.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
         lib.orc_moe_forward.restype = i32
         self.lib = lib
@@ -128,6 +130,18 @@ class Oracle:
         w = np.empty((T, k), dtype=np.float32)
         _check(self.lib.orc_route(_ptr(logits), T, E, k, _ptr(idx), _ptr(w)), "route")
         return idx, w
+
+    def router_logits(self, x_bf16: np.ndarray, w_router_bf16: np.ndarray) -> np.ndarray:
+        """The router GEMM: x [T, H] (bf16 bits) times W_r [E, H] (bf16 bits, one row per
+        expert), transposed: float64 logits [T, E]."""
+        x_bf16 = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+        w = np.ascontiguousarray(w_router_bf16, dtype=np.uint16)
+        T, H = x_bf16.shape
+        E = w.shape[0]
+        assert w.shape == (E, H)
+        out = np.empty((T, E), dtype=np.float64)
+        _check(self.lib.orc_router_logits(_ptr(x_bf16), _ptr(w), T, H, E, _ptr(out)), "router_logits")
+        return out
 
     def group(self, idx: np.ndarray, E: int):
         idx = np.ascontiguousarray(idx, dtype=np.int32)

@@ -12,6 +12,8 @@
  * History"; the SiLU(gate)*up product of "FastInfer", section "Confirmed
  * elementwise SwiGLU scheduling"):
  *
+ *   0. router GEMM (when the logits are not given): logits[t][e] =
+ *      sum_h x[t][h] W_r[e][h], one bf16 row of W_r per expert, in fp64;
  *   1. router: per token, experts ordered by (logit descending, index
  *      ascending); the first k are the token's slots j = 0..k-1; the slot
  *      weights are the softmax of the k selected logits (fp64, stored fp32);
@@ -188,6 +190,29 @@ int orc_route(const float* logits, int T, int E, int k, int32_t* idx, float* w)
             w[(int64_t)t * k + j] = (float)(exp((double)l[idx[(int64_t)t * k + j]] - l0) / den);
     }
     free(taken);
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Router GEMM ("FireEcho Engine", section "Architecture": MoEFFN, the packed */
+/* MoE whose dispatch starts from the router's scores; "Speed Optimization   */
+/* History" step 1, the router in front of the grouped dispatch):           */
+/*   logits[t][e] = sum_{h = 0..H-1} x[t][h] * W_r[e][h]                    */
+/* x_bf16 [T][H], w_bf16 [E][H] (expert e's router row), logits [T][E] fp64; */
+/* each product of two bf16 values is exact in fp64, and the sum runs in    */
+/* the order h = 0, 1, ..., H-1.                                            */
+/* ---------------------------------------------------------------------- */
+int orc_router_logits(const uint16_t* x_bf16, const uint16_t* w_bf16, int T, int H, int E, double* logits)
+{
+    if (T < 0 || H <= 0 || E <= 0 || (T > 0 && (!x_bf16 || !w_bf16 || !logits))) return ORC_EINVAL;
+    for (int t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h)
+                acc += (double)orc_bf16_to_f32(x_bf16[(int64_t)t * H + h]) *
+                       (double)orc_bf16_to_f32(w_bf16[(int64_t)e * H + h]);
+            logits[(int64_t)t * E + e] = acc;
+        }
     return ORC_OK;
 }
 

@@ -14,7 +14,10 @@ oracle disagrees with:
   sort, the full softmax at k = E, and sum_j w = 1;
 * numpy's stable argsort for the grouping;
 * the closed form of a layer whose codes are all equal;
-* a dense, unpermuted brute-force layer written here with numpy.
+* a dense, unpermuted brute-force layer written here with numpy;
+* for the router GEMM: the closed form of all-equal weights (an exact sum by
+  math.fsum), one-hot rows (a permutation of x's columns, exactly), numpy's
+  dot product, and a router whose expert ranking is built in.
 """
 from __future__ import annotations
 
@@ -320,6 +323,72 @@ def check_bf16_output_rounding(o, rng):
         assert got == best[1], (v, hex(got), hex(best[1]))
 
 
+def _bf16_bits(v) -> np.ndarray:
+    """float64 values that are exact in bfloat16 -> their bit patterns."""
+    f = np.asarray(v, dtype=np.float32)
+    bits = (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    assert np.array_equal(bf16_to_f64(bits), np.asarray(v, dtype=np.float64)), "value not exact in bf16"
+    return bits
+
+
+def _random_bf16(rng, shape, scale=1.0) -> np.ndarray:
+    """Random bfloat16 bit patterns (float32 normal values truncated to bf16)."""
+    f = (rng.standard_normal(shape) * scale).astype(np.float32)
+    return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def check_router_gemm_equal_weights(o, rng):
+    """W_r[e][h] = c for all e, h: every logit of token t is c * sum_h x[t][h] (the sum
+    exact by math.fsum, then one rounding)."""
+    T, H, E = 3, 256, 5
+    x = _random_bf16(rng, (T, H))
+    c = 0.375
+    w = np.full((E, H), _bf16_bits([c])[0], dtype=np.uint16)
+    got = o.router_logits(x, w)
+    xs = bf16_to_f64(x)
+    for t in range(T):
+        ref = c * math.fsum(xs[t].tolist())
+        bound = 1e-15 * c * float(np.abs(xs[t]).sum())
+        assert np.all(np.abs(got[t] - ref) <= bound), (t, got[t], ref)
+
+
+def check_router_gemm_onehot(o, rng):
+    """W_r row e = the unit vector of column perm[e]: logit[t][e] = x[t][perm[e]] exactly
+    (a transposed operand or a wrong row/column index moves the values)."""
+    T, H, E = 4, 64, 7
+    x = _random_bf16(rng, (T, H))
+    perm = rng.permutation(H)[:E]
+    wv = np.zeros((E, H))
+    wv[np.arange(E), perm] = 1.0
+    got = o.router_logits(x, _bf16_bits(wv))
+    assert np.array_equal(got, bf16_to_f64(x)[:, perm]), (got, perm)
+
+
+def check_router_gemm_numpy(o, rng):
+    """Random bf16 x and W_r against numpy's float64 dot product."""
+    T, H, E = 5, 512, 9
+    x = _random_bf16(rng, (T, H))
+    w = _random_bf16(rng, (E, H), 0.05)
+    got = o.router_logits(x, w)
+    xs, ws = bf16_to_f64(x), bf16_to_f64(w)
+    ref = xs @ ws.T
+    bound = 1e-13 * (np.abs(xs) @ np.abs(ws).T)
+    assert np.all(np.abs(got - ref) <= bound)
+
+
+def check_router_gemm_ranking(o, rng):
+    """x = all ones, W_r row e = r_e (a constant row): logit e = H r_e, so the top-k
+    are the k largest r_e, largest first, with equal r broken by the lower index."""
+    H, E, k = 128, 10, 4
+    r = np.array([0.5, 2.0, -1.0, 3.0, 2.0, 0.25, 3.0, -2.0, 1.0, 0.0])
+    x = _bf16_bits(np.ones((2, H)))
+    w = _bf16_bits(np.repeat(r[:, None], H, axis=1))
+    lg = o.router_logits(x, w)
+    assert np.array_equal(lg, np.tile(H * r, (2, 1)))
+    idx, _ = o.route(lg.astype(np.float32), k)
+    assert idx[0].tolist() == [3, 6, 1, 4] and idx[1].tolist() == [3, 6, 1, 4], idx
+
+
 ALL_CHECKS = [
     ("e2m1_table", lambda o, rng: check_e2m1_table(o)),
     ("encode_bruteforce", check_encode_bruteforce),
@@ -331,4 +400,8 @@ ALL_CHECKS = [
     ("closed_form", check_closed_form),
     ("dense_bruteforce", check_dense_bruteforce),
     ("bf16_output_rounding", check_bf16_output_rounding),
+    ("router_gemm_equal_weights", check_router_gemm_equal_weights),
+    ("router_gemm_onehot", check_router_gemm_onehot),
+    ("router_gemm_numpy", check_router_gemm_numpy),
+    ("router_gemm_ranking", check_router_gemm_ranking),
 ]

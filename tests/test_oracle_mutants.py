@@ -28,6 +28,13 @@ MUTANTS = [
     ("group_unstable", "for (int64_t p = 0; p < P; ++p)\n            if (idx[p] == e) {",
      "for (int64_t p = P - 1; p >= 0; --p)\n            if (idx[p] == e) {"),
     ("bf16_round_half_up", "u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0x8000u;"),
+    ("router_gemm_transposed",
+     "(double)orc_bf16_to_f32(w_bf16[(int64_t)e * H + h]);",
+     "(double)orc_bf16_to_f32(w_bf16[(int64_t)h * E + e]);"),
+    ("router_gemm_drops_last_column", "for (int h = 0; h < H; ++h)\n                acc +=",
+     "for (int h = 0; h < H - 1; ++h)\n                acc +="),
+    ("router_gemm_first_token_only", "acc += (double)orc_bf16_to_f32(x_bf16[(int64_t)t * H + h]) *",
+     "acc += (double)orc_bf16_to_f32(x_bf16[h]) *"),
     ("down_scale_group", "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[(k / 32) * N + n]);",
      "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[((k / 32) / 2) * N + n]);"),
 ]
