@@ -499,6 +499,76 @@ def run_workload(name, args, device, world, rank, headline=False):
     return res
 
 
+def run_router(device):
+    """The router GEMM fused with the top-k (fe_moe_router) on the decode layer's router
+    (E 128, H 2048, top-8): at one token through 384 distinct W_r (192 MB, more than L2,
+    so each call reads its W_r from HBM), and at 4096 tokens (a tensor-core GEMM),
+    each timed over a CUDA graph of back-to-back calls."""
+    import torch
+
+    import fp4_expert_gemv_b200 as fe
+    E, H, k = 128, 2048, 8
+    peaks, src = measured_peaks()
+    out = {}
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4242)
+    for T, n in ((1, 384), (4096, 16)):
+        layer = fe.MoELayer(E, H, 64, T, k)
+        wr = (torch.randn((n, E, H), generator=gen, device=device) / H ** 0.5).to(torch.bfloat16)
+        x = torch.randn((T, H), generator=gen, device=device).to(torch.bfloat16)
+        lg = torch.empty((n, T, E), dtype=torch.float32, device=device)
+        idx = torch.empty((n, T, k), dtype=torch.int32, device=device)
+        w = torch.empty((n, T, k), dtype=torch.float32, device=device)
+        s = torch.cuda.Stream()
+
+        def calls():
+            for i in range(n):
+                fe.check(fe.fe_moe_router(layer.h, x.data_ptr(), wr[i].data_ptr(), T, k, lg[i].data_ptr(),
+                                          idx[i].data_ptr(), w[i].data_ptr(), s.cuda_stream), "fe_moe_router")
+
+        with torch.cuda.stream(s):
+            calls()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            calls()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(reps):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * n)
+        st, bits = layer.status()
+        rec = {"T": T, "E": E, "H": H, "top_k": k, "calls_per_graph": n, "us_per_call": us,
+               "status_bits": bits, "splits_of_K": None}
+        if T == 1:
+            nbytes = E * H * 2 + T * H * 2 + T * E * 4 + T * k * 8
+            gbs = nbytes / (us * 1e-6) / 1e9
+            rec.update({"bound": "hbm", "algorithmic_bytes": nbytes, "achieved": gbs, "unit": "GB/s",
+                        "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "peak_source": src,
+                        "note": "latency-bound at one token: 512 KB of W_r, one dependent chain of loads, "
+                                "partial sums, the last CTA's sum and top-k"})
+        else:
+            flops = 2.0 * T * E * H
+            tf = flops / (us * 1e-6) / 1e12
+            rec.update({"bound": "tensor", "flops": flops, "achieved": tf, "unit": "TFLOP/s",
+                        "peak": peaks["bf16_tflops"], "frac": tf / peaks["bf16_tflops"], "peak_source": src,
+                        "note": "mma.sync bf16 tiles of 16 tokens x 8 experts; a small GEMM (2.1 GFLOP)"})
+        del rec["splits_of_K"]
+        out[f"T{T}"] = rec
+        del g
+        layer.close()
+        del wr, x, lg, idx, w
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args):
     import torch
 
@@ -544,6 +614,8 @@ def run_gpu(args):
         line["one_launch_per_layer"] = head["one_launch_per_layer"]
     if extra:
         line["workloads"] = extra
+    if args.workload == "all":
+        line["router_gemm"] = run_router(device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
         reps = args.cpu_reps

@@ -70,6 +70,8 @@ _SIGS = {
     "fe_moe_stack_set_prefetch": (_st, [_P, _i32]),
     "fe_moe_stack_last_launches": (_i32, [_P]),
     "fe_moe_set_exchange_test": (_st, [_P, _i32, ctypes.c_uint64]),
+    "fe_moe_router": (_st, [_P, _P, _P, _i32, _i32, _P, _P, _P, _P]),
+    "fe_moe_forward_router": (_st, [_P, _P, _P, _i32, _i32, _P, _P, _P]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -151,6 +153,33 @@ class MoELayer:
         check(fe_moe_forward(self.h, _dptr(x_bf16), _dptr(logits), T, top_k, _dptr(y_bf16), _stream_ptr(stream)),
               "fe_moe_forward")
         return y_bf16
+
+    def router(self, x_bf16, w_router_bf16, top_k: int, logits=None, idx=None, w=None, stream=None):
+        """The router GEMM fused with the top-k: (logits [T, E] f32, idx [T, k] i32, w [T, k] f32)."""
+        import torch
+        T = x_bf16.shape[0]
+        dev = x_bf16.device
+        if logits is None:
+            logits = torch.empty((T, self.E), dtype=torch.float32, device=dev)
+        if idx is None:
+            idx = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+        if w is None:
+            w = torch.empty((T, top_k), dtype=torch.float32, device=dev)
+        check(fe_moe_router(self.h, _dptr(x_bf16), _dptr(w_router_bf16), T, top_k, _dptr(logits), _dptr(idx),
+                            _dptr(w), _stream_ptr(stream)), "fe_moe_router")
+        return logits, idx, w
+
+    def forward_router(self, x_bf16, w_router_bf16, top_k: int, y_bf16=None, logits=None, stream=None):
+        """The layer from x alone (router GEMM, top-k, layer): (y [T, H] bf16, logits [T, E] f32)."""
+        import torch
+        T = x_bf16.shape[0]
+        if y_bf16 is None:
+            y_bf16 = torch.empty((T, self.H), dtype=torch.bfloat16, device=x_bf16.device)
+        if logits is None:
+            logits = torch.empty((T, self.E), dtype=torch.float32, device=x_bf16.device)
+        check(fe_moe_forward_router(self.h, _dptr(x_bf16), _dptr(w_router_bf16), T, top_k, _dptr(y_bf16),
+                                    _dptr(logits), _stream_ptr(stream)), "fe_moe_forward_router")
+        return y_bf16, logits
 
     def forward_host(self, x_bf16_host, logits_host, top_k: int, y_bf16_host, stream=None):
         """Host (ideally pinned) numpy/torch CPU buffers in and out; synchronous."""

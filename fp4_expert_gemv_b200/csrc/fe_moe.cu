@@ -19,6 +19,7 @@
 #include "pack.cuh"
 #include "route.cuh"
 #include "route_large.cuh"
+#include "router.cuh"
 #include "stack_decode.cuh"
 #include "stream.cuh"
 #include "tcgen05.cuh"
@@ -67,6 +68,8 @@ struct fe_moe_s {
     int32_t* tc_tiles = nullptr;            // [max tiles][3]
     int32_t* tc_ntiles = nullptr;           // [1]
     int32_t* grp_bh = nullptr;              // grouping for many tokens: [P / kGroupChunk + 1][E]
+    float* rt_part = nullptr;               // router GEMM: K-split partials (router.cuh)
+    unsigned* rt_ticket = nullptr;          // router GEMM: per 16-token tile, CTAs done
     uint32_t* status = nullptr;
     uint16_t* x_stage = nullptr;
     float* logits_stage = nullptr;
@@ -142,7 +145,7 @@ void free_workspace(fe_moe_s* h)
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
                     h->dec_part, h->dec_epoch, h->sg_table, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
-                    h->tc_tiles, h->tc_ntiles, h->grp_bh};
+                    h->tc_tiles, h->tc_ntiles, h->grp_bh, h->rt_part, h->rt_ticket};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
@@ -154,6 +157,8 @@ void free_workspace(fe_moe_s* h)
     h->tc_x = nullptr; h->tc_xshift = nullptr; h->tc_act = nullptr; h->tc_ashift = nullptr;
     h->tc_tiles = nullptr; h->tc_ntiles = nullptr;
     h->grp_bh = nullptr;
+    h->rt_part = nullptr;
+    h->rt_ticket = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -615,6 +620,13 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
     if (e == cudaSuccess) e = dmalloc(&h->sg_table, 8 * (size_t)h->sm_count, &acc);
     if (e == cudaSuccess) e = cudaMemset(h->dec_epoch, 0, sizeof(unsigned long long) * ((size_t)h->sm_count + 1));
     if (e == cudaSuccess) e = dmalloc(&h->grp_bh, (P / fe::kGroupChunk + 1) * (size_t)h->E, &acc);
+    {
+        const size_t rt_floats = std::max((size_t)fe::kRtSplitFloats, (size_t)max_T * h->E);
+        const size_t tiles = ((size_t)max_T + fe::kRtTok - 1) / fe::kRtTok;
+        if (e == cudaSuccess) e = dmalloc(&h->rt_part, rt_floats, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->rt_ticket, tiles, &acc);
+        if (e == cudaSuccess) e = cudaMemset(h->rt_ticket, 0, sizeof(unsigned) * tiles);
+    }
     // fp16 token and act rows (row-major for the tensor-core tiles, fragment
     // order for the streaming kernels: each forward writes before it reads)
     if (e == cudaSuccess) e = dmalloc(&h->tc_x, (size_t)max_T * h->H, &acc);
@@ -774,9 +786,63 @@ fe_status forward_impl(fe_moe_t h, const void* x_bf16, const float* router_logit
     return FE_OK;
 }
 
+// The router GEMM fused with the top-k (router.cuh).
+fe_status router_impl(fe_moe_s* h, const void* x_bf16, const void* w_router_bf16, int T, int top_k, float* logits,
+                      int32_t* idx, float* w, cudaStream_t s)
+{
+    if (!h || T < 0 || top_k < 1 || top_k > h->E) return FE_ERR_INVALID_ARG;
+    if (T == 0) return FE_OK;
+    if (!x_bf16 || !w_router_bf16 || !logits) return FE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(w_router_bf16)) & 15u) return FE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(logits) & 3u) return FE_ERR_INVALID_ARG;
+    const int J = h->E <= 32 ? 1 : h->E <= 64 ? 2 : h->E <= 128 ? 4 : h->E <= 256 ? 8 : 16;
+    if (h->H % 64 != 0 || h->E > 512 || top_k > fe::kRtMaxK || top_k * J > fe::kRtCand) return FE_ERR_UNSUPPORTED;
+    if (!h->rt_part || T > h->max_T) return FE_ERR_CAPACITY;
+    fe::RouterParams rp;
+    rp.x = static_cast<const uint16_t*>(x_bf16);
+    rp.wr = static_cast<const uint16_t*>(w_router_bf16);
+    rp.T = T;
+    rp.H = h->H;
+    rp.E = h->E;
+    rp.k = top_k;
+    rp.ks = fe::router_splits(T, h->H, h->E);
+    rp.part = h->rt_part;
+    rp.ticket = h->rt_ticket;
+    rp.logits = logits;
+    rp.idx = idx;
+    rp.w = w;
+    rp.status = h->status;
+    const dim3 grid((T + fe::kRtTok - 1) / fe::kRtTok, (h->E + fe::kRtExp - 1) / fe::kRtExp, rp.ks);
+    fe::router_kernel<<<grid, fe::kRtThreads, 0, s>>>(rp);
+    FE_CUDA_TRY(cudaGetLastError());
+    return FE_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+fe_status fe_moe_router(fe_moe_t h, const void* x_bf16, const void* w_router_bf16, int T, int top_k, float* logits,
+                        int32_t* idx, float* w, fe_stream_t stream)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    return router_impl(h, x_bf16, w_router_bf16, T, top_k, logits, idx, w, (cudaStream_t)stream);
+}
+
+fe_status fe_moe_forward_router(fe_moe_t h, const void* x_bf16, const void* w_router_bf16, int T, int top_k,
+                                void* y_bf16, float* logits, fe_stream_t stream)
+{
+    if (!h) return FE_ERR_INVALID_ARG;
+    if (T > 0 && !h->loaded) return FE_ERR_NOT_LOADED;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    const fe_status st = router_impl(h, x_bf16, w_router_bf16, T, top_k, logits, nullptr, nullptr,
+                                     (cudaStream_t)stream);
+    if (st != FE_OK) return st;
+    return forward_impl(h, x_bf16, logits, T, top_k, y_bf16, stream);
+}
 
 fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k, void* y_bf16,
                          fe_stream_t stream)

@@ -122,6 +122,35 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uin
 fe_status fe_moe_forward(fe_moe_t h, const void* x_bf16, const float* router_logits, int T, int top_k,
                          void* y_bf16, fe_stream_t stream);
 
+/* The router GEMM fused with the top-k ("FireEcho Engine", "Architecture":
+ * MoEFFN, the packed MoE whose dispatch starts from the router's scores;
+ * "Speed Optimization History" step 1: the router in front of the grouped
+ * dispatch, expert ids chosen on the GPU).  In one launch:
+ *   logits[t][e] = sum_h x[t][h] * W_r[e][h]   (bf16 products, fp32 sums),
+ * then per token the top_k experts by logit (ties to the lower index) and the
+ * softmax of their logits, as fe_moe_forward routes.
+ *   x_bf16        device bf16 [T][H], 16-byte aligned (caller-owned, read);
+ *   w_router_bf16 device bf16 [E][H], one row per expert, 16-byte aligned;
+ *   logits        device float [T][E] (written);
+ *   idx, w        device int32 / float [T][top_k] in slot order (written), or
+ *                 NULL to skip.
+ * The sums run in fp32 in an order of the library's choosing (deterministic
+ * for given T, H, E): within sum_h |x W_r| * H * 2^-24 of the exact sum.  Needs
+ * H % 64 == 0, E <= 512, top_k <= 32 and top_k * ceil(E/32 rounded up to a
+ * power of two) <= 256 (else FE_ERR_UNSUPPORTED), T <= max_T (else
+ * FE_ERR_CAPACITY); misaligned or NULL required pointers: FE_ERR_INVALID_ARG.
+ * T = 0 is a no-op.  Asynchronous on stream, no allocation: capturable. */
+fe_status fe_moe_router(fe_moe_t h, const void* x_bf16, const void* w_router_bf16, int T, int top_k,
+                        float* logits, int32_t* idx, float* w, fe_stream_t stream);
+
+/* The layer from x alone: fe_moe_router (logits into the caller's `logits`,
+ * device float [T][E], which the call also returns), then fe_moe_forward on
+ * those logits.  Same argument rules as both; the layer's own routing (idx,
+ * w, grouping) is the router's, taken again from the same fp32 logits.
+ * Asynchronous on stream, no allocation. */
+fe_status fe_moe_forward_router(fe_moe_t h, const void* x_bf16, const void* w_router_bf16, int T, int top_k,
+                                void* y_bf16, float* logits, fe_stream_t stream);
+
 /* The layer on HOST buffers (no counterpart on the pages: the same layer as
  * fe_moe_forward for a caller whose x and logits are in host memory): copies
  * x and the logits to the device, runs

@@ -41,6 +41,7 @@ S_CENTER = 393210          # 12 * (2**16 - 1) / 2
 WEIGHT_STD = np.float32(0.02)
 
 TID_GATE, TID_UP, TID_DOWN, TID_X, TID_LOGITS = 0, 1, 2, 3, 4
+TID_ROUTER = 5
 
 _CHUNK = 1 << 22
 
@@ -166,6 +167,13 @@ def router_logits(seed: int, T: int, E: int, zipf_s: float | None = None) -> np.
         bias = np.array([-zipf_s * math.log(e + 1) for e in range(E)], dtype=np.float64)
         z = (z + bias.astype(np.float32)[None, :]).astype(np.float32)
     return np.ascontiguousarray(z, dtype=np.float32)
+
+
+def router_weights_bf16(seed: int, E: int, H: int) -> np.ndarray:
+    """Router rows W_r as bfloat16 bit patterns, uint16 [E, H]: N(0, 1) / sqrt(H), so that
+    with N(0, 1) activations the logits are about N(0, 1)."""
+    z = normal_range_f32(seed, TID_ROUTER, 0, E * H).reshape(E, H)
+    return bf16_bits_rne((z * np.float32(1.0 / math.sqrt(H))).astype(np.float32))
 
 
 # Workload recipes: shapes, seeds and value distributions of the five layer
