@@ -90,6 +90,12 @@ FE_DEV void st_relaxed_u64(unsigned long long* p, unsigned long long v)
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Two 64-bit words to a 16-byte aligned address.
+FE_DEV void st_relaxed_u64x2(unsigned long long* p, unsigned long long a, unsigned long long b)
+{
+    asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+
 FE_DEV unsigned long long ld_relaxed_u64(const unsigned long long* p)
 {
     unsigned long long v;

@@ -77,7 +77,8 @@ struct StackParams {
     const float* logits;        // layer l: logits + l*E
     uint16_t* y;                // layer l writes y + l*H
     int chained;                // y + l*H == x + (l+1)*H
-    unsigned long long* part;   // [kStkBufs][grid][H]: (tag << 32) | fp32 bits
+    unsigned long long* part;   // [kStkBufs][grid][H]: (tag << 32) | fp32 bits; within each 16-column
+                                //   tile, word 2g holds column g and word 2g + 1 column g + 8
     unsigned long long* ctr;    // [grid + 2 kStkBufs]: launches of CTA c; then per partial buffer b
                                 //   (the layers l with l % kStkBufs = b) the CTAs' arrivals, and
                                 //   then per buffer the output slices summed
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                     }
                     if (uniform(all_in)) {
                         const long long ts = htrace ? clock64() : 0;
-                        // lane (grp, cp) adds columns 16 sl + 2 cp, + 1 over CTAs grp, grp + 4,
+                        // lane (grp, cp) adds columns 16 sl + cp, + 8 over CTAs grp, grp + 4,
                         // ... in order, and the four groups are added in order.  Its 16-byte
                         // words first land in shared memory (cp.async: every load of the slice
                         // in flight at once, no registers held), one round trip in all
@@ -489,9 +490,11 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                         const float c0v = __shfl_sync(0xffffffffu, a0, cp + 8), c1v = __shfl_sync(0xffffffffu, a1, cp + 8);
                         const float d0 = __shfl_sync(0xffffffffu, a0, cp + 16), d1 = __shfl_sync(0xffffffffu, a1, cp + 16);
                         const float e0 = __shfl_sync(0xffffffffu, a0, cp + 24), e1 = __shfl_sync(0xffffffffu, a1, cp + 24);
-                        if (grp == 0 && !late) {
+                        if (grp == 0 && !late) {   // words 2cp, 2cp + 1 of a tile: columns cp, cp + 8
                             const uint32_t two = bf16x2_rn(((b0 + c0v) + d0) + e0, ((b1 + c1v) + d1) + e1);
-                            reinterpret_cast<uint32_t*>(p.y + (size_t)rl * H + 16 * sl)[cp] = two;
+                            uint16_t* yr = p.y + (size_t)rl * H + 16 * sl;
+                            yr[cp] = (uint16_t)(two & 0xffffu);
+                            yr[cp + 8] = (uint16_t)(two >> 16);
                         }
                         if (p.chained) __threadfence();   // the slice is visible before it is counted
                         __syncwarp();
@@ -662,19 +665,25 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
             if (!S.abort) {
                 unsigned long long* part = p.part + ((size_t)(l % kStkBufs) * G + c) * H;
                 const unsigned long long tg = (unsigned long long)stack_tag(epoch, L, l) << 32;
-                if (c4 == 0) {
+                // the token's outputs sit in the lanes (g, 0): columns g and g + 8 of each
+                // 16-column tile.  Lane (g, c4) takes tile 4q + c4 and stores its two columns
+                // side by side (words 2g, 2g + 1 of the tile) in one 16-byte store
 #pragma unroll
-                    for (int qs = 0; qs < kStkHQ; ++qs) {
-                        const int q = warp + kStkWarps * qs;
-                        if (q < nq) {
+                for (int qs = 0; qs < kStkHQ; ++qs) {
+                    const int q = warp + kStkWarps * qs;
+                    float v0 = 0.0f, v1 = 0.0f;
 #pragma unroll
-                            for (int s4 = 0; s4 < 4; ++s4) {
-                                const int h0 = 16 * (4 * q + s4) + g;
-                                st_relaxed_u64(part + h0, tg | __float_as_uint(Y[qs][s4][0]));
-                                st_relaxed_u64(part + h0 + 8, tg | __float_as_uint(Y[qs][s4][2]));
-                            }
+                    for (int s4 = 0; s4 < 4; ++s4) {
+                        const float a = __shfl_sync(0xffffffffu, Y[qs][s4][0], lane & ~3);
+                        const float b = __shfl_sync(0xffffffffu, Y[qs][s4][2], lane & ~3);
+                        if (c4 == s4) {
+                            v0 = a;
+                            v1 = b;
                         }
                     }
+                    if (q < nq)
+                        st_relaxed_u64x2(part + 16 * (4 * q + c4) + 2 * g, tg | __float_as_uint(v0),
+                                         tg | __float_as_uint(v1));
                 }
             }
             cbar();
