@@ -119,7 +119,6 @@ struct StackShared {
     int bshift;
     int xshift[2];                      // shift of the x row staged in xs buffer b
     volatile int xs_layer[2];           // layer whose x is staged in xs buffer b (exchange -> compute)
-    volatile int consumed;              // units the compute warps are done with (compute -> copy)
     volatile int layer_done;            // last layer whose units and partial are done (compute -> exchange)
     volatile int guard_ok;              // last layer whose partial buffer is free (sync -> compute)
     volatile int abort;
@@ -134,7 +133,7 @@ __host__ __device__ inline StackSmem stack_smem_layout(int H)
 {
     StackSmem L;
     L.mbar = (uint32_t)kStkSlots * dec_unit_bytes(H);
-    L.shared = L.mbar + 8 * (2 * kStkSlots + 2);
+    L.shared = L.mbar + 8 * (3 * kStkSlots + 2);
     L.red = align16(L.shared + (uint32_t)sizeof(StackShared));
     static_assert(kStkRedFloats * 4 >= kStkRouteWarps * kStkCand * 8, "routing candidates space");
     // after routing, the candidates' space holds the gate_up partials and, behind them,
@@ -192,6 +191,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
     auto bar_gu = [&](int s) { return mbar0 + 8u * (uint32_t)s; };
     auto bar_dn = [&](int s) { return mbar0 + 8u * (uint32_t)(kStkSlots + s); };
     auto bar_x = [&](int b) { return mbar0 + 8u * (uint32_t)(2 * kStkSlots + b); };
+    // slot s is free again once every compute warp has arrived (one arrival per warp per unit)
+    auto bar_empty = [&](int s) { return mbar0 + 8u * (uint32_t)(2 * kStkSlots + 2 + s); };
     const bool copier = warp == kStkWarps, exchanger = warp == kStkWarps + 1, syncer = warp == kStkWarps + 2;
     // diagnostics: compute thread 0's cycles per phase
     unsigned long long ph_acc[11] = {};
@@ -204,9 +205,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
 
     if (tid == 0) {
         for (int b = 0; b < 2 * kStkSlots + 2; ++b) mbar_init(mbar0 + 8u * b, 1);
+        for (int s = 0; s < kStkSlots; ++s) mbar_init(bar_empty(s), kStkWarps);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         S.abort = 0;
-        S.consumed = 0;
         S.layer_done = -1;
         S.guard_ok = kStkBufs - 1;   // the first kStkBufs layers' buffers are free
         S.xs_layer[0] = -1;
@@ -268,8 +269,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
 
     if (copier) {
         // ==== the copy warp: unit q of this CTA's sequence goes into slot q % 3 as soon
-        // as the compute warps are done with unit q - 3.  Lane 0 alone; nothing else in
-        // the loop, so that a freed slot is refilled at once.
+        // as every compute warp has arrived on the slot's empty barrier for unit q - 3.
+        // Lane 0 alone; nothing else in the loop, so that a freed slot is refilled at once.
         if (lane != 0) return;
         int total = 0;
         for (int l = 0; l < L; ++l) {
@@ -282,11 +283,10 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
         int issued = 0;
         for (; issued < total; ++issued) {
             if (issued >= kStkSlots) {
-                const unsigned long long t0 = globaltimer_ns();
-                bool gone = false;
-                while (S.consumed <= issued - kStkSlots && !S.abort && !gone)
-                    gone = globaltimer_ns() - t0 > p.timeout_ns;
-                if (gone) {
+                // use (issued - 3) / 3 of the slot: phases complete in order, and the next
+                // one cannot complete before this copy is issued
+                const uint32_t ph = (uint32_t)((issued - kStkSlots) / kStkSlots) & 1u;
+                if (!S.abort && !mbar_wait(bar_empty(issued % kStkSlots), ph, p.timeout_ns)) {
                     atomicOr(p.status, kDevBarrierTimeout);
                     S.abort = 1;
                 }
@@ -640,8 +640,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                     }
                 }
                 ph_end(kPhDown);
-                cbar();   // every compute warp is done with the slot
-                if (tid == 0) S.consumed = n + 1;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_empty(s));   // this warp is done with the slot
                 ph_end(kPhSlot);
                 if (tracing) ph_acc[kPhUnits] += 1;
             }
