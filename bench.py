@@ -52,17 +52,12 @@ PATH_NAMES = {1: "moderate-T path: routing + streaming mma.sync projections (sg_
               3: "single-launch decode; a stack at T=1 runs as one persistent launch (stack_decode_kernel)"}
 CSRC = os.path.join(ROOT, "fp4_expert_gemv_b200", "csrc")
 
-# DRAM bytes (read + write) per launch of a workload's dominant kernel, read
-# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# kernel built from the sources whose hash is given: reported only while the
-# sources still hash to that value, null otherwise (the counters would describe
-# another kernel).
-NCU_TRAFFIC = {
-    # workload: (bytes per launch, kernel, sha256[:16] of the source files listed)
-}
-TRAFFIC_SOURCES = {"decode_kernel": ["decode.cuh", "mma.cuh", "common.cuh"],
-                   "sg_kernel gate_up": ["stream.cuh", "mma.cuh", "common.cuh"],
-                   "tc_gemm_kernel gate_up": ["tcgen05.cuh", "mma.cuh", "common.cuh"]}
+# DRAM bytes (read + write) of a workload's dominant kernel come from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum), kept with the capture
+# command and a hash of the kernel's source files in profiles/traffic.json.  They
+# are reported only while those sources still hash to the captured value, null
+# otherwise (the counters would describe another kernel).
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def source_hash(files):
@@ -73,13 +68,20 @@ def source_hash(files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
-    if workload not in NCU_TRAFFIC:
+def ncu_traffic(workload, layers):
+    """(DRAM bytes per launch of the kernel that runs all `layers` layers, kernel name), or
+    (None, kernel) when the kernel changed since the capture, or (None, None)."""
+    if not os.path.exists(TRAFFIC_FILE):
         return None, None
-    nbytes, kernel, digest = NCU_TRAFFIC[workload]
-    if source_hash(TRAFFIC_SOURCES[kernel]) != digest:
-        return None, kernel
-    return nbytes, kernel
+    with open(TRAFFIC_FILE) as f:
+        entries = json.load(f).get("entries", [])
+    for ent in entries:
+        if ent.get("workload") != workload:
+            continue
+        if source_hash(ent["sources"]) != ent["sources_sha256_16"]:
+            return None, ent["kernel"]
+        return float(ent["dram_bytes_per_layer"]) * layers, ent["kernel"]
+    return None, None
 
 
 def bytes_per_expert(H, I):
@@ -444,7 +446,7 @@ def run_workload(name, args, device, world, rank, headline=False):
     bytes_layer = [algorithmic_bytes_per_layer(E, H, I, T, d) for d in distinct]
     bytes_step = float(sum(bytes_layer))
     us_layer = ms_local * 1e3 / layers
-    traffic, traffic_kernel = ncu_traffic(name)
+    traffic, traffic_kernel = ncu_traffic(name, layers) if launches_per_step == 1 else (None, None)
     prefill = name.startswith("prefill")
     if prefill:
         flops_layer = 2.0 * T * k * 3 * H * I
@@ -469,7 +471,8 @@ def run_workload(name, args, device, world, rank, headline=False):
                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS}
     if traffic_kernel:
         roofline["traffic_kernel"] = traffic_kernel
-        roofline["traffic_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum per launch"
+        roofline["traffic_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum per layer of an "
+                                    "8-layer capture x the layers of this launch (profiles/traffic.json)"
                                     if traffic is not None else "kernel changed since its ncu capture")
     res = {
         "workload": name, "E": E, "H": H, "I": I, "top_k": k, "T": T, "layers_per_step": layers,
