@@ -45,20 +45,24 @@ class ExpertWeights:
     """Per-expert packed buffers handed to the oracle (None = not materialised).
 
     gate_up codes uint8 [H/2, 2I] (gate columns, then up columns), scales
-    bf16 bits [H/32, 2I]; down codes uint8 [I/2, H], scales [I/32, H].
+    bf16 bits [H/32, 2I]; down codes uint8 [I/2, H], scales [I/32, H].  An
+    expert set with fmt=1 holds INT2 codes instead: [H/4, 2I] and [I/4, H].
     """
 
     def __init__(self, E: int, H: int, I: int):
         self.E, self.H, self.I = E, H, I
+        self.fmt = np.zeros(E, dtype=np.uint8)
         self.gu_codes = [None] * E
         self.gu_scales = [None] * E
         self.dn_codes = [None] * E
         self.dn_scales = [None] * E
 
-    def set(self, e: int, gu_codes, gu_scales, dn_codes, dn_scales):
+    def set(self, e: int, gu_codes, gu_scales, dn_codes, dn_scales, fmt: int = 0):
         H, I = self.H, self.I
-        assert gu_codes.shape == (H // 2, 2 * I) and gu_scales.shape == (H // 32, 2 * I)
-        assert dn_codes.shape == (I // 2, H) and dn_scales.shape == (I // 32, H)
+        per = 4 if fmt else 2
+        assert gu_codes.shape == (H // per, 2 * I) and gu_scales.shape == (H // 32, 2 * I)
+        assert dn_codes.shape == (I // per, H) and dn_scales.shape == (I // 32, H)
+        self.fmt[e] = 1 if fmt else 0
         self.gu_codes[e] = np.ascontiguousarray(gu_codes, dtype=np.uint8)
         self.gu_scales[e] = np.ascontiguousarray(gu_scales, dtype=np.uint16)
         self.dn_codes[e] = np.ascontiguousarray(dn_codes, dtype=np.uint8)
@@ -92,6 +96,16 @@ class Oracle:
         lib.orc_route.restype = i32
         lib.orc_group.argtypes = [P, i32, i32, i32, P, P, P, P]
         lib.orc_group.restype = i32
+        lib.orc_int2_decode.argtypes = [i32]
+        lib.orc_int2_decode.restype = ctypes.c_double
+        lib.orc_int2_encode.argtypes = [ctypes.c_float]
+        lib.orc_int2_encode.restype = i32
+        lib.orc_quantize_int2.argtypes = [P, i64, i64, i64, P, P]
+        lib.orc_quantize_int2.restype = i32
+        lib.orc_dequant_int2.argtypes = [P, P, i64, i64, i64]
+        lib.orc_dequant_int2.restype = ctypes.c_float
+        lib.orc_moe_forward_fmt.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]
+        lib.orc_moe_forward_fmt.restype = i32
         lib.orc_router_logits.argtypes = [P, P, i32, i32, i32, P]
         lib.orc_router_logits.restype = i32
         lib.orc_moe_forward.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
@@ -116,6 +130,26 @@ class Oracle:
         scales = np.empty((E, K // 32, N), dtype=np.uint16)
         _check(self.lib.orc_quantize(_ptr(W), E, K, N, _ptr(codes), _ptr(scales)), "quantize")
         return codes, scales
+
+    def int2_decode(self, code: int) -> float:
+        return self.lib.orc_int2_decode(int(code))
+
+    def int2_encode(self, r: float) -> int:
+        return self.lib.orc_int2_encode(float(r))
+
+    def quantize_int2(self, W: np.ndarray):
+        """float32 W [E, K, N] -> (INT2 codes uint8 [E, K/4, N], scales uint16 [E, K/32, N])."""
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        E, K, N = W.shape
+        codes = np.empty((E, K // 4, N), dtype=np.uint8)
+        scales = np.empty((E, K // 32, N), dtype=np.uint16)
+        _check(self.lib.orc_quantize_int2(_ptr(W), E, K, N, _ptr(codes), _ptr(scales)), "quantize_int2")
+        return codes, scales
+
+    def dequant_int2(self, codes: np.ndarray, scales: np.ndarray, k: int, n: int) -> float:
+        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+        scales = np.ascontiguousarray(scales, dtype=np.uint16)
+        return self.lib.orc_dequant_int2(_ptr(codes), _ptr(scales), codes.shape[-1], int(k), int(n))
 
     def dequant(self, codes: np.ndarray, scales: np.ndarray, k: int, n: int) -> float:
         """One dequantised weight of a single expert's [K/2, N] codes / [K/32, N] scales."""
@@ -165,25 +199,28 @@ class Oracle:
         y64 = np.zeros((T, H), dtype=np.float64)
         yb = np.zeros((T, H), dtype=np.uint16)
         act = np.zeros((T * k, I), dtype=np.float64) if want_act else None
-        rc = self.lib.orc_moe_forward(E, H, I, T, k, _ptr(x_bf16), _ptr(logits),
+        rc = self.lib.orc_moe_forward_fmt(E, H, I, T, k, _ptr(x_bf16), _ptr(logits), _ptr(weights.fmt),
                                       weights._ptrs(weights.gu_codes), weights._ptrs(weights.gu_scales),
                                       weights._ptrs(weights.dn_codes), weights._ptrs(weights.dn_scales),
                                       _ptr(y64), _ptr(yb), _ptr(act))
         _check(rc, "moe_forward")
         return (y64, yb, act) if want_act else (y64, yb)
 
-    def quantized_experts(self, E: int, Wgu: np.ndarray, Wdn: np.ndarray, experts) -> ExpertWeights:
+    def quantized_experts(self, E: int, Wgu: np.ndarray, Wdn: np.ndarray, experts, fmt=None) -> ExpertWeights:
         """Quantise dense float32 gate_up [n, H, 2I] and down [n, I, H] weights of the listed
-        expert ids (row a belongs to experts[a]) with this oracle's quantiser."""
+        expert ids (row a belongs to experts[a]) with this oracle's quantisers: E2M1, or INT2
+        for the experts e with fmt[e] = 1 (fmt: None or a length-E sequence)."""
         n, H, I2 = Wgu.shape
         I = I2 // 2
         experts = list(experts)
         assert len(experts) == n and Wdn.shape == (n, I, H)
         ew = ExpertWeights(E, H, I)
-        gc, gs = self.quantize(Wgu)
-        dc, ds = self.quantize(Wdn)
         for a, e in enumerate(experts):
-            ew.set(e, gc[a], gs[a], dc[a], ds[a])
+            f = int(fmt[e]) if fmt is not None else 0
+            q = self.quantize_int2 if f else self.quantize
+            gc, gs = q(Wgu[a:a + 1])
+            dc, ds = q(Wdn[a:a + 1])
+            ew.set(e, gc[0], gs[0], dc[0], ds[0], fmt=f)
         return ew
 
 

@@ -24,7 +24,8 @@
  *      group of k that holds k; two codes per byte, the low nibble holding
  *      the even k; all experts in one [E, K/2, N] code buffer and one
  *      [E, K/32, N] scale buffer (FireEcho's packed [E, K//2, N] expert
- *      buffer);
+ *      buffer); an expert may instead hold INT2 codes, W = (q - 1.5) * the
+ *      same group scale, four codes per byte (orc_moe_forward_fmt);
  *   4. gate_up: g[n] = sum_k x[k] W[k][n], u[n] = sum_k x[k] W[k][I+n]
  *      (gate columns first, then up columns, one fused matrix);
  *      act[n] = silu(g[n]) * u[n], silu(v) = v / (1 + exp(-v));
@@ -194,6 +195,64 @@ int orc_route(const float* logits, int T, int E, int k, int32_t* idx, float* w)
 }
 
 /* ---------------------------------------------------------------------- */
+/* INT2 scalar codes ("FireEcho Engine", sections "Quantization Formats":   */
+/* INT2, 2 bits, 8x, scalar, for the coldest experts; and "FE-XC / INT2 Cold */
+/* Expert Demotion": a scalar 2-bit format for rarely used experts).  The    */
+/* pages give no code table; the reading here is the symmetric four-level   */
+/* scalar quantiser: a 2-bit unsigned code q decodes to (q - 1.5) times the */
+/* bf16 scale of its 32-element group along K, s = bf16_rne(max|w| / 1.5),  */
+/* the code of r = w / s is the nearest level, a tie (r = -1, 0 or 1) going */
+/* to the level above.  Four codes per byte: the code of k = 4 r + i sits  */
+/* in bits 2i and 2i + 1 of byte row r; layout [E][K/4][N], scales          */
+/* [E][K/32][N] as for E2M1.                                                */
+/* ---------------------------------------------------------------------- */
+double orc_int2_decode(int q) { return (double)(q & 3) - 1.5; }
+
+int orc_int2_encode(float r)
+{
+    if (r < -1.0f) return 0;
+    if (r < 0.0f) return 1;
+    if (r < 1.0f) return 2;
+    return 3;
+}
+
+int orc_quantize_int2(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales)
+{
+    if (E < 0 || K <= 0 || N <= 0 || K % 32 || !W || !codes || !scales) return ORC_EINVAL;
+    memset(codes, 0, (size_t)(E * (K / 4) * N));
+    for (int64_t e = 0; e < E; ++e)
+        for (int64_t g = 0; g < K / 32; ++g)
+            for (int64_t n = 0; n < N; ++n) {
+                float mx = 0.0f;
+                for (int64_t kk = 0; kk < 32; ++kk) {
+                    const float a = fabsf(W[(e * K + g * 32 + kk) * N + n]);
+                    if (a > mx) mx = a;
+                }
+                const uint16_t sb = orc_f32_to_bf16_rne(mx / 1.5f);
+                scales[(e * (K / 32) + g) * N + n] = sb;
+                const float sv = orc_bf16_to_f32(sb);
+                for (int64_t kk = 0; kk < 32; ++kk) {
+                    const int64_t k = g * 32 + kk;
+                    const int q = sv != 0.0f ? orc_int2_encode(W[(e * K + k) * N + n] / sv) : 2;
+                    codes[(e * (K / 4) + k / 4) * N + n] |= (uint8_t)(q << (2 * (k % 4)));
+                }
+            }
+    return ORC_OK;
+}
+
+/* One dequantised INT2 weight of a single expert's [K/4][N] codes / [K/32][N] scales. */
+static float orc_weight_int2(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t k, int64_t n)
+{
+    const int q = (codes[(k / 4) * N + n] >> (2 * (k % 4))) & 3;
+    return (float)orc_int2_decode(q) * orc_bf16_to_f32(scales[(k / 32) * N + n]);
+}
+
+float orc_dequant_int2(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t k, int64_t n)
+{
+    return orc_weight_int2(codes, scales, N, k, n);
+}
+
+/* ---------------------------------------------------------------------- */
 /* Router GEMM ("FireEcho Engine", section "Architecture": MoEFFN, the packed */
 /* MoE whose dispatch starts from the router's scores; "Speed Optimization   */
 /* History" step 1, the router in front of the grouped dispatch):           */
@@ -253,10 +312,18 @@ int orc_group(const int32_t* idx, int T, int k, int E, int32_t* counts, int32_t*
 /*   (either may be NULL), act64 [T*k][I] in pair order p = t*k + j (NULL   */
 /*   to skip).                                                              */
 /* ---------------------------------------------------------------------- */
-int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, const float* logits,
-                    const uint8_t* const* gu_codes, const uint16_t* const* gu_scales,
-                    const uint8_t* const* dn_codes, const uint16_t* const* dn_scales, double* y64,
-                    uint16_t* y_bf16, double* act64)
+static float orc_weight_fmt(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t k, int64_t n)
+{
+    return fmt ? orc_weight_int2(codes, scales, N, k, n) : orc_weight(codes, scales, N, k, n);
+}
+
+/* The layer with a format per expert: fmt[e] = 0 E2M1 (codes [K/2][N]), 1 INT2 */
+/* (codes [K/4][N]); fmt NULL: every expert E2M1.  Otherwise as             */
+/* orc_moe_forward.                                                         */
+int orc_moe_forward_fmt(int E, int H, int I, int T, int k, const uint16_t* x_bf16, const float* logits,
+                        const uint8_t* fmt, const uint8_t* const* gu_codes, const uint16_t* const* gu_scales,
+                        const uint8_t* const* dn_codes, const uint16_t* const* dn_scales, double* y64,
+                        uint16_t* y_bf16, double* act64)
 {
     if (E <= 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || T < 0 || k < 1 || k > E) return ORC_EINVAL;
     if (T == 0) return ORC_OK;
@@ -279,11 +346,12 @@ int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, c
         for (int j = 0; j < k; ++j) {
             const int e = idx[j];
             if (!gu_codes[e] || !gu_scales[e] || !dn_codes[e] || !dn_scales[e]) { rc = ORC_EINVAL; goto done; }
+            const int f = fmt ? fmt[e] : 0;
             /* gate_up: K = H, N = 2I */
             for (int64_t n = 0; n < N1; ++n) gu[n] = 0.0;
             for (int64_t kk = 0; kk < H; ++kk)
                 for (int64_t n = 0; n < N1; ++n)
-                    gu[n] += x[kk] * (double)orc_weight(gu_codes[e], gu_scales[e], N1, kk, n);
+                    gu[n] += x[kk] * (double)orc_weight_fmt(f, gu_codes[e], gu_scales[e], N1, kk, n);
             for (int i = 0; i < I; ++i) {
                 double g = gu[i], u = gu[I + i];
                 act[i] = g / (1.0 + exp(-g)) * u;
@@ -293,7 +361,7 @@ int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, c
             for (int h = 0; h < H; ++h) o[h] = 0.0;
             for (int64_t kk = 0; kk < I; ++kk)
                 for (int64_t h = 0; h < H; ++h)
-                    o[h] += act[kk] * (double)orc_weight(dn_codes[e], dn_scales[e], H, kk, h);
+                    o[h] += act[kk] * (double)orc_weight_fmt(f, dn_codes[e], dn_scales[e], H, kk, h);
             /* weighted combine, slot order */
             for (int h = 0; h < H; ++h) y[h] += (double)w[j] * o[h];
         }
@@ -305,4 +373,13 @@ int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, c
 done:
     free(idx); free(w); free(x); free(gu); free(act); free(o); free(y);
     return rc;
+}
+
+int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, const float* logits,
+                    const uint8_t* const* gu_codes, const uint16_t* const* gu_scales,
+                    const uint8_t* const* dn_codes, const uint16_t* const* dn_scales, double* y64,
+                    uint16_t* y_bf16, double* act64)
+{
+    return orc_moe_forward_fmt(E, H, I, T, k, x_bf16, logits, NULL, gu_codes, gu_scales, dn_codes, dn_scales, y64,
+                               y_bf16, act64);
 }

@@ -17,7 +17,12 @@ oracle disagrees with:
 * a dense, unpermuted brute-force layer written here with numpy;
 * for the router GEMM: the closed form of all-equal weights (an exact sum by
   math.fsum), one-hot rows (a permutation of x's columns, exactly), numpy's
-  dot product, and a router whose expert ranking is built in.
+  dot product, and a router whose expert ranking is built in;
+* for the INT2 codec: the symmetry and spacing of the four levels, brute-force
+  nearest-level encoding with the stated tie rule, single-element layout probes
+  (two bits per code, four codes per byte, one scale max|w|/1.5 per 32 along
+  K), the rounding bound, and a dense brute-force layer whose experts mix
+  E2M1 and INT2.
 """
 from __future__ import annotations
 
@@ -389,6 +394,110 @@ def check_router_gemm_ranking(o, rng):
     assert idx[0].tolist() == [3, 6, 1, 4] and idx[1].tolist() == [3, 6, 1, 4], idx
 
 
+# -- INT2 -------------------------------------------------------------------------
+
+INT2_LEVELS = np.array([-1.5, -0.5, 0.5, 1.5])
+
+
+def int2_dequant_dense(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """INT2 codes [..., K/4, N] (code of k = 4r + i in bits 2i, 2i+1), scales [..., K/32, N]
+    -> float64 [..., K, N]."""
+    K4, N = codes.shape[-2:]
+    vals = np.empty(codes.shape[:-2] + (4 * K4, N), dtype=np.float64)
+    for i in range(4):
+        vals[..., i::4, :] = INT2_LEVELS[(codes >> (2 * i)) & 3]
+    return vals * np.repeat(bf16_to_f64(scales), 32, axis=-2)
+
+
+def check_int2_table(o):
+    """Four levels, equally spaced by 1, symmetric about 0, the largest 1.5."""
+    v = np.array([o.int2_decode(q) for q in range(4)])
+    assert np.array_equal(v, INT2_LEVELS), v
+    assert np.all(np.diff(v) == 1.0) and np.all(v == -v[::-1])
+
+
+def check_int2_encode_bruteforce(o, rng):
+    """Nearest level; an exact midpoint (-1, 0, 1) goes to the level above."""
+    probes = np.concatenate([rng.standard_normal(400) * 1.2, [-1.0, 0.0, 1.0, -2.0, 2.0, 1.5, -1.5, 7.0, -7.0],
+                             np.nextafter(np.float32([-1, 0, 1]), np.float32(-9)),
+                             np.nextafter(np.float32([-1, 0, 1]), np.float32(9))]).astype(np.float32)
+    levels = [Fraction(float(v)) for v in INT2_LEVELS]
+    for r in probes:
+        d = [abs(Fraction(float(r)) - lv) for lv in levels]   # exact distances
+        best = max(q for q in range(4) if d[q] == min(d))      # ties: the higher level
+        assert o.int2_encode(float(r)) == best, (float(r), o.int2_encode(float(r)), best)
+
+
+def check_int2_quantize_layout(o):
+    """One nonzero weight per group: its code lands in bits 2(k % 4) of byte row k // 4,
+    the group's scale is bf16(|w| / 1.5), and the other (zero) weights take code 2."""
+    E, K, N = 2, 64, 3
+    for (e, k, n, wv) in [(0, 0, 0, 0.75), (1, 5, 2, -0.3), (0, 38, 1, 1.0), (1, 63, 0, -2.5)]:
+        W = np.zeros((E, K, N), dtype=np.float32)
+        W[e, k, n] = wv
+        codes, scales = o.quantize_int2(W)
+        s = float(bf16_to_f64(scales[e, k // 32, n]))
+        assert scales[e, k // 32, n] == nearest_bf16_bits(np.float32(np.float32(abs(wv)) / np.float32(1.5)))
+        q = (int(codes[e, k // 4, n]) >> (2 * (k % 4))) & 3
+        assert q == (3 if wv > 0 else 0), (q, wv)
+        assert abs(INT2_LEVELS[q] * s - wv) <= 0.01 * abs(wv)
+        # every other weight of the group is 0: r = 0 takes the level 0.5 (code 2)
+        for kk in range(32 * (k // 32), 32 * (k // 32) + 32):
+            if kk != k:
+                assert (int(codes[e, kk // 4, n]) >> (2 * (kk % 4))) & 3 == 2
+        # other columns and groups: all-zero groups (scale 0)
+        assert scales[e, (k // 32) ^ 1, n] == 0 and scales[1 - e].max() == 0
+
+
+def check_int2_roundtrip(o, rng):
+    """|w - dequant(w)| <= s/2 (+ the bf16 rounding of s), with s = bf16(max|w| / 1.5)."""
+    W = (rng.standard_normal((2, 128, 24)) * 0.02).astype(np.float32)
+    codes, scales = o.quantize_int2(W)
+    deq = int2_dequant_dense(codes, scales)
+    s = np.repeat(bf16_to_f64(scales), 32, axis=-2)
+    assert np.all(np.abs(W - deq) <= 0.5 * s * (1 + 2.0 ** -7) + 1e-30)
+    for (e, k, n) in [(0, 3, 5), (1, 100, 0), (1, 31, 23)]:
+        assert o.dequant_int2(codes[e], scales[e], k, n) == np.float32(deq[e, k, n])
+
+
+def check_mixed_dense_bruteforce(o, rng):
+    """A layer whose experts mix E2M1 and INT2, against an unpermuted dense brute force."""
+    import oracle as _oracle_pkg
+    E, H, I, T, k = 6, 64, 32, 3, 3
+    fmt = [1, 0, 1, 1, 0, 1]
+    gu_c, gu_s, dn_c, dn_s = _layer_inputs(rng, E, H, I, T, random_codes=True)
+    gu_c2 = rng.integers(0, 256, (E, H // 4, 2 * I), dtype=np.uint8)
+    dn_c2 = rng.integers(0, 256, (E, I // 4, H), dtype=np.uint8)
+    ew = _oracle_pkg.ExpertWeights(E, H, I)
+    Wgu = np.empty((E, H, 2 * I))
+    Wdn = np.empty((E, I, H))
+    for e in range(E):
+        if fmt[e]:
+            ew.set(e, gu_c2[e], gu_s[e], dn_c2[e], dn_s[e], fmt=1)
+            Wgu[e] = int2_dequant_dense(gu_c2[e], gu_s[e])
+            Wdn[e] = int2_dequant_dense(dn_c2[e], dn_s[e])
+        else:
+            ew.set(e, gu_c[e], gu_s[e], dn_c[e], dn_s[e])
+            Wgu[e] = dequant_dense(gu_c[e], gu_s[e])
+            Wdn[e] = dequant_dense(dn_c[e], dn_s[e])
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    x_bf16 = (x.view(np.uint32) >> 16).astype(np.uint16)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    y64, _ = o.moe_forward(ew, x_bf16, logits, k)
+    xs = bf16_to_f64(x_bf16)
+    ref = np.zeros((T, H))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))
+        sel = order[:k]
+        ls = logits[t, sel].astype(np.float64)
+        wsel = (np.exp(ls - ls[0]) / np.exp(ls - ls[0]).sum()).astype(np.float32).astype(np.float64)
+        for j, e in enumerate(sel):
+            h = xs[t] @ Wgu[e]
+            a = h[:I] / (1.0 + np.exp(-h[:I])) * h[I:]
+            ref[t] += wsel[j] * (a @ Wdn[e])
+    assert np.abs(y64 - ref).max() <= 1e-10 * np.abs(ref).max()
+
+
 ALL_CHECKS = [
     ("e2m1_table", lambda o, rng: check_e2m1_table(o)),
     ("encode_bruteforce", check_encode_bruteforce),
@@ -404,4 +513,9 @@ ALL_CHECKS = [
     ("router_gemm_onehot", check_router_gemm_onehot),
     ("router_gemm_numpy", check_router_gemm_numpy),
     ("router_gemm_ranking", check_router_gemm_ranking),
+    ("int2_table", lambda o, rng: check_int2_table(o)),
+    ("int2_encode_bruteforce", check_int2_encode_bruteforce),
+    ("int2_quantize_layout", lambda o, rng: check_int2_quantize_layout(o)),
+    ("int2_roundtrip", check_int2_roundtrip),
+    ("mixed_dense_bruteforce", check_mixed_dense_bruteforce),
 ]

@@ -35,6 +35,14 @@ MUTANTS = [
      "for (int h = 0; h < H - 1; ++h)\n                acc +="),
     ("router_gemm_first_token_only", "acc += (double)orc_bf16_to_f32(x_bf16[(int64_t)t * H + h]) *",
      "acc += (double)orc_bf16_to_f32(x_bf16[h]) *"),
+    ("int2_level_offset", "double orc_int2_decode(int q) { return (double)(q & 3) - 1.5; }",
+     "double orc_int2_decode(int q) { return (double)(q & 3) - 1.0; }"),
+    ("int2_tie_rule", "    if (r < 0.0f) return 1;\n    if (r < 1.0f) return 2;",
+     "    if (r <= 0.0f) return 1;\n    if (r < 1.0f) return 2;"),
+    ("int2_bit_order", "codes[(e * (K / 4) + k / 4) * N + n] |= (uint8_t)(q << (2 * (k % 4)));",
+     "codes[(e * (K / 4) + k / 4) * N + n] |= (uint8_t)(q << (6 - 2 * (k % 4)));"),
+    ("int2_scale_divisor", "orc_f32_to_bf16_rne(mx / 1.5f)", "orc_f32_to_bf16_rne(mx / 2.0f)"),
+    ("mixed_ignores_format", "const int f = fmt ? fmt[e] : 0;", "const int f = 0;"),
     ("down_scale_group", "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[(k / 32) * N + n]);",
      "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[((k / 32) / 2) * N + n]);"),
 ]
