@@ -572,6 +572,94 @@ def run_router(device):
     return out
 
 
+def int2_bytes_per_expert(H, I):
+    """INT2 codes (2 bits) + bf16 group scales of one expert's gate_up and down matrices."""
+    return (H // 4) * 2 * I + (H // 32) * 2 * I * 2 + (I // 4) * H + (I // 32) * H * 2
+
+
+def run_int2(device, n_layers=16, steps=20):
+    """The decode layer (E 128, H 2048, I 768, top-8, T = 1) with every odd expert held as
+    INT2 codes (fe_moe_load_int2), 16 layers with their own seeded weights, x and logits
+    (more bytes per step than L2 holds), one launch per layer in a CUDA graph; against the
+    same 16 layers with every expert E2M1."""
+    import torch
+
+    import fp4_expert_gemv_b200 as fe
+    import synth
+    cfg = synth.WORKLOADS[HEADLINE]
+    E, H, I, k, T = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"], cfg["T"]
+    fmt = np.array([e % 2 for e in range(E)], dtype=np.uint8)
+    handles = build_stack(cfg, n_layers, device)
+    x, lg = stack_inputs(cfg, n_layers)
+    st = torch.cuda.current_stream().cuda_stream
+    peaks, src = measured_peaks()
+
+    def timed():
+        xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+        ld = torch.from_numpy(lg).to(device)
+        yd = torch.empty_like(xd)
+        s = torch.cuda.Stream()
+
+        def calls():
+            for l, m in enumerate(handles):
+                fe.check(fe.fe_moe_forward(m.h, xd[l].data_ptr(), ld[l].data_ptr(), T, k, yd[l].data_ptr(),
+                                           s.cuda_stream), "fe_moe_forward")
+
+        with torch.cuda.stream(s):
+            calls()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            calls()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(steps):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / (steps * n_layers)
+
+    us_fp4 = timed()
+    Wgu = torch.empty((E, H, 2 * I), dtype=torch.float32, device=device)
+    Wdn = torch.empty((E, I, H), dtype=torch.float32, device=device)
+    for l, m in enumerate(handles):
+        seed = synth.STACK_SEED0 + l
+        synth.device_gate_up(Wgu.data_ptr(), seed, E, H, I, st)
+        gc, gs = fe.pack_int2_device(Wgu)
+        synth.device_down(Wdn.data_ptr(), seed, E, I, H, st)
+        dc, ds = fe.pack_int2_device(Wdn)
+        m.load_int2(fmt, gc, gs, dc, ds)
+        del gc, gs, dc, ds
+    del Wgu, Wdn
+    us_mixed = timed()
+    # algorithmic bytes: each layer's distinct routed experts in their own format, x, logits, y
+    nbytes = 0.0
+    for l in range(n_layers):
+        order = np.lexsort((np.arange(E), -lg[l, 0].astype(np.float64)))
+        for e in order[:k]:
+            nbytes += int2_bytes_per_expert(H, I) if fmt[e] else bytes_per_expert(H, I)
+        nbytes += T * H * 2 + T * E * 4 + T * H * 2
+    per_layer = nbytes / n_layers
+    gbs = per_layer / (us_mixed * 1e-6) / 1e9
+    st_bits = [m.status()[1] for m in handles]
+    for m in handles:
+        m.close()
+    torch.cuda.empty_cache()
+    return {"workload": "decode_e128_t1, every odd expert INT2", "layers": n_layers, "T": T, "top_k": k,
+            "us_per_layer": us_mixed, "tokens_per_s": T / (us_mixed * 1e-6),
+            "algorithmic_bytes_per_layer_mean": per_layer,
+            "roofline": {"bound": "hbm", "achieved": gbs, "unit": "GB/s", "peak": float(peaks["hbm_gbs"]),
+                         "frac": gbs / float(peaks["hbm_gbs"]), "peak_source": src},
+            "all_e2m1_us_per_layer": us_fp4,
+            "path": "single-launch decode kernel, one launch per layer (the persistent kernel reads E2M1 only)",
+            "status_bits": int(max(st_bits))}
+
+
 def run_gpu(args):
     import torch
 
@@ -619,6 +707,7 @@ def run_gpu(args):
         line["workloads"] = extra
     if args.workload == "all":
         line["router_gemm"] = run_router(device)
+        line["int2_mixed"] = run_int2(device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
         reps = args.cpu_reps

@@ -71,6 +71,9 @@ _SIGS = {
     "fe_moe_stack_last_launches": (_i32, [_P]),
     "fe_moe_set_exchange_test": (_st, [_P, _i32, ctypes.c_uint64]),
     "fe_moe_router": (_st, [_P, _P, _P, _i32, _i32, _P, _P, _P, _P]),
+    "fe_moe_load_int2": (_st, [_P, _P, _P, _P, _P, _P, _i32, _P]),
+    "fe_moe_pack_int2_host": (_st, [_P, _i64, _i64, _i64, _P, _P]),
+    "fe_moe_pack_int2_device": (_st, [_P, _i64, _i64, _i64, _P, _P, _P]),
     "fe_moe_forward_router": (_st, [_P, _P, _P, _i32, _i32, _P, _P, _P]),
 }
 
@@ -153,6 +156,20 @@ class MoELayer:
         check(fe_moe_forward(self.h, _dptr(x_bf16), _dptr(logits), T, top_k, _dptr(y_bf16), _stream_ptr(stream)),
               "fe_moe_forward")
         return y_bf16
+
+    def load_int2(self, formats, gu_codes, gu_scales, dn_codes, dn_scales, stream=None):
+        """INT2 weights for the experts e with formats[e] = 1 (host numpy arrays or device
+        torch tensors, full size [E, ...]); synchronous."""
+        import numpy as np
+        fmt = np.ascontiguousarray(np.asarray(formats, dtype=np.uint8))
+        assert fmt.shape == (self.E,)
+        if isinstance(gu_codes, np.ndarray):
+            arrs = [np.ascontiguousarray(a) for a in (gu_codes, gu_scales, dn_codes, dn_scales)]
+            check(fe_moe_load_int2(self.h, fmt.ctypes.data, *[a.ctypes.data for a in arrs], 0, _stream_ptr(stream)),
+                  "fe_moe_load_int2")
+        else:
+            check(fe_moe_load_int2(self.h, fmt.ctypes.data, _dptr(gu_codes), _dptr(gu_scales), _dptr(dn_codes),
+                                   _dptr(dn_scales), 1, _stream_ptr(stream)), "fe_moe_load_int2")
 
     def router(self, x_bf16, w_router_bf16, top_k: int, logits=None, idx=None, w=None, stream=None):
         """The router GEMM fused with the top-k: (logits [T, E] f32, idx [T, k] i32, w [T, k] f32)."""
@@ -302,6 +319,31 @@ def pack_host(W):
     codes = np.empty((E, K // 2, N), dtype=np.uint8)
     scales = np.empty((E, K // 32, N), dtype=np.uint16)
     check(fe_moe_pack_host(W.ctypes.data, E, K, N, codes.ctypes.data, scales.ctypes.data), "fe_moe_pack_host")
+    return codes, scales
+
+
+def pack_int2_host(W):
+    """numpy float32 [E, K, N] -> (INT2 codes uint8 [E, K/4, N], scales uint16 [E, K/32, N])."""
+    import numpy as np
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    E, K, N = W.shape
+    codes = np.empty((E, K // 4, N), dtype=np.uint8)
+    scales = np.empty((E, K // 32, N), dtype=np.uint16)
+    check(fe_moe_pack_int2_host(W.ctypes.data, E, K, N, codes.ctypes.data, scales.ctypes.data),
+          "fe_moe_pack_int2_host")
+    return codes, scales
+
+
+def pack_int2_device(W, codes=None, scales=None, stream=None):
+    """torch float32 CUDA [E, K, N] -> (INT2 codes uint8 [E, K/4, N], scales int16 bf16-bits)."""
+    import torch
+    E, K, N = W.shape
+    if codes is None:
+        codes = torch.empty((E, K // 4, N), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty((E, K // 32, N), dtype=torch.int16, device=W.device)
+    check(fe_moe_pack_int2_device(_dptr(W), E, K, N, _dptr(codes), _dptr(scales), _stream_ptr(stream)),
+          "fe_moe_pack_int2_device")
     return codes, scales
 
 

@@ -73,6 +73,9 @@ struct DecodeParams {
     int T, E, H, I, k;
     const uint8_t* gu_blocks; // [E][I/16] gate_up units of 2 blocks (18H bytes)
     const uint8_t* dn_rows;   // [E][I/32] row groups of W_dn (18H bytes, pack.cuh)
+    const uint8_t* fmt;       // [E]: 1 = the expert's weights are INT2 codes (below); null: all E2M1
+    const uint8_t* gu2_blocks;  // INT2 experts: [E][I/16] gate_up units of 2 INT2 blocks (10H bytes)
+    const uint8_t* dn2_rows;    // INT2 experts: [E][I/32] INT2 row groups of W_dn (10H bytes)
     int32_t* idx;
     float* w;
     int32_t* counts;
@@ -111,6 +114,7 @@ struct DecodeShared {
     uint32_t u_codes[kDecMaxUnits];           // shared-memory offsets of a unit's down codes
     uint32_t u_scales[kDecMaxUnits];          // ... and of its row group's scales
     int u_dnbar[kDecMaxUnits];                // barrier of its down copy
+    int u_fmt[kDecMaxUnits];                  // 1: the unit's expert is INT2
     uint32_t dn_bytes[kDecMaxUnits];          // bytes of the down copy a unit issued (0: shares one)
     int bshift[kDecMaxT];                     // current unit: power-of-two shift of each token's B column
     uint32_t bfrag[kDecMaxT][8];              // current unit's down B operand: token t, 16 values as f16x2
@@ -303,8 +307,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         const bool mine = lane < nu;
         const bool first = mine && (j & 1) == 0 && lane + 1 < nu && d_next == d;
         const bool second = mine && (j & 1) == 1 && lane > 0 && d_prev == d;
-        const uint32_t H8 = 8u * H, H10 = 10u * H;
-        const uint32_t dn_bytes = !mine || second ? 0u : first ? 18u * H : H10;
+        // an INT2 expert (fmt) has half the code bytes: 4H per 16 rows of W_dn, 5H per
+        // gate_up block; its row groups and units come from the INT2 buffers
+        const bool i2 = mine && p.fmt != nullptr && p.fmt[S.dex[d]] != 0;
+        const uint32_t CH = i2 ? 4u * H : 8u * H, SH = 2u * H;   // codes of 16 rows; scales of 32
+        const uint32_t dn_bytes = !mine || second ? 0u : first ? 2u * CH + SH : CH + SH;
+        const uint32_t gu_bytes = i2 ? 2u * int2_block_bytes(H) : gu_unit;
         uint32_t incl = dn_bytes;   // inclusive scan of the down bytes over the lanes
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -313,31 +321,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
         }
         const uint32_t off = (uint32_t)nu * gu_unit + incl - dn_bytes;
         const uint32_t off_prev = __shfl_up_sync(0xffffffffu, off, 1);   // a pair's first unit
-        const long long grp = mine ? ((long long)S.dex[d] * (I / 32) + j / 2) * 18ll * H : 0ll;
+        const long long grp = mine ? ((long long)S.dex[d] * (I / 32) + j / 2) * (long long)(2u * CH + SH) : 0ll;
         if (mine) {
             uint32_t codes, scales;
             if (second) {
-                codes = off_prev + H10;
-                scales = off_prev + H8;
+                codes = off_prev + CH + SH;
+                scales = off_prev + CH;
             } else if ((j & 1) == 0) {
                 codes = off;
-                scales = off + H8;
+                scales = off + CH;
             } else {
-                codes = off + 2u * H;
+                codes = off + SH;
                 scales = off;
             }
             S.u_codes[lane] = codes;
             S.u_scales[lane] = scales;
             S.u_dnbar[lane] = second ? lane - 1 : lane;
+            S.u_fmt[lane] = i2 ? 1 : 0;
             S.dn_bytes[lane] = dn_bytes;
-            mbar_expect_tx(bar_gu(lane), gu_unit);
+            mbar_expect_tx(bar_gu(lane), gu_bytes);
             if (dn_bytes) mbar_expect_tx(bar_dn(lane), dn_bytes);
         }
         if (tracing && lane == 0) stamp(trace, 15);
         if (mine) {
             const uint32_t wb = smem_addr(wbuf);
-            bulk_g2s(wb + lane * gu_unit, p.gu_blocks + ((size_t)S.dex[d] * upe + j) * gu_unit, gu_unit, bar_gu(lane));
-            if (dn_bytes) bulk_g2s(wb + off, p.dn_rows + grp + ((j & 1) && !first ? H8 : 0u), dn_bytes, bar_dn(lane));
+            const uint8_t* gsrc = i2 ? p.gu2_blocks : p.gu_blocks;
+            const uint8_t* dsrc = i2 ? p.dn2_rows : p.dn_rows;
+            bulk_g2s(wb + lane * gu_unit, gsrc + ((size_t)S.dex[d] * upe + j) * gu_bytes, gu_bytes, bar_gu(lane));
+            if (dn_bytes) bulk_g2s(wb + off, dsrc + grp + ((j & 1) && !first ? CH : 0u), dn_bytes, bar_dn(lane));
         }
         if (tracing && lane == 0) stamp(trace, 1);
     } else if (warp == 0) {
@@ -429,19 +440,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             S.abort = 1;
         }
         if (tracing && tid == 0 && (i == 0 || i == nu - 1)) stamp(trace, i == 0 ? 11 : 13);
+        const bool ui2 = S.u_fmt[i] != 0;   // the same in every thread
         const uint8_t* blk0 = wbuf + i * gu_unit;
-        const uint8_t* blk1 = blk0 + block_bytes(H);
+        const uint8_t* blk1 = blk0 + (ui2 ? int2_block_bytes(H) : block_bytes(H));
         const int r0 = S.dstart[d], nvalid = S.dstart[d + 1] - r0;   // the expert's tokens (<= T <= 8)
         const uint32_t* brow = xs + (g < nvalid ? S.sp[r0 + g] / k : T) * xrw;
         float t0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         // warp w takes the 64-k quads w, w + W, ...: one compact loop (the code of a
         // launch is fetched cold, so a short loop body beats unrolled copies), the
         // quad's x fragments read from shared memory with two 16-byte loads
+        if (ui2) {
 #pragma unroll 1
-        for (int q = warp; q < nq; q += kDecWarps) {
-            uint32_t b[8];
-            load_bfrag(brow, q, lane, b);
-            quad_mma2_b(blk0, blk1, H, b, q, lane, t0, t1);
+            for (int q = warp; q < nq; q += kDecWarps) {
+                uint32_t b[8];
+                load_bfrag(brow, q, lane, b);
+                quad_mma2_b_int2(blk0, blk1, H, b, q, lane, t0, t1);
+            }
+        } else {
+#pragma unroll 1
+            for (int q = warp; q < nq; q += kDecWarps) {
+                uint32_t b[8];
+                load_bfrag(brow, q, lane, b);
+                quad_mma2_b(blk0, blk1, H, b, q, lane, t0, t1);
+            }
         }
         if (tracing && tid == 0 && i == nu - 1) stamp(trace, 17);
         // partials of the valid token columns: [warp][column][gate 16 | up 16];
@@ -504,24 +525,54 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             const float m0 = pow2f(S.bshift[2 * c4]), m1 = pow2f(S.bshift[2 * c4 + 1]);
             const uint8_t* codes = wbuf + S.u_codes[i];
             const uint8_t* scl = wbuf + S.u_scales[i];
+            // an INT2 register holds twice the level: the scale is halved
+            if (ui2) {
 #pragma unroll
-            for (int qs = 0; qs < HQ; ++qs) {
-                const int q = warp + kDecWarps * qs;
-                if (q < nq) {
-                    const uint4 cw = *reinterpret_cast<const uint4*>(codes + 512 * q + 16 * lane);
-                    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                for (int qs = 0; qs < HQ; ++qs) {
+                    const int q = warp + kDecWarps * qs;
+                    if (q < nq) {
+                        const uint2 cw = *reinterpret_cast<const uint2*>(codes + 256 * q + 8 * lane);
 #pragma unroll
-                    for (int s4 = 0; s4 < 4; ++s4) {
-                        uint32_t a[4];
-                        e2m1x8_to_f16x2x4(words[s4], a);
-                        float dd[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                        mma16816(dd, a, b0, b1);
-                        const uint32_t sw = *reinterpret_cast<const uint32_t*>(scl + 32 * (4 * q + s4) + 4 * g);
-                        const float slo = __uint_as_float(sw << 16), shi = __uint_as_float(sw & 0xffff0000u);
-                        Y[qs][s4][0] = fmaf(dd[0], slo * m0, Y[qs][s4][0]);
-                        Y[qs][s4][1] = fmaf(dd[1], slo * m1, Y[qs][s4][1]);
-                        Y[qs][s4][2] = fmaf(dd[2], shi * m0, Y[qs][s4][2]);
-                        Y[qs][s4][3] = fmaf(dd[3], shi * m1, Y[qs][s4][3]);
+                        for (int h2 = 0; h2 < 2; ++h2) {   // word h2: column tiles 2 h2, 2 h2 + 1
+                            uint32_t ar[8];
+                            int2x8_to_f16x2x8(h2 ? cw.y : cw.x, ar);
+#pragma unroll
+                            for (int sl = 0; sl < 2; ++sl) {
+                                const int s4 = 2 * h2 + sl;
+                                const uint32_t a[4] = {ar[4 * sl], ar[4 * sl + 1], ar[4 * sl + 2], ar[4 * sl + 3]};
+                                float dd[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                                mma16816(dd, a, b0, b1);
+                                const uint32_t sw = *reinterpret_cast<const uint32_t*>(scl + 32 * (4 * q + s4) + 4 * g);
+                                const float slo = __uint_as_float(sw << 16) * 0.5f;
+                                const float shi = __uint_as_float(sw & 0xffff0000u) * 0.5f;
+                                Y[qs][s4][0] = fmaf(dd[0], slo * m0, Y[qs][s4][0]);
+                                Y[qs][s4][1] = fmaf(dd[1], slo * m1, Y[qs][s4][1]);
+                                Y[qs][s4][2] = fmaf(dd[2], shi * m0, Y[qs][s4][2]);
+                                Y[qs][s4][3] = fmaf(dd[3], shi * m1, Y[qs][s4][3]);
+                            }
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int qs = 0; qs < HQ; ++qs) {
+                    const int q = warp + kDecWarps * qs;
+                    if (q < nq) {
+                        const uint4 cw = *reinterpret_cast<const uint4*>(codes + 512 * q + 16 * lane);
+                        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4) {
+                            uint32_t a[4];
+                            e2m1x8_to_f16x2x4(words[s4], a);
+                            float dd[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                            mma16816(dd, a, b0, b1);
+                            const uint32_t sw = *reinterpret_cast<const uint32_t*>(scl + 32 * (4 * q + s4) + 4 * g);
+                            const float slo = __uint_as_float(sw << 16), shi = __uint_as_float(sw & 0xffff0000u);
+                            Y[qs][s4][0] = fmaf(dd[0], slo * m0, Y[qs][s4][0]);
+                            Y[qs][s4][1] = fmaf(dd[1], slo * m1, Y[qs][s4][1]);
+                            Y[qs][s4][2] = fmaf(dd[2], shi * m0, Y[qs][s4][2]);
+                            Y[qs][s4][3] = fmaf(dd[3], shi * m1, Y[qs][s4][3]);
+                        }
                     }
                 }
             }

@@ -26,6 +26,7 @@
 
 namespace fe_host {
 void pack(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales);
+void pack_int2(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales);
 }
 
 struct fe_moe_s {
@@ -40,6 +41,11 @@ struct fe_moe_s {
     uint8_t* dn_blocks = nullptr;   // [E][H/16] x 9I bytes
     uint8_t* dn_rows = nullptr;     // [E][I/32] x 18H bytes: W_dn in row groups (single-launch decode)
     bool loaded = false;
+    // experts held as INT2 codes (fe_moe_load_int2): only the single-launch decode path reads them
+    bool has_int2 = false;
+    uint8_t* fmt = nullptr;         // [E]: 1 = INT2
+    uint8_t* gu2_blocks = nullptr;  // [E][I/16] x 10H bytes: INT2 gate_up units
+    uint8_t* dn2_rows = nullptr;    // [E][I/32] x 10H bytes: INT2 row groups of W_dn
     // workspace
     int max_T = 0, max_k = 0;
     int32_t* idx = nullptr;
@@ -222,6 +228,8 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
     dp.y = static_cast<uint16_t*>(y);
     dp.T = T; dp.E = h->E; dp.H = h->H; dp.I = h->I; dp.k = k;
     dp.gu_blocks = h->gu_blocks; dp.dn_rows = h->dn_rows;
+    dp.fmt = h->has_int2 ? h->fmt : nullptr;
+    dp.gu2_blocks = h->gu2_blocks; dp.dn2_rows = h->dn2_rows;
     dp.idx = h->idx; dp.w = h->w; dp.counts = h->counts; dp.offsets = h->offsets;
     dp.sorted_pair = h->sorted_pair; dp.pair_row = h->pair_row;
     dp.part = h->dec_part;
@@ -716,6 +724,63 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
     return FE_OK;
 }
 
+fe_status fe_moe_load_int2(fe_moe_t h, const uint8_t* formats, const uint8_t* gu_codes, const uint16_t* gu_scales,
+                           const uint8_t* dn_codes, const uint16_t* dn_scales, int src_on_device, fe_stream_t stream)
+{
+    if (!h || !formats || !gu_codes || !gu_scales || !dn_codes || !dn_scales) return FE_ERR_INVALID_ARG;
+    if (h->H % 64 != 0 || h->I % 64 != 0) return FE_ERR_UNSUPPORTED;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t E = h->E, H = h->H, I = h->I;
+    const size_t gu_c = (size_t)E * (H / 4) * (2 * I), gu_s = (size_t)E * (H / 32) * (2 * I);
+    const size_t dn_c = (size_t)E * (I / 4) * H, dn_s = (size_t)E * (I / 32) * H;
+    if (!h->gu2_blocks) {
+        cudaError_t e = cudaSuccess;
+        size_t acc = 0;
+        if (e == cudaSuccess) e = dmalloc(&h->fmt, (size_t)E, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->gu2_blocks, (size_t)E * (I / 16) * 2 * fe::int2_block_bytes((int)H), &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->dn2_rows, (size_t)E * (I / 32) * 10 * (size_t)H, &acc);
+        if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? FE_ERR_OOM : FE_ERR_CUDA;
+        h->weight_bytes += acc;
+    }
+    const uint8_t* sgc = gu_codes;
+    const uint16_t* sgs = gu_scales;
+    const uint8_t* sdc = dn_codes;
+    const uint16_t* sds = dn_scales;
+    void* staging = nullptr;
+    if (!src_on_device) {
+        const size_t bytes = gu_c + 2 * gu_s + dn_c + 2 * dn_s;
+        FE_CUDA_TRY(cudaMallocAsync(&staging, bytes, s));
+        uint8_t* b = static_cast<uint8_t*>(staging);
+        FE_CUDA_TRY(cudaMemcpyAsync(b, gu_codes, gu_c, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c, gu_scales, 2 * gu_s, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c + 2 * gu_s, dn_codes, dn_c, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c + 2 * gu_s + dn_c, dn_scales, 2 * dn_s, cudaMemcpyHostToDevice, s));
+        sgc = b;
+        sgs = reinterpret_cast<const uint16_t*>(b + gu_c);
+        sdc = b + gu_c + 2 * gu_s;
+        sds = reinterpret_cast<const uint16_t*>(b + gu_c + 2 * gu_s + dn_c);
+    }
+    bool any = false;
+    for (int64_t e = 0; e < E; ++e) any |= formats[e] != 0;
+    FE_CUDA_TRY(cudaMemcpyAsync(h->fmt, formats, (size_t)E, cudaMemcpyHostToDevice, s));
+    fe::RelayoutParams rp{};
+    rp.src_codes = sgc; rp.src_scales = sgs; rp.dst = h->gu2_blocks;
+    rp.E = E; rp.K = H; rp.N = 2 * I; rp.gate_up = 1;
+    fe::relayout_int2_kernel<<<1184, 256, 0, s>>>(rp);
+    fe::RowRelayoutParams rr{};
+    rr.src_codes = sdc; rr.src_scales = sds; rr.dst = h->dn2_rows;
+    rr.E = E; rr.I = I; rr.H = H;
+    fe::relayout_int2_rows_kernel<<<1184, 256, 0, s>>>(rr);
+    FE_CUDA_TRY(cudaGetLastError());
+    if (staging) FE_CUDA_TRY(cudaFreeAsync(staging, s));
+    // the host's format table and buffers are read by the copies: wait before returning
+    FE_CUDA_TRY(cudaStreamSynchronize(s));
+    h->has_int2 = any;
+    return FE_OK;
+}
+
 }  // extern "C"
 
 namespace {
@@ -753,6 +818,8 @@ fe_status forward_impl(fe_moe_t h, const void* x_bf16, const float* router_logit
         }
         if (h->path == FE_PATH_FUSED_DECODE) return FE_ERR_UNSUPPORTED;
     }
+    // INT2 experts are read by the single-launch decode kernel only
+    if (h->has_int2) return FE_ERR_UNSUPPORTED;
 
     const bool use_tc = tc_ok && (h->path == FE_PATH_TCGEN05 || (h->path == FE_PATH_AUTO && P >= kTcAutoPairs));
     SgSetup sg;
@@ -957,6 +1024,7 @@ int stack_persistent_mode(fe_moe_stack_s* st, const void* x, void* y, int T, int
     for (int l = 0; l < n; ++l) {
         fe_moe_s* h = st->layers[l];
         if (h->path != FE_PATH_AUTO && h->path != FE_PATH_FUSED_DECODE) return 0;
+        if (h->has_int2) return 0;   // the persistent kernel reads E2M1 experts only
         if (decode_weight_bytes(h, 1, top_k) == 0) return 0;
         const fe::StackLayer& s = st->h_layers[l];
         if (s.gu_blocks != h->gu_blocks || s.dn_rows != h->dn_rows || s.idx != h->idx || s.w != h->w ||
@@ -1182,7 +1250,7 @@ void fe_moe_destroy(fe_moe_t h)
         DeviceGuard g(h->device);
         cudaDeviceSynchronize();
         free_workspace(h);
-        void* ptrs[] = {h->gu_blocks, h->dn_blocks, h->dn_rows};
+        void* ptrs[] = {h->gu_blocks, h->dn_blocks, h->dn_rows, h->fmt, h->gu2_blocks, h->dn2_rows};
         for (void* p : ptrs)
             if (p) cudaFree(p);
     }
@@ -1198,6 +1266,24 @@ fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint
     if (!W || !codes || !scales || E < 1 || K < 32 || N < 1 || K % 32) return FE_ERR_INVALID_ARG;
     fe_host::pack(W, E, K, N, codes, scales);
     return FE_OK;
+}
+
+fe_status fe_moe_pack_int2_host(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes,
+                                uint16_t* scales)
+{
+    if (!W || !codes || !scales || E < 1 || K < 32 || N < 1 || K % 32) return FE_ERR_INVALID_ARG;
+    fe_host::pack_int2(W, E, K, N, codes, scales);
+    return FE_OK;
+}
+
+fe_status fe_moe_pack_int2_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,
+                                  fe_stream_t stream)
+{
+    if (!W || !codes || !scales || E < 1 || K < 32 || N < 1 || K % 32) return FE_ERR_INVALID_ARG;
+    const int64_t total = E * (K / 32) * N;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, 148 * 32);
+    fe::pack_int2_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(W, E, K, N, codes, scales);
+    return cudaGetLastError() == cudaSuccess ? FE_OK : FE_ERR_CUDA;
 }
 
 fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,

@@ -101,6 +101,69 @@ FE_DEV void quad_mma2(const uint8_t* blk0, const uint8_t* blk1, int K, const uin
     }
 }
 
+// ---- INT2 codes ----------------------------------------------------------------------
+// An INT2 block (16 columns x K, see pack.cuh) keeps the E2M1 block's fragment
+// order with two bits per code: per quad (64 k) 256 bytes, lane L's 8 at 8L;
+// word w of them holds the A registers of k-steps 2w and 2w + 1, register
+// r = 4 (s & 1) + j in bits 2r, 2r + 1 (the even k's code) and 16 + 2r,
+// 17 + 2r (the odd k's code); then the K/32 x 8 scale words as in an E2M1
+// block: 5K bytes.  A code q stands for the level q - 1.5.
+__host__ __device__ inline uint32_t int2_block_bytes(int K) { return 5u * (uint32_t)K; }
+
+// The 8 A registers of one INT2 word, register r = f16x2 (2 q_even - 3,
+// 2 q_odd - 3): the codes go into the mantissa of 1024 (0x6400), giving
+// 1024 + 2q, and 1027 is subtracted; all exact.  Twice the level, so the
+// group scale is halved to match.
+FE_DEV void int2x8_to_f16x2x8(uint32_t w, uint32_t (&a)[8])
+{
+    const __half2 off = __half2half2(__ushort_as_half((unsigned short)0x6403u));   // 1027
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const uint32_t bits = (r == 0 ? (w << 1) : (w >> (2 * r - 1))) & 0x00060006u;
+        const uint32_t v = bits | 0x64006400u;
+        const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&v), off);
+        a[r] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+
+// quad_mma2_b for two INT2 blocks.
+FE_DEV void quad_mma2_b_int2(const uint8_t* blk0, const uint8_t* blk1, int K, const uint32_t (&b)[8], int q,
+                             int lane, float (&tot0)[4], float (&tot1)[4])
+{
+    const int g = lane >> 2;
+    const uint2 c0 = *reinterpret_cast<const uint2*>(blk0 + 256 * q + 8 * lane);
+    const uint2 c1 = *reinterpret_cast<const uint2*>(blk1 + 256 * q + 8 * lane);
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {   // scale group gi: k-steps 2gi, 2gi + 1 = word gi
+        uint32_t a0[8], a1[8];
+        int2x8_to_f16x2x8(gi ? c0.y : c0.x, a0);
+        int2x8_to_f16x2x8(gi ? c1.y : c1.x, a1);
+        float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ss = 0; ss < 2; ++ss) {
+            const int s = 2 * gi + ss;
+            const uint32_t x0[4] = {a0[4 * ss], a0[4 * ss + 1], a0[4 * ss + 2], a0[4 * ss + 3]};
+            const uint32_t x1[4] = {a1[4 * ss], a1[4 * ss + 1], a1[4 * ss + 2], a1[4 * ss + 3]};
+            mma16816(d0, x0, b[2 * s], b[2 * s + 1]);
+            mma16816(d1, x1, b[2 * s], b[2 * s + 1]);
+        }
+        const int wo = 4 * ((2 * q + gi) * 8 + g);
+        const uint32_t s0 = *reinterpret_cast<const uint32_t*>(blk0 + 4 * K + wo);
+        const uint32_t s1 = *reinterpret_cast<const uint32_t*>(blk1 + 4 * K + wo);
+        const float s0l = __uint_as_float(s0 << 16) * 0.5f, s0h = __uint_as_float(s0 & 0xffff0000u) * 0.5f;
+        const float s1l = __uint_as_float(s1 << 16) * 0.5f, s1h = __uint_as_float(s1 & 0xffff0000u) * 0.5f;
+        tot0[0] = fmaf(d0[0], s0l, tot0[0]);
+        tot0[1] = fmaf(d0[1], s0l, tot0[1]);
+        tot0[2] = fmaf(d0[2], s0h, tot0[2]);
+        tot0[3] = fmaf(d0[3], s0h, tot0[3]);
+        tot1[0] = fmaf(d1[0], s1l, tot1[0]);
+        tot1[1] = fmaf(d1[1], s1l, tot1[1]);
+        tot1[2] = fmaf(d1[2], s1h, tot1[2]);
+        tot1[3] = fmaf(d1[3], s1h, tot1[3]);
+    }
+}
+
 // ---- B operands held in registers --------------------------------------------
 // A staged row in "fragment order": the 8 words lane (g, t) feeds to the 4
 // k-steps of quad q (k-pairs 8(4q+s)+t and 8(4q+s)+t+4, s = 0..3) sit

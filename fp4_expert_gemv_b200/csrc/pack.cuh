@@ -8,6 +8,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "mma.cuh"
 
 namespace fe {
 
@@ -55,6 +56,43 @@ __global__ void pack_kernel(const float* __restrict__ W, int64_t E, int64_t K, i
         for (int r = 0; r < 16; ++r) {
             uint32_t byte = 0;
             if (s != 0.0f) byte = e2m1x2_from_f32(__fdiv_rn(v[2 * r], s), __fdiv_rn(v[2 * r + 1], s));
+            dst[(int64_t)r * N] = (uint8_t)byte;
+        }
+    }
+}
+
+// INT2 scalar codes (the host packer's rule: scale bf16(max|w| / 1.5) per 32
+// along K, the nearest level q - 1.5, midpoints to the level above, four codes
+// per byte, the code of k = 4 b + i in bits 2i of byte row b).  One thread per
+// (expert, group of 32 k, column n).
+FE_DEV uint32_t int2_from_ratio(float r) { return r < -1.0f ? 0u : r < 0.0f ? 1u : r < 1.0f ? 2u : 3u; }
+
+__global__ void pack_int2_kernel(const float* __restrict__ W, int64_t E, int64_t K, int64_t N,
+                                 uint8_t* __restrict__ codes, uint16_t* __restrict__ scales)
+{
+    const int64_t G = K / 32;
+    const int64_t total = E * G * N;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i % N;
+        const int64_t eg = i / N;
+        const int64_t e = eg / G, g = eg - e * G;
+        const float* src = W + ((e * K) + g * 32) * N + n;
+        float v[32];
+        float mx = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) {
+            v[kk] = src[(int64_t)kk * N];
+            mx = fmaxf(mx, fabsf(v[kk]));
+        }
+        const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(mx, 1.5f));
+        scales[eg * N + n] = __bfloat16_as_ushort(sb);
+        const float s = __bfloat162float(sb);
+        uint8_t* dst = codes + (e * (K / 4) + g * 8) * N + n;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            uint32_t byte = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) byte |= (s != 0.0f ? int2_from_ratio(__fdiv_rn(v[4 * r + q], s)) : 2u) << (2 * q);
             dst[(int64_t)r * N] = (uint8_t)byte;
         }
     }
@@ -193,6 +231,106 @@ __global__ void relayout_rows_kernel(RowRelayoutParams p)
             const uint16_t* srow = p.src_scales + (e * G + g) * H;
             const uint32_t lo = srow[16 * tile + gg], hi = srow[16 * tile + gg + 8];
             *reinterpret_cast<uint32_t*>(dst + 8 * H + 4 * ws) = lo | (hi << 16);
+        }
+    }
+}
+
+// INT2 column blocks (mma.cuh, int2_block_bytes): the E2M1 blocks' fragment
+// order with two bits per code.  Source codes [E][K/4][N] (code of k in bits
+// 2(k % 4) of byte row k / 4).  One thread per destination 32-bit word: word
+// w (0, 1) of lane L = 4g + t in quad q holds register r = 4 (s & 1) + j of
+// k-step s = 2w + (r >> 2): the codes of column g + 8 (j & 1) at k =
+// 64q + 16s + 2t + 8 (j >> 1) (bits 2r) and k + 1 (bits 16 + 2r).
+FE_DEV uint32_t int2_code(const uint8_t* src, int64_t N, int64_t k, int64_t col)
+{
+    return (src[(k >> 2) * N + col] >> (2 * (k & 3))) & 3u;
+}
+
+__global__ void relayout_int2_kernel(RelayoutParams p)
+{
+    const int64_t nblk = p.N / 16, K = p.K;
+    const int64_t blk_bytes = int2_block_bytes((int)K);
+    const int64_t code_words = (K / 64) * 64;
+    const int64_t scale_words = (K / 32) * 8;
+    const int64_t per_blk = code_words + scale_words;
+    const int64_t total = p.E * nblk * per_blk;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t w = i % per_blk;
+        const int64_t eb = i / per_blk;
+        const int64_t e = eb / nblk, blk = eb % nblk;
+        const int64_t col0 = relayout_block_col0(p, blk);
+        uint8_t* dst = p.dst + eb * blk_bytes;
+        if (w < code_words) {
+            const int64_t q = w / 64, r64 = w % 64;
+            const int L = (int)(r64 / 2), ww = (int)(r64 % 2);
+            const int g = L >> 2, t = L & 3;
+            const uint8_t* src = p.src_codes + e * (K / 4) * p.N;
+            uint32_t v = 0;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int s = 2 * ww + (r >> 2), j = r & 3;
+                const int64_t col = col0 + g + 8 * (j & 1);
+                const int64_t ke = 64 * q + 16 * s + 2 * t + 8 * (j >> 1);
+                v |= int2_code(src, p.N, ke, col) << (2 * r);
+                v |= int2_code(src, p.N, ke + 1, col) << (16 + 2 * r);
+            }
+            *reinterpret_cast<uint32_t*>(dst + 256 * q + 8 * L + 4 * ww) = v;
+        } else {
+            const int64_t ws = w - code_words;
+            const int64_t G = ws / 8;
+            const int g = (int)(ws % 8);
+            const uint32_t lo = p.src_scales[(e * (K / 32) + G) * p.N + col0 + g];
+            const uint32_t hi = p.src_scales[(e * (K / 32) + G) * p.N + col0 + g + 8];
+            *reinterpret_cast<uint32_t*>(dst + 4 * K + 4 * ws) = lo | (hi << 16);
+        }
+    }
+}
+
+// INT2 W_dn row groups for the decode kernel: per expert and 32 rows, one 10H
+// run [codes of rows 0-15 (4H)][scales of the group (2H)][codes of rows 16-31
+// (4H)], the row groups of relayout_rows_kernel with two bits per code: word
+// w (0, 1) of lane L = 4g + c in quad q holds register r = 4 (s & 1) + j of
+// column tile 4q + s, s = 2w + (r >> 2): the codes of rows 2c + 8 (j >> 1)
+// (bits 2r) and that + 1 (bits 16 + 2r) of the 16, at column 16 tile + g +
+// 8 (j & 1).  Source codes [E][I/4][H].
+__global__ void relayout_int2_rows_kernel(RowRelayoutParams p)
+{
+    const int64_t H = p.H, G = p.I / 32;
+    const int64_t half_words = H;          // 4H bytes of codes
+    const int64_t scale_words = H / 2;     // 2H bytes of scales
+    const int64_t per_group = 2 * half_words + scale_words;
+    const int64_t total = p.E * G * per_group;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t w = i % per_group, eg = i / per_group;
+        const int64_t e = eg / G, g = eg % G;
+        uint8_t* dst = p.dst + eg * 10 * H;
+        if (w < half_words || w >= half_words + scale_words) {
+            const int half = w < half_words ? 0 : 1;
+            const int64_t wc = half == 0 ? w : w - half_words - scale_words;
+            const int64_t q = wc / 64, r64 = wc % 64;
+            const int L = (int)(r64 / 2), ww = (int)(r64 % 2);
+            const int gg = L >> 2, c = L & 3;
+            const uint8_t* src = p.src_codes + e * (p.I / 4) * H;
+            uint32_t v = 0;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int s = 2 * ww + (r >> 2), j = r & 3;
+                const int64_t tile = 4 * q + s;
+                const int64_t col = 16 * tile + gg + 8 * (j & 1);
+                const int64_t row = 32 * g + 16 * half + 2 * c + 8 * (j >> 1);
+                v |= int2_code(src, H, row, col) << (2 * r);
+                v |= int2_code(src, H, row + 1, col) << (16 + 2 * r);
+            }
+            const int64_t base = half == 0 ? 0 : 6 * H;
+            *reinterpret_cast<uint32_t*>(dst + base + 256 * q + 8 * L + 4 * ww) = v;
+        } else {
+            const int64_t ws = w - half_words;
+            const int64_t tile = ws / 8, gg = ws % 8;
+            const uint16_t* srow = p.src_scales + (e * G + g) * H;
+            const uint32_t lo = srow[16 * tile + gg], hi = srow[16 * tile + gg + 8];
+            *reinterpret_cast<uint32_t*>(dst + 4 * H + 4 * ws) = lo | (hi << 16);
         }
     }
 }

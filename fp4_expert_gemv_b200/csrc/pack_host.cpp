@@ -86,4 +86,57 @@ void pack(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint1
     for (auto& th : pool) th.join();
 }
 
+// INT2 scalar codes ("FireEcho Engine", sections "Quantization Formats" and
+// "FE-XC / INT2 Cold Expert Demotion": a scalar 2-bit format for the coldest
+// experts).  Per group of 32 k and column n: scale = bf16(float32(max|w| /
+// 1.5)); the code q of r = float32(w / scale) is the nearest of the levels
+// q - 1.5 (q = 0..3), an exact midpoint (r = -1, 0, 1) to the level above;
+// four codes per byte, the code of k = 4 b + i in bits 2i, 2i + 1 of byte
+// row b.  An all-zero group stores scale 0 and codes 2.
+static inline uint32_t encode_int2(float r)
+{
+    if (r < -1.0f) return 0;
+    if (r < 0.0f) return 1;
+    if (r < 1.0f) return 2;
+    return 3;
+}
+
+static void pack_int2_range(const float* W, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales, int64_t eg0,
+                            int64_t eg1)
+{
+    const int64_t G = K / 32;
+    for (int64_t eg = eg0; eg < eg1; ++eg) {
+        const int64_t e = eg / G, g = eg % G;
+        for (int64_t n = 0; n < N; ++n) {
+            const float* src = W + (e * K + g * 32) * N + n;
+            float mx = 0.0f;
+            for (int kk = 0; kk < 32; ++kk) mx = std::fmax(mx, std::fabs(src[kk * N]));
+            const uint16_t sb = bf16_rne_bits(mx / 1.5f);
+            scales[eg * N + n] = sb;
+            const float s = bf16_value(sb);
+            uint8_t* dst = codes + (e * (K / 4) + g * 8) * N + n;
+            for (int r = 0; r < 8; ++r) {
+                uint32_t byte = 0;
+                for (int i = 0; i < 4; ++i)
+                    byte |= (s != 0.0f ? encode_int2(src[(4 * r + i) * N] / s) : 2u) << (2 * i);
+                dst[r * N] = (uint8_t)byte;
+            }
+        }
+    }
+}
+
+void pack_int2(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales)
+{
+    const int64_t total = E * (K / 32);
+    unsigned nt = std::thread::hardware_concurrency();
+    if (nt == 0) nt = 1;
+    if ((int64_t)nt > total) nt = (unsigned)(total > 0 ? total : 1);
+    std::vector<std::thread> pool;
+    for (unsigned t = 0; t < nt; ++t) {
+        const int64_t a = total * t / nt, b = total * (t + 1) / nt;
+        pool.emplace_back(pack_int2_range, W, K, N, codes, scales, a, b);
+    }
+    for (auto& th : pool) th.join();
+}
+
 }  // namespace fe_host

@@ -109,6 +109,27 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uin
                              const uint8_t* down_codes, const uint16_t* down_scales, int src_on_device,
                              fe_stream_t stream);
 
+/* Load INT2 experts ("FireEcho Engine", "Quantization Formats": INT2, a
+ * scalar 2-bit format, 8x, for the coldest experts; "FE-XC / INT2 Cold Expert
+ * Demotion": hot experts FP4, the coldest INT2).  formats: host uint8 [E], 1 =
+ * expert e runs on the INT2 weights given here, 0 = on its E2M1 weights of
+ * fe_moe_load_packed (which stays required: it makes the layer loaded; the
+ * E2M1 bytes of INT2 experts are then ignored).  INT2 format: a 2-bit code q
+ * stands for (q - 1.5) times the bf16 scale of its group of 32 along K
+ * (scale = bf16(max|w| / 1.5), as fe_moe_pack_int2_host makes them); four
+ * codes per byte, the code of k = 4b + i in bits 2i, 2i+1 of byte row b:
+ *   gate_up_codes uint8 [E][H/4][2I], gate_up_scales bf16 [E][H/32][2I],
+ *   down_codes    uint8 [E][I/4][H],  down_scales    bf16 [E][I/32][H],
+ * full size (rows of E2M1 experts are ignored), host (src_on_device = 0) or
+ * device memory.  The first call allocates the INT2 buffers (15 * E * I * H
+ * / 16 bytes); the call waits for stream.  A layer with INT2 experts runs on the single-launch decode path
+ * only (T <= 8, T * top_k <= 16): fe_moe_forward returns FE_ERR_UNSUPPORTED
+ * for larger T, and a stack of such layers makes one launch per layer.
+ * H % 64 and I % 64 must be 0 (else FE_ERR_UNSUPPORTED). */
+fe_status fe_moe_load_int2(fe_moe_t h, const uint8_t* formats, const uint8_t* gate_up_codes,
+                           const uint16_t* gate_up_scales, const uint8_t* down_codes, const uint16_t* down_scales,
+                           int src_on_device, fe_stream_t stream);
+
 /* The layer: y = MoE(x) ("FireEcho Engine", "Speed Optimization History"
  * steps 1-5 and "The Goliath Kernel: Why It's Fast": grouped dispatch with
  * expert ids read from device memory, fused gate_up projection, FP4 decoded
@@ -237,6 +258,20 @@ fe_status fe_moe_pack_host(const float* W, int64_t E, int64_t K, int64_t N, uint
  * bytes identical to fe_moe_pack_host. */
 fe_status fe_moe_pack_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales,
                              fe_stream_t stream);
+
+/* The INT2 packer of fe_moe_load_int2's format: float W [E][K][N] -> codes
+ * [E][K/4][N] and bf16 scales [E][K/32][N].  Per group of 32 along k and
+ * column n: scale = bf16_rne(max|w| / 1.5) (float32 division); the code q of
+ * r = w / scale (float32) is the nearest of the levels q - 1.5, an exact
+ * midpoint (r = -1, 0, 1) going to the level above; an all-zero group stores
+ * scale 0 and codes 2.  K % 32 == 0.  Host version: host pointers,
+ * multithreaded, synchronous. */
+fe_status fe_moe_pack_int2_host(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes, uint16_t* scales);
+
+/* The same INT2 packer on the GPU: device pointers, enqueued on stream; bytes
+ * identical to fe_moe_pack_int2_host. */
+fe_status fe_moe_pack_int2_device(const float* W, int64_t E, int64_t K, int64_t N, uint8_t* codes,
+                                  uint16_t* scales, fe_stream_t stream);
 
 /* Allocation-free forward.  No counterpart on the source pages: an addition for
  * callers that must not allocate device memory -- for instance code running

@@ -72,6 +72,26 @@ def test_pack_host_matches_oracle_quantiser():
         assert np.array_equal(c, c_ref)
 
 
+def test_pack_int2_host_matches_oracle_quantiser():
+    import fp4_expert_gemv_b200 as fe
+    rng = np.random.default_rng(6)
+    cases = [(rng.standard_normal((2, 64, 40)) * 0.02).astype(np.float32),
+             (rng.standard_normal((1, 96, 8)) * 5).astype(np.float32)]
+    # exact midpoints between levels (r = -1, 0, 1 with the group max 1.5 -> scale 1)
+    W = np.zeros((1, 32, 4), np.float32)
+    W[0, 0, :] = 1.5
+    W[0, 1:8, 0] = [-1.0, 0.0, 1.0, -0.5, 0.5, -1.5, 0.999]
+    W[0, 1:8, 1] = [-1.0001, -0.9999, 1.0001, 0.9999, -0.0001, 0.0001, 2.0]
+    cases.append(W)
+    cases.append(np.zeros((1, 64, 3), np.float32))   # all-zero groups: scale 0, codes 2
+    orc = oracle.default()
+    for W in cases:
+        c, s = fe.pack_int2_host(W)
+        c_ref, s_ref = orc.quantize_int2(W)
+        assert np.array_equal(s, s_ref)
+        assert np.array_equal(c, c_ref)
+
+
 def test_synth_device_library_is_built():
     path = os.path.join(ROOT, "synth", "libfe_synth.so")
     assert os.path.exists(path)
