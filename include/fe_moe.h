@@ -227,7 +227,14 @@ fe_status fe_moe_last_forward_info(fe_moe_t h, int* path, int* kernels);
  * contents.  The streaming kernels of the moderate-T path write
  * [2][number of SMs][8] instead (gate_up, then down; per CTA clock64 at
  * start, range known, first unit landed, end; its unit count; %globaltimer
- * at start and end).  NULL switches it off. */
+ * at start and end).  The persistent stack launch (fe_moe_stack_forward at
+ * T = 1) uses the buffer of its first layer's handle as [number of SMs][16]:
+ * per CTA, compute thread 0's clock64 cycles summed over the stack per phase
+ * (0 x wait, 1 gate_up bytes wait, 2 gate_up, 3 SwiGLU step, 4 down bytes
+ * wait, 5 down, 6 slot release, 7 partial-buffer guard, 8 partial stores),
+ * 9 its units, 10 the whole layer loop, and the exchange warp's 11 poll
+ * cycles, 12 polls, 13 slice-sum cycles, 14 of them landing the words, 15
+ * adding them.  NULL switches it off. */
 fe_status fe_moe_set_trace(fe_moe_t h, unsigned long long* device_buf);
 
 /* For tests of the failure path: with unreachable = 1 the single-launch
