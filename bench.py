@@ -372,10 +372,12 @@ def run_workload(name, args, device, world, rank, headline=False):
     cur = torch.cuda.current_stream()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     torch.cuda.nvtx.range_push(f"timed {name}")   # lets a profiler select the timed launches
     e0.record(cur)
-    for _ in range(args.steps):
+    for i in range(args.steps):
         g.replay()
+        step_ev[i].record(cur)   # per-step samples (median, min) besides the total
     e1.record(cur)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -389,6 +391,7 @@ def run_workload(name, args, device, world, rank, headline=False):
         torch.cuda.synchronize()
     clk = clocks.stop()
     ms_local = e0.elapsed_time(e1) / args.steps
+    step_ms = [(e0 if i == 0 else step_ev[i - 1]).elapsed_time(step_ev[i]) for i in range(args.steps)]
     ms = max_over_ranks(ms_local, world, device)
     tokens_step = sum_over_ranks(layers * T, world, device)
     value = tokens_step / (ms / 1e3)
@@ -484,6 +487,7 @@ def run_workload(name, args, device, world, rank, headline=False):
                         "synchronous)"},
         "gpu_launches": launches_per_step * args.steps,
         "launches_per_step": launches_per_step,
+        "ms_per_step_median": float(np.median(step_ms)), "ms_per_step_min": float(np.min(step_ms)),
         "setup_s": setup_s,
         "l2": (f"inputs larger than L2: each step streams {layers} layers' routed experts ({bytes_step / 1e9:.2f} GB)"
                if bytes_step > L2_BYTES else
@@ -493,6 +497,9 @@ def run_workload(name, args, device, world, rank, headline=False):
         res["parity"] = parity
     if no_prefetch is not None:
         res["one_launch_per_layer"] = no_prefetch
+    if headline and not prefill_like(name):
+        res["single_layer_l2_flushed"] = single_layer_flushed(handles[0], x_dev[0], lg_dev[0], k, y_dev[0],
+                                                              bytes_layer[0], peaks)
     del g
     stack.close()
     for m in handles:
@@ -500,6 +507,45 @@ def run_workload(name, args, device, world, rank, headline=False):
     del handles
     torch.cuda.empty_cache()
     return res
+
+
+def prefill_like(name):
+    return name.startswith("prefill")
+
+
+def single_layer_flushed(layer, x, lg, k, y, nbytes, peaks, samples=40):
+    """One layer (the stack's layer 0) as a one-forward CUDA graph, replayed with L2
+    flushed between replays (a write of twice the L2 size, outside the timed events):
+    median and min over the samples, after 10 warm-up replays."""
+    import torch
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        layer.forward(x, lg, k, y, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        layer.forward(x, lg, k, y, stream=s)
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=x.device)
+    for _ in range(10):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(samples)]
+    cur = torch.cuda.current_stream()
+    for a, b in ev:
+        flush.fill_(1)
+        a.record(cur)
+        g.replay()
+        b.record(cur)
+    torch.cuda.synchronize()
+    us = np.array([a.elapsed_time(b) * 1e3 for a, b in ev])
+    del g, flush
+    med = float(np.median(us))
+    gbs = nbytes / (med * 1e-6) / 1e9
+    return {"us_median": med, "us_min": float(us.min()), "samples": samples,
+            "kernel": "single-launch decode kernel (fe_moe_forward)",
+            "achieved_gbs_at_median": gbs, "frac_of_measured_hbm": gbs / float(peaks["hbm_gbs"]),
+            "l2": f"{2 * l2 / 1e6:.0f} MB written between replays, outside the timed events"}
 
 
 def run_router(device):
@@ -703,6 +749,10 @@ def run_gpu(args):
         line["parity"] = head["parity"]
     if "one_launch_per_layer" in head:
         line["one_launch_per_layer"] = head["one_launch_per_layer"]
+    line["ms_per_step_median"] = head["ms_per_step_median"]
+    line["ms_per_step_min"] = head["ms_per_step_min"]
+    if "single_layer_l2_flushed" in head:
+        line["single_layer_l2_flushed"] = head["single_layer_l2_flushed"]
     if extra:
         line["workloads"] = extra
     if args.workload == "all":
