@@ -1017,9 +1017,14 @@ namespace {
 // one token, every layer on the single-launch decode kernel's shapes, the
 // layers' buffers unchanged since the stack was made, and x / y either chained
 // (y = x + H) or disjoint.  Returns 1 (independent), 2 (chained) or 0.
+// The persistent launch computes one token per launch: a call at T = 1, or at a few
+// tokens whose routing is sparse (T * top_k at most a quarter of E, so the tokens
+// rarely share an expert and a launch per token reads about the bytes one launch for
+// all would) runs as T launches.
 int stack_persistent_mode(fe_moe_stack_s* st, const void* x, void* y, int T, int top_k)
 {
-    if (!st->persistent_ok || !st->prefetch || T != 1 || top_k > fe::kStkMaxK) return 0;
+    if (!st->persistent_ok || !st->prefetch || top_k > fe::kStkMaxK) return 0;
+    if (T != 1 && (T > fe::kStkMaxTokens || 4 * T * top_k > st->E)) return 0;
     const int n = (int)st->layers.size();
     for (int l = 0; l < n; ++l) {
         fe_moe_s* h = st->layers[l];
@@ -1032,25 +1037,26 @@ int stack_persistent_mode(fe_moe_stack_s* st, const void* x, void* y, int T, int
             s.pair_row != h->pair_row)
             return 0;
     }
-    const size_t bytes = sizeof(uint16_t) * (size_t)n * st->H;
+    const size_t bytes = sizeof(uint16_t) * (size_t)n * T * st->H;
     const char* xb = static_cast<const char*>(x);
     const char* yb = static_cast<const char*>(y);
-    if (yb == xb + sizeof(uint16_t) * st->H) return 2;
+    if (yb == xb + sizeof(uint16_t) * (size_t)T * st->H) return 2;
     if (yb + bytes <= xb || xb + bytes <= yb) return 1;
     return 0;
 }
 
-fe_status stack_persistent_launch(fe_moe_stack_s* st, const void* x, const float* logits, int top_k, void* y,
-                                  int mode, cudaStream_t s)
+fe_status stack_persistent_launch(fe_moe_stack_s* st, const void* x, const float* logits, int T, int top_k,
+                                  void* y, int mode, cudaStream_t s)
 {
     fe_moe_s* h0 = st->layers[0];
     fe::StackParams sp{};
     sp.layers = st->d_layers;
     sp.L = (int)st->layers.size();
     sp.E = st->E; sp.H = st->H; sp.I = h0->I; sp.k = top_k;
-    sp.x = static_cast<const uint16_t*>(x);
-    sp.logits = logits;
-    sp.y = static_cast<uint16_t*>(y);
+    sp.T = T;
+    sp.ldx = (size_t)T * st->H;
+    sp.ldl = (size_t)T * st->E;
+    sp.ldy = (size_t)T * st->H;
     sp.chained = mode == 2;
     sp.part = st->part;
     sp.ctr = st->ctr;
@@ -1067,14 +1073,20 @@ fe_status stack_persistent_launch(fe_moe_stack_s* st, const void* x, const float
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    FE_CUDA_TRY(cudaLaunchKernelEx(&cfg, fe::stack_decode_kernel, sp));
+    for (int t = 0; t < T; ++t) {   // one launch per token: rows t of every layer
+        sp.t = t;
+        sp.x = static_cast<const uint16_t*>(x) + (size_t)t * st->H;
+        sp.logits = logits + (size_t)t * st->E;
+        sp.y = static_cast<uint16_t*>(y) + (size_t)t * st->H;
+        FE_CUDA_TRY(cudaLaunchKernelEx(&cfg, fe::stack_decode_kernel, sp));
+    }
     for (fe_moe_s* h : st->layers) {
-        h->last_T = 1;
+        h->last_T = T;
         h->last_k = top_k;
         h->last_path = FE_PATH_FUSED_DECODE;
         h->last_kernels = 0;
     }
-    st->last_launches = 1;
+    st->last_launches = T;
     return FE_OK;
 }
 
@@ -1105,7 +1117,7 @@ fe_status fe_moe_stack_forward(fe_moe_stack_t st, const void* x_bf16, const floa
     if (mode > 0) {
         DeviceGuard g(st->device);
         if (!g.ok) return FE_ERR_CUDA;
-        return stack_persistent_launch(st, x_bf16, logits, top_k, y_bf16, mode, (cudaStream_t)stream);
+        return stack_persistent_launch(st, x_bf16, logits, T, top_k, y_bf16, mode, (cudaStream_t)stream);
     }
     int launches = 0;
     for (int l = 0; l < n; ++l) {

@@ -54,6 +54,7 @@ constexpr int kStkBufs = 6;           // partial-output buffers, by layer mod 6
 constexpr int kStkRotate = 53;        // rotation of the unit split and the output slices per layer
 constexpr int kStkRouteWarps = 8;     // warps routing the layers at the start
 constexpr int kStkCand = 256;         // candidate keys per routing warp (k * E/32 at most)
+constexpr int kStkMaxTokens = 4;      // tokens of a stack call run as one launch each, at most
 constexpr int kStkRedFloats = 4096;   // routing candidates (8 x 256 keys); later the gate_up partials
 constexpr int kStkPartFloats = 512;   // gate_up partials: 16 warps x 32
 constexpr int kStkLandRow = 128;      // bytes of one CTA's share of one output slice (16 tagged words)
@@ -73,10 +74,13 @@ struct StackLayer {
 struct StackParams {
     const StackLayer* layers;   // [L], device memory
     int L, E, H, I, k;
-    const uint16_t* x;          // layer l reads x + l*H (bf16)
-    const float* logits;        // layer l: logits + l*E
-    uint16_t* y;                // layer l writes y + l*H
-    int chained;                // y + l*H == x + (l+1)*H
+    const uint16_t* x;          // layer l reads the row x + l*ldx (bf16)
+    const float* logits;        // layer l: the row logits + l*ldl
+    uint16_t* y;                // layer l writes the row y + l*ldy
+    size_t ldx, ldl, ldy;       // elements from one layer's row to the next (H, E, H for one token)
+    int T, t;                   // this launch computes token t of the layers' T tokens (x, logits and y
+                                //   point at token t's rows; launch t = 0 also writes every token's routing)
+    int chained;                // y + l*ldy == x + (l+1)*ldx
     unsigned long long* part;   // [kStkBufs][grid][H]: (tag << 32) | fp32 bits; within each 16-column
                                 //   tile, word 2g holds column g and word 2g + 1 column g + 8
     unsigned long long* ctr;    // [grid + 2 kStkBufs]: launches of CTA c; then per partial buffer b
@@ -136,6 +140,7 @@ __host__ __device__ inline StackSmem stack_smem_layout(int H)
     L.shared = L.mbar + 8 * (3 * kStkSlots + 2);
     L.red = align16(L.shared + (uint32_t)sizeof(StackShared));
     static_assert(kStkRedFloats * 4 >= kStkRouteWarps * kStkCand * 8, "routing candidates space");
+    static_assert(2 * kStkMaxTokens * kStkMaxK * 4 <= kStkCand * 8, "grouping of a few tokens in the candidates' space");
     // after routing, the candidates' space holds the gate_up partials and, behind them,
     // the landing rows of an output slice (one 128-byte row per CTA, written by cp.async)
     L.land = L.red + 4u * kStkPartFloats;
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
         int* se = S.rsel_e[warp];
         float* sw = S.rsel_w[warp];
         for (int l = warp; l < L; l += kStkRouteWarps) {
-            const bool nan = warp_route(p.logits + (size_t)l * E, E, k, lane, cand, kStkCand, se, sw);
+            const bool nan = warp_route(p.logits + (size_t)l * p.ldl, E, k, lane, cand, kStkCand, se, sw);
             if (nan && lane == 0) atomicOr(p.status, kDevNanLogit);
             warp_softmax(sw, k, lane);
             int pos = 0;
@@ -242,8 +247,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                 S.dex[l][pos] = se[lane];
                 S.dw[l][pos] = sw[lane];
             }
-            // the layer's routing outputs, from one CTA per layer
-            if (c == l % G) {
+            // the layer's routing outputs, from one CTA per layer: at one token, this one;
+            // with T tokens (one launch each), launch 0 routes them all (below)
+            if (c == l % G && p.T == 1) {
                 const StackLayer& ly = p.layers[l];
                 if (lane < k) {
                     ly.idx[lane] = se[lane];
@@ -260,6 +266,53 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                     ly.offsets[e] = below;
                     if (e < E) ly.counts[e] = eq;
                 }
+            }
+            if (c == l % G && p.T > 1 && p.t == 0) {
+                // every token of the layer routed (idx, w in slot order), then the pairs p =
+                // t*k + j grouped: the rank of a pair by (expert, pair id), and the offsets by
+                // binary search in the sorted experts, in the candidates' space (free again)
+                const StackLayer& ly = p.layers[l];
+                const int P = p.T * k;
+                for (int tt = 0; tt < p.T; ++tt) {
+                    warp_route(p.logits + (size_t)l * p.ldl + (size_t)tt * E, E, k, lane, cand, kStkCand, se, sw);
+                    warp_softmax(sw, k, lane);
+                    if (lane < k) {
+                        ly.idx[tt * k + lane] = se[lane];
+                        ly.w[tt * k + lane] = sw[lane];
+                    }
+                    __syncwarp();
+                }
+                int* sidx = reinterpret_cast<int*>(cand);
+                int* ssort = sidx + kStkMaxTokens * kStkMaxK;
+                for (int q = lane; q < P; q += 32) sidx[q] = ly.idx[q];
+                __syncwarp();
+                for (int q = lane; q < P; q += 32) {
+                    const int eq = sidx[q];
+                    int rank = 0;
+                    for (int r = 0; r < P; ++r) {
+                        const int er = sidx[r];
+                        rank += er < eq || (er == eq && r < q);
+                    }
+                    ssort[rank] = eq;
+                    ly.sorted_pair[rank] = q;
+                    ly.pair_row[q] = rank;
+                }
+                __syncwarp();
+                for (int e = lane; e <= E; e += 32) {
+                    int lo = 0, hi = P;   // first sorted position with expert >= e
+                    while (lo < hi) {
+                        const int m = (lo + hi) >> 1;
+                        if (ssort[m] < e) lo = m + 1; else hi = m;
+                    }
+                    int lo2 = lo, hi2 = P;   // ... and with expert > e
+                    while (lo2 < hi2) {
+                        const int m = (lo2 + hi2) >> 1;
+                        if (ssort[m] <= e) lo2 = m + 1; else hi2 = m;
+                    }
+                    ly.offsets[e] = lo;
+                    if (e < E) ly.counts[e] = lo2 - lo;
+                }
+                __syncwarp();
             }
             __syncwarp();
         }
@@ -365,7 +418,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
         if (lane == 0) {
             for (int l = 0; l < xin; ++l) {
                 mbar_expect_tx(bar_x(l), 2u * H);
-                bulk_g2s(smem_addr(xr + (size_t)l * H), p.x + (size_t)l * H, 2u * H, bar_x(l));
+                bulk_g2s(smem_addr(xr + (size_t)l * H), p.x + (size_t)l * p.ldx, 2u * H, bar_x(l));
             }
         }
         const unsigned long long t_start = globaltimer_ns();
@@ -392,7 +445,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                 }
                 if (uniform(ready)) {
                     const bool global_src = p.chained && xl > 0;
-                    const uint32_t* src = global_src ? reinterpret_cast<const uint32_t*>(p.x + (size_t)xl * H)
+                    const uint32_t* src = global_src ? reinterpret_cast<const uint32_t*>(p.x + (size_t)xl * p.ldx)
                                                      : reinterpret_cast<const uint32_t*>(xr + (size_t)(xl & 1) * H);
                     float m = 0.0f;
                     for (int r = lane; r < H / 2; r += 32) {
@@ -418,7 +471,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                         // the row buffer just read takes layer xl + 2's x
                         if (!p.chained && xl + 2 < L) {
                             mbar_expect_tx(bar_x(xl & 1), 2u * H);
-                            bulk_g2s(smem_addr(xr + (size_t)(xl & 1) * H), p.x + (size_t)(xl + 2) * H, 2u * H,
+                            bulk_g2s(smem_addr(xr + (size_t)(xl & 1) * H), p.x + (size_t)(xl + 2) * p.ldx, 2u * H,
                                      bar_x(xl & 1));
                             ++xin;
                         }
@@ -492,7 +545,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                         const float e0 = __shfl_sync(0xffffffffu, a0, cp + 24), e1 = __shfl_sync(0xffffffffu, a1, cp + 24);
                         if (grp == 0 && !late) {   // words 2cp, 2cp + 1 of a tile: columns cp, cp + 8
                             const uint32_t two = bf16x2_rn(((b0 + c0v) + d0) + e0, ((b1 + c1v) + d1) + e1);
-                            uint16_t* yr = p.y + (size_t)rl * H + 16 * sl;
+                            uint16_t* yr = p.y + (size_t)rl * p.ldy + 16 * sl;
                             yr[cp] = (uint16_t)(two & 0xffffu);
                             yr[cp + 8] = (uint16_t)(two >> 16);
                         }

@@ -362,8 +362,12 @@ fe_status fe_moe_stack_forward_host(fe_moe_stack_t s, const uint16_t* x_bf16_hos
 
 /* Cross-layer streaming on (1, the default) or off (0).  On: a call at T = 1
  * whose layers all take the single-launch decode kernel (same shape, x and y
- * chained as y = x + H or not overlapping) runs the whole stack as ONE
- * persistent launch, one CTA per SM: every layer is routed up front (the stack
+ * chained as y = x + T*H or not overlapping) runs the whole stack as ONE
+ * persistent launch, one CTA per SM; a call at T <= 4 tokens whose routing is
+ * sparse (4 * T * top_k <= E, so the tokens rarely share an expert) runs as
+ * one such launch per token, token t's rows of every layer in launch t (the
+ * first launch also writes every layer's routing and grouping of all T
+ * tokens, as fe_moe_forward leaves them): every layer is routed up front (the stack
  * takes every layer's logits at once), each CTA streams its share of the
  * layers' weights through a ring of shared-memory slots without stopping at
  * layer boundaries, so the next layer's weights arrive while the current one
@@ -376,8 +380,8 @@ fe_status fe_moe_stack_forward_host(fe_moe_stack_t s, const uint16_t* x_bf16_hos
  * their outputs agree to within rounding, not bit for bit. */
 fe_status fe_moe_stack_set_prefetch(fe_moe_stack_t s, int on);
 
-/* Kernels the last fe_moe_stack_forward enqueued (1 for the persistent
- * launch); -1 for a NULL stack. */
+/* Kernels the last fe_moe_stack_forward enqueued (1 per token for the
+ * persistent launches); -1 for a NULL stack. */
 int fe_moe_stack_last_launches(fe_moe_stack_t s);
 
 /* Free the stack's buffers (not the layers).  Waits for the device first. */

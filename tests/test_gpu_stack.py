@@ -188,3 +188,64 @@ def test_persistent_stack_one_token(torch_cuda, E, H, I, k):
     st, bits = layers[0].status()
     assert st == fe.FE_OK and bits == 0, f"device status bits {bits:#x}"
     stack.close()
+
+
+@pytest.mark.parametrize("T", [2, 4])
+def test_persistent_stack_few_sparse_tokens(torch_cuda, T):
+    """A few tokens with sparse routing (the 512-expert layer, top-10) run as one persistent
+    launch per token: against one launch per layer, the oracle on layer 0, and every layer's
+    routing and grouping of all T tokens bit for bit; independent and chained layers."""
+    torch = torch_cuda
+    import fp4_expert_gemv_b200 as fe
+    import oracle
+    E, H, I, k, n = 512, 2048, 512, 10, 3
+    layers = [harness.GpuLayer(E, H, I, 600 + l, max_T=T, max_k=k).layer for l in range(n)]
+    stack = fe.Stack(layers)
+    xs = np.stack([synth.activations_bf16(610 + l, T, H) for l in range(n)])
+    lg = np.ascontiguousarray(np.stack([synth.router_logits(620 + l, T, E) for l in range(n)]), dtype=np.float32)
+    x_dev = torch.from_numpy(xs.view(np.int16)).cuda()
+    lg_dev = torch.from_numpy(lg).cuda()
+    y1 = torch.empty_like(x_dev)
+    for _ in range(2):
+        stack.forward(x_dev.view(torch.bfloat16), lg_dev, k, y1.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert stack.last_launches() == T
+    ya = y1.cpu().numpy().view(np.uint16)
+    orc = oracle.default()
+    for l, layer in enumerate(layers):
+        idx, w, off, sp = layer.routing(T, k)
+        counts, pr = layer.grouping(T, k)
+        torch.cuda.synchronize()
+        idx_ref, w_ref = orc.route(lg[l], k)
+        c_ref, off_ref, sp_ref, pr_ref = orc.group(idx_ref, E)
+        assert np.array_equal(idx.cpu().numpy(), idx_ref) and np.array_equal(off.cpu().numpy(), off_ref)
+        assert np.array_equal(sp.cpu().numpy(), sp_ref) and np.array_equal(pr.cpu().numpy(), pr_ref)
+        assert np.array_equal(counts.cpu().numpy(), c_ref)
+        np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=1e-6, atol=1e-7)
+    osd = harness.OracleSide(E, H, I, 600)
+    harness.assert_output_close(ya[0], osd.forward(xs[0], lg[0], k)[0], f"persistent T={T}, layer 0")
+    stack.set_prefetch(False)
+    y2 = torch.empty_like(x_dev)
+    stack.forward(x_dev.view(torch.bfloat16), lg_dev, k, y2.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert stack.last_launches() > T
+    yb = y2.cpu().numpy().view(np.uint16)
+    for l in range(n):
+        harness.assert_output_close(ya[l], harness.bf16_to_f64(yb[l]), f"T={T} persistent against per-layer, layer {l}")
+    # chained: y = x shifted by one layer, per token
+    buf = torch.zeros((n + 1, T, H), dtype=torch.int16, device="cuda")
+    buf[0].copy_(x_dev[0])
+    stack.forward(buf[0:].view(torch.bfloat16), lg_dev, k, buf[1:].view(torch.bfloat16))
+    torch.cuda.synchronize()
+    yc_per = buf.cpu().numpy().view(np.uint16).copy()
+    stack.set_prefetch(True)
+    buf2 = torch.zeros_like(buf)
+    buf2[0].copy_(x_dev[0])
+    stack.forward(buf2[0:].view(torch.bfloat16), lg_dev, k, buf2[1:].view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert stack.last_launches() == T
+    yc = buf2.cpu().numpy().view(np.uint16)
+    harness.assert_output_close(yc[1], harness.bf16_to_f64(yc_per[1]), f"T={T} chained, layer 0 against per-layer")
+    st, bits = layers[0].status()
+    assert st == fe.FE_OK and bits == 0, f"device status bits {bits:#x}"
+    stack.close()
