@@ -32,6 +32,9 @@
 //     reads layer l's y) the exchange warp stages x_{l+1} once every slice of
 //     y_l is written.
 //
+// A stack call at a few tokens whose routing is sparse runs one launch per token
+// (layer rows T apart; launch 0 also writes every token's routing and grouping).
+//
 // Every wait is bounded by %globaltimer; the grid is one CTA per SM, all
 // resident at once (checked on the host from the kernel's occupancy).
 #pragma once

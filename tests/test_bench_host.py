@@ -1,0 +1,42 @@
+"""Host logic of bench.py (no GPU): the roofline's byte counts, the hash-gated
+ncu traffic record, and the count of distinct routed experts."""
+import json
+
+import numpy as np
+
+import bench
+import oracle
+import synth
+
+
+def test_algorithmic_bytes_match_the_stated_figures():
+    # per expert: gate_up codes + scales + down codes + scales (H 2048, I 768 and I 512)
+    assert bench.bytes_per_expert(2048, 768) == 2_654_208
+    assert bench.bytes_per_expert(2048, 512) == 1_769_472
+    # the decode layer at one token: 8 experts, x, logits, y
+    assert bench.algorithmic_bytes_per_layer(128, 2048, 768, 1, 8) == 21_242_368
+    # INT2: two bits per code, the same bf16 scales
+    H, I = 2048, 768
+    assert bench.int2_bytes_per_expert(H, I) == H * 2 * I // 4 + (H // 32) * 2 * I * 2 + I * H // 4 + (I // 32) * H * 2
+
+
+def test_distinct_routed_matches_the_oracle_routing():
+    lg = synth.router_logits(17, 64, 128, zipf_s=1.1)
+    idx, _ = oracle.default().route(lg, 8)
+    assert bench.distinct_routed(lg, 8) == len(np.unique(idx))
+
+
+def test_traffic_is_reported_only_while_the_sources_match(tmp_path, monkeypatch):
+    files = ["stack_decode.cuh", "common.cuh"]
+    good = bench.source_hash(files)
+    rec = {"entries": [{"workload": "decode_e128_t1", "kernel": "stack_decode_kernel", "sources": files,
+                        "sources_sha256_16": good, "dram_bytes_per_layer": 1000.0}]}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    assert bench.ncu_traffic("decode_e128_t1", 48) == (48000.0, "stack_decode_kernel")
+    assert bench.ncu_traffic("prefill_e128_t4096", 1) == (None, None)
+    rec["entries"][0]["sources_sha256_16"] = "0" * 16   # the kernel changed since the capture
+    path.write_text(json.dumps(rec))
+    assert bench.ncu_traffic("decode_e128_t1", 48) == (None, "stack_decode_kernel")
+
