@@ -495,9 +495,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeParams p)
             const int pid = S.sp[r0 + warp], t = pid / k;
             const float m = pow2f(S.xshift[t]);
             const float v = half == 0 ? silu_mul_fast(s * m, other * m) * S.sel_w[pid] : 0.0f;
-            float mx = fabsf(v);
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            // the row max: non-negative floats order as their bits, so one warp reduction
+            // (the other half-warp holds zeros)
+            const float mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v))));
             const int sh = fp16_shift(mx);
             const float sc = pow2f(-sh);
             const float vn = __shfl_down_sync(0xffffffffu, v, 1);

@@ -655,9 +655,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) stack_decode_kernel(StackParam
                     for (int w2 = 0; w2 < kStkWarps; ++w2) sacc += red[w2 * 32 + half * 16 + cc];
                     const float other = __shfl_xor_sync(0xffffffffu, sacc, 16);
                     const float v = half == 0 ? silu_mul_fast(sacc * xm, other * xm) * S.dw[l][d] : 0.0f;
-                    float mx = fabsf(v);
-#pragma unroll
-                    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    // the row max: non-negative floats order as their bits, so one warp reduction
+                    // (the other half-warp holds zeros)
+                    const float mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v))));
                     const int sh = fp16_shift(mx);
                     const float sc = pow2f(-sh);
                     const float vn = __shfl_down_sync(0xffffffffu, v, 1);
