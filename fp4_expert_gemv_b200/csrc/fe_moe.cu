@@ -964,7 +964,7 @@ fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack
     if (e == cudaSuccess) e = dmalloc(&st->a_stage, ((size_t)n_layers + 1) * row, nullptr);
     if (e == cudaSuccess) e = dmalloc(&st->b_stage, (size_t)n_layers * row, nullptr);
     if (e == cudaSuccess) e = dmalloc(&st->logits_stage, (size_t)n_layers * st->max_T * st->E, nullptr);
-    // the persistent launch for one token: every layer of one shape, small enough, the
+    // the persistent launches (one token each): every layer of one shape, small enough, the
     // kernel resident on every SM
     st->sm_count = layers[0]->sm_count;
     bool same = true;
@@ -1013,14 +1013,14 @@ fe_status fe_moe_stack_create(const fe_moe_t* layers, int n_layers, fe_moe_stack
 
 namespace {
 
-// Whether fe_moe_stack_forward can run the whole stack as one persistent launch:
-// one token, every layer on the single-launch decode kernel's shapes, the
-// layers' buffers unchanged since the stack was made, and x / y either chained
-// (y = x + H) or disjoint.  Returns 1 (independent), 2 (chained) or 0.
-// The persistent launch computes one token per launch: a call at T = 1, or at a few
-// tokens whose routing is sparse (T * top_k at most a quarter of E, so the tokens
-// rarely share an expert and a launch per token reads about the bytes one launch for
-// all would) runs as T launches.
+// Whether fe_moe_stack_forward can run the stack on the persistent kernel, which
+// computes one token per launch: a call at T = 1, or at a few tokens whose routing
+// is sparse (T * top_k at most a quarter of E, so the tokens rarely share an expert
+// and a launch per token reads about the bytes one launch for all would), runs as T
+// launches.  Also needed: every layer on the single-launch decode kernel's shapes
+// at one token, E2M1 experts only, the layers' buffers unchanged since the stack
+// was made, and x / y either chained (y = x + T*H) or disjoint.  Returns 1
+// (independent), 2 (chained) or 0.
 int stack_persistent_mode(fe_moe_stack_s* st, const void* x, void* y, int T, int top_k)
 {
     if (!st->persistent_ok || !st->prefetch || top_k > fe::kStkMaxK) return 0;

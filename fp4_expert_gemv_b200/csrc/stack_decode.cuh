@@ -1,4 +1,4 @@
-// A stack of decode layers at one token in one persistent launch.
+// A stack of decode layers, one token per persistent launch.
 //
 // "FireEcho Engine", sections "Benchmark Results" (row L6: the 48-layer
 // forward captured as one CUDA graph; row L2: the next layer pinned in L2
