@@ -49,7 +49,15 @@ NOMINAL_FP4_TFLOPS = 9000.0
 L2_BYTES = 126e6
 PATH_NAMES = {1: "moderate-T path: routing + streaming mma.sync projections (sg_kernel) + ordered combine",
               2: "large-T path: routing + tensor-core tiles (tc_gemm_kernel) + ordered combine",
-              3: "single-launch decode; a stack at T=1 runs as one persistent launch (stack_decode_kernel)"}
+              3: "single-launch decode kernel (decode_kernel), one launch per layer"}
+
+
+def kernel_label(path, launches_per_step, T):
+    """What ran the step: the persistent stack kernel when the step was one launch per token."""
+    if path == 3 and launches_per_step == T:
+        return ("persistent stack kernel (stack_decode_kernel): every layer in one launch"
+                + (" per token" if T > 1 else ""))
+    return PATH_NAMES.get(path, str(path))
 CSRC = os.path.join(ROOT, "fp4_expert_gemv_b200", "csrc")
 
 # DRAM bytes (read + write) of a workload's dominant kernel come from one ncu
@@ -456,7 +464,7 @@ def run_workload(name, args, device, world, rank, headline=False):
         tf = flops_layer * layers / (ms_local / 1e3) / 1e12
         tpeak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
         roofline = {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
-                    "traffic": traffic, "kernel": PATH_NAMES.get(path, str(path)),
+                    "traffic": traffic, "kernel": kernel_label(path, launches_per_step, T),
                     "peak_kind": f"{peak_kind} sustained dense bf16 (f16 operands run at the same rate)",
                     "algorithmic_flops_per_layer": flops_layer,
                     "frac_of_nominal_fp4_9pflops": tf / NOMINAL_FP4_TFLOPS}
@@ -468,7 +476,7 @@ def run_workload(name, args, device, world, rank, headline=False):
             no_prefetch["frac"] = a2 / float(peaks["hbm_gbs"])
         roofline = {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                     "frac": achieved / float(peaks["hbm_gbs"]), "traffic": traffic,
-                    "kernel": PATH_NAMES.get(path, str(path)), "peak_kind": f"{peak_kind} HBM copy",
+                    "kernel": kernel_label(path, launches_per_step, T), "peak_kind": f"{peak_kind} HBM copy",
                     "algorithmic_bytes_per_layer_mean": bytes_step / layers,
                     "distinct_experts_per_layer_mean": float(np.mean(distinct)),
                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS}

@@ -40,3 +40,10 @@ def test_traffic_is_reported_only_while_the_sources_match(tmp_path, monkeypatch)
     path.write_text(json.dumps(rec))
     assert bench.ncu_traffic("decode_e128_t1", 48) == (None, "stack_decode_kernel")
 
+
+
+def test_kernel_label_follows_the_launch_count():
+    assert "stack_decode_kernel" in bench.kernel_label(3, 1, 1)
+    assert "per token" in bench.kernel_label(3, 4, 4)
+    assert "decode_kernel" in bench.kernel_label(3, 48, 1) and "stack" not in bench.kernel_label(3, 48, 1)
+    assert "sg_kernel" in bench.kernel_label(1, 336, 64)
