@@ -110,6 +110,14 @@ class Oracle:
         lib.orc_router_logits.restype = i32
         lib.orc_moe_forward.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
         lib.orc_moe_forward.restype = i32
+        lib.orc_e4m3_decode.argtypes = [i32]
+        lib.orc_e4m3_decode.restype = ctypes.c_double
+        lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.orc_e4m3_encode.restype = i32
+        lib.orc_nvfp4_quantize.argtypes = [P, i64, i64, P, P, P]
+        lib.orc_nvfp4_quantize.restype = i32
+        lib.orc_moe_forward_nvfp4.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
+        lib.orc_moe_forward_nvfp4.restype = i32
         self.lib = lib
         self.path = path
 
@@ -204,6 +212,43 @@ class Oracle:
                                       weights._ptrs(weights.dn_codes), weights._ptrs(weights.dn_scales),
                                       _ptr(y64), _ptr(yb), _ptr(act))
         _check(rc, "moe_forward")
+        return (y64, yb, act) if want_act else (y64, yb)
+
+    def e4m3_decode(self, byte: int) -> float:
+        return self.lib.orc_e4m3_decode(int(byte))
+
+    def e4m3_encode(self, t: float) -> int:
+        return self.lib.orc_e4m3_encode(float(t))
+
+    def nvfp4_quantize(self, V: np.ndarray):
+        """NVFP4 encoding of the rows of float32 V [R, K]: (codes uint8 [R, K/2], E4M3 scale
+        factors uint8 [R, K/16], row scales float32 [R])."""
+        V = np.ascontiguousarray(V, dtype=np.float32)
+        R, K = V.shape
+        codes = np.empty((R, K // 2), dtype=np.uint8)
+        sf = np.empty((R, K // 16), dtype=np.uint8)
+        g = np.empty(R, dtype=np.float32)
+        _check(self.lib.orc_nvfp4_quantize(_ptr(V), R, K, _ptr(codes), _ptr(sf), _ptr(g)), "nvfp4_quantize")
+        return codes, sf, g
+
+    def moe_forward_nvfp4(self, weights: ExpertWeights, x_bf16: np.ndarray, logits: np.ndarray, k: int,
+                          want_act: bool = False):
+        """The block-scaled FP4 (NVFP4) variant of the layer: (y64, y_bf16[, act64]), act64 the
+        bf16-rounded act in pair order."""
+        E, H, I = weights.E, weights.H, weights.I
+        assert not weights.fmt.any(), "the NVFP4 variant re-encodes E2M1 experts"
+        x_bf16 = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+        logits = np.ascontiguousarray(logits, dtype=np.float32)
+        T = x_bf16.shape[0]
+        assert x_bf16.shape == (T, H) and logits.shape == (T, E)
+        y64 = np.zeros((T, H), dtype=np.float64)
+        yb = np.zeros((T, H), dtype=np.uint16)
+        act = np.zeros((T * k, I), dtype=np.float64) if want_act else None
+        rc = self.lib.orc_moe_forward_nvfp4(E, H, I, T, k, _ptr(x_bf16), _ptr(logits),
+                                            weights._ptrs(weights.gu_codes), weights._ptrs(weights.gu_scales),
+                                            weights._ptrs(weights.dn_codes), weights._ptrs(weights.dn_scales),
+                                            _ptr(y64), _ptr(yb), _ptr(act))
+        _check(rc, "moe_forward_nvfp4")
         return (y64, yb, act) if want_act else (y64, yb)
 
     def quantized_experts(self, E: int, Wgu: np.ndarray, Wdn: np.ndarray, experts, fmt=None) -> ExpertWeights:

@@ -383,3 +383,209 @@ int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, c
     return orc_moe_forward_fmt(E, H, I, T, k, x_bf16, logits, NULL, gu_codes, gu_scales, dn_codes, dn_scales, y64,
                                y_bf16, act64);
 }
+
+/* ---------------------------------------------------------------------- */
+/* Block-scaled FP4 variant of the projections (NVFP4).  An approximation  */
+/* of the layer above, not its definition: the tensor cores' FP4 rate      */
+/* ("FireEcho Engine", "The Goliath Kernel: Why It's Fast": FP4 operands at */
+/* the matmul) takes only scale factors that are E4M3 per 16 elements (or   */
+/* powers of two per 32), so the BF16 group scales cannot be fed exactly.  */
+/* This is the variant's own definition:                                   */
+/*                                                                          */
+/*   E4M3 (the scale factors): 1 sign, 4 exponent bits (bias 7), 3 mantissa */
+/*   bits; exponent field 0 is subnormal, m/8 * 2^-6; 0x7F and 0xFF are NaN; */
+/*   the largest finite value is 448 (0x7E).                                 */
+/*                                                                          */
+/*   NVFP4 encoding of a row of K values v (K a multiple of 16), every step */
+/*   in float32:                                                            */
+/*     g   = amax(|v|) / 2688          (2688 = 6 * 448: the row's scale)     */
+/*     d6  = 6 * g                                                          */
+/*     s_b = E4M3(amax_b / d6) for each block b of 16 (nearest, ties to the */
+/*           even mantissa, above 448 -> 448; 0 when d6 = 0)               */
+/*     q   = E2M1(v / (s_b * g))       (orc_e2m1_encode; 0 when s_b g = 0)   */
+/*   decoded value: E2M1(q) * s_b * g (exact in fp64).                      */
+/*                                                                          */
+/*   The layer: x (bf16) is encoded per token row; the gate_up and down     */
+/*   weights (the packed E2M1 * bf16 values, exact in float32) per output   */
+/*   column along K; gate_up and SwiGLU in fp64 on the decoded values; act  */
+/*   is rounded to bf16 (the form in which it crosses to the down           */
+/*   projection), encoded per pair row, down in fp64; routing and the       */
+/*   slot-order combine as in orc_moe_forward.                              */
+/* ---------------------------------------------------------------------- */
+double orc_e4m3_decode(int byte)
+{
+    const int b = byte & 0xFF;
+    const int e = (b >> 3) & 0xF, m = b & 7;
+    if ((b & 0x7F) == 0x7F) return NAN;
+    const double mag = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (b & 0x80) ? -mag : mag;
+}
+
+/* Nearest non-negative finite E4M3 value to t >= 0 by search over all of them, */
+/* ties to the even code; t above 448 gives 448.                               */
+int orc_e4m3_encode(float t)
+{
+    if (isnan(t)) return 0x7F;
+    if (t >= 448.0f) return 0x7E;
+    if (t <= 0.0f) return 0;
+    int best = 0;
+    double bd = fabs((double)t);
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double d = fabs((double)t - orc_e4m3_decode(c));
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            bd = d;
+            best = c;
+        }
+    }
+    return best;
+}
+
+static void orc_nvfp4_row(const float* v, int64_t K, uint8_t* codes, uint8_t* sf, float* g_out)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k)
+        if (fabsf(v[k]) > amax) amax = fabsf(v[k]);
+    const float g = amax / 2688.0f;
+    const float d6 = 6.0f * g;
+    for (int64_t c = 0; c < K / 2; ++c) codes[c] = 0;
+    for (int64_t b = 0; b < K / 16; ++b) {
+        float ab = 0.0f;
+        for (int64_t kk = 0; kk < 16; ++kk)
+            if (fabsf(v[b * 16 + kk]) > ab) ab = fabsf(v[b * 16 + kk]);
+        const int sb = (d6 > 0.0f) ? orc_e4m3_encode(ab / d6) : 0;
+        sf[b] = (uint8_t)sb;
+        const float dq = (float)orc_e4m3_decode(sb) * g;
+        for (int64_t kk = 0; kk < 16; ++kk) {
+            const int64_t k = b * 16 + kk;
+            const int code = (dq > 0.0f) ? orc_e2m1_encode(v[k] / dq) : 0;
+            if (k % 2 == 0) codes[k / 2] = (uint8_t)((codes[k / 2] & 0xF0) | code);
+            else            codes[k / 2] = (uint8_t)((codes[k / 2] & 0x0F) | (code << 4));
+        }
+    }
+    *g_out = g;
+}
+
+/* NVFP4 encoding of R rows of K values: codes [R][K/2] (low nibble = even k), */
+/* scale factors [R][K/16] (E4M3 bytes), row scales g [R].                     */
+int orc_nvfp4_quantize(const float* V, int64_t R, int64_t K, uint8_t* codes, uint8_t* sf, float* g)
+{
+    if (!V || !codes || !sf || !g || R < 0 || K <= 0 || K % 16) return ORC_EINVAL;
+    for (int64_t r = 0; r < R; ++r) orc_nvfp4_row(V + r * K, K, codes + r * (K / 2), sf + r * (K / 16), g + r);
+    return ORC_OK;
+}
+
+/* Decoded value of element k of an encoded row. */
+static double orc_nvfp4_value(const uint8_t* codes, const uint8_t* sf, float g, int64_t k)
+{
+    const int code = (k & 1) ? (codes[k / 2] >> 4) : (codes[k / 2] & 0x0F);
+    return orc_e2m1_decode(code) * orc_e4m3_decode(sf[k / 16]) * (double)g;
+}
+
+/* One expert matrix's columns [K/2][N] codes, [K/32][N] bf16 scales, encoded */
+/* column by column along K: qc [N][K/2], qs [N][K/16], qg [N].               */
+static void orc_nvfp4_columns(const uint8_t* codes, const uint16_t* scales, int64_t K, int64_t N, uint8_t* qc,
+                              uint8_t* qs, float* qg, float* col)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) col[k] = orc_weight(codes, scales, N, k, n);
+        orc_nvfp4_row(col, K, qc + n * (K / 2), qs + n * (K / 16), qg + n);
+    }
+}
+
+typedef struct {
+    uint8_t *gc, *gs, *dc, *ds;
+    float *gg, *dg;
+} orc_nvfp4_expert;
+
+/* The NVFP4 variant of the layer (arguments as orc_moe_forward, E2M1 experts; */
+/* act64 [T*k][I] receives the bf16-rounded act in pair order).                */
+int orc_moe_forward_nvfp4(int E, int H, int I, int T, int k, const uint16_t* x_bf16, const float* logits,
+                          const uint8_t* const* gu_codes, const uint16_t* const* gu_scales,
+                          const uint8_t* const* dn_codes, const uint16_t* const* dn_scales, double* y64,
+                          uint16_t* y_bf16, double* act64)
+{
+    if (E <= 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || T < 0 || k < 1 || k > E) return ORC_EINVAL;
+    if (T == 0) return ORC_OK;
+    if (!x_bf16 || !logits || !gu_codes || !gu_scales || !dn_codes || !dn_scales) return ORC_EINVAL;
+    const int64_t N1 = 2 * (int64_t)I;
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    float* w = (float*)malloc(sizeof(float) * (size_t)k);
+    float* xf = (float*)malloc(sizeof(float) * (size_t)H);
+    uint8_t* xc = (uint8_t*)malloc((size_t)H / 2);
+    uint8_t* xs = (uint8_t*)malloc((size_t)H / 16);
+    float* af = (float*)malloc(sizeof(float) * (size_t)I);
+    uint8_t* ac = (uint8_t*)malloc((size_t)I / 2);
+    uint8_t* as = (uint8_t*)malloc((size_t)I / 16);
+    float* col = (float*)malloc(sizeof(float) * (size_t)(H > I ? H : I));
+    double* gu = (double*)malloc(sizeof(double) * (size_t)N1);
+    double* o = (double*)malloc(sizeof(double) * (size_t)H);
+    double* y = (double*)malloc(sizeof(double) * (size_t)H);
+    orc_nvfp4_expert* ex = (orc_nvfp4_expert*)calloc((size_t)E, sizeof(orc_nvfp4_expert));
+    int rc = ORC_OK;
+    if (!idx || !w || !xf || !xc || !xs || !af || !ac || !as || !col || !gu || !o || !y || !ex) {
+        rc = ORC_ENOMEM;
+        goto done;
+    }
+    for (int t = 0; t < T; ++t) {
+        rc = orc_route(logits + (int64_t)t * E, 1, E, k, idx, w);
+        if (rc) goto done;
+        float gx;
+        for (int h = 0; h < H; ++h) xf[h] = orc_bf16_to_f32(x_bf16[(int64_t)t * H + h]);
+        orc_nvfp4_row(xf, H, xc, xs, &gx);
+        for (int h = 0; h < H; ++h) y[h] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[j];
+            if (!gu_codes[e] || !gu_scales[e] || !dn_codes[e] || !dn_scales[e]) { rc = ORC_EINVAL; goto done; }
+            orc_nvfp4_expert* q = &ex[e];
+            if (!q->gc) {   /* encode this expert's weights once */
+                q->gc = (uint8_t*)malloc((size_t)(N1 * H / 2));
+                q->gs = (uint8_t*)malloc((size_t)(N1 * H / 16));
+                q->gg = (float*)malloc(sizeof(float) * (size_t)N1);
+                q->dc = (uint8_t*)malloc((size_t)H * (size_t)I / 2);
+                q->ds = (uint8_t*)malloc((size_t)H * (size_t)I / 16);
+                q->dg = (float*)malloc(sizeof(float) * (size_t)H);
+                if (!q->gc || !q->gs || !q->gg || !q->dc || !q->ds || !q->dg) { rc = ORC_ENOMEM; goto done; }
+                orc_nvfp4_columns(gu_codes[e], gu_scales[e], H, N1, q->gc, q->gs, q->gg, col);
+                orc_nvfp4_columns(dn_codes[e], dn_scales[e], I, H, q->dc, q->ds, q->dg, col);
+            }
+            /* gate_up: K = H, N = 2I */
+            for (int64_t n = 0; n < N1; ++n) {
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < H; ++kk)
+                    acc += orc_nvfp4_value(xc, xs, gx, kk) *
+                           orc_nvfp4_value(q->gc + n * (H / 2), q->gs + n * (H / 16), q->gg[n], kk);
+                gu[n] = acc;
+            }
+            for (int i = 0; i < I; ++i) {
+                const double gv = gu[i], uv = gu[I + i];
+                af[i] = orc_bf16_to_f32(orc_f64_to_bf16_rne(gv / (1.0 + exp(-gv)) * uv));
+            }
+            if (act64)
+                for (int i = 0; i < I; ++i) act64[((int64_t)t * k + j) * I + i] = (double)af[i];
+            float ga;
+            orc_nvfp4_row(af, I, ac, as, &ga);
+            /* down: K = I, N = H */
+            for (int64_t h = 0; h < H; ++h) {
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < I; ++kk)
+                    acc += orc_nvfp4_value(ac, as, ga, kk) *
+                           orc_nvfp4_value(q->dc + h * (I / 2), q->ds + h * (I / 16), q->dg[h], kk);
+                o[h] = acc;
+            }
+            /* weighted combine, slot order */
+            for (int h = 0; h < H; ++h) y[h] += o[h] * (double)w[j];
+        }
+        for (int h = 0; h < H; ++h) {
+            if (y64) y64[(int64_t)t * H + h] = y[h];
+            if (y_bf16) y_bf16[(int64_t)t * H + h] = orc_f64_to_bf16_rne(y[h]);
+        }
+    }
+done:
+    if (ex)
+        for (int e = 0; e < E; ++e) {
+            free(ex[e].gc); free(ex[e].gs); free(ex[e].gg); free(ex[e].dc); free(ex[e].ds); free(ex[e].dg);
+        }
+    free(ex); free(idx); free(w); free(xf); free(xc); free(xs); free(af); free(ac); free(as); free(col);
+    free(gu); free(o); free(y);
+    return rc;
+}

@@ -22,7 +22,15 @@ oracle disagrees with:
   nearest-level encoding with the stated tie rule, single-element layout probes
   (two bits per code, four codes per byte, one scale max|w|/1.5 per 32 along
   K), the rounding bound, and a dense brute-force layer whose experts mix
-  E2M1 and INT2.
+  E2M1 and INT2;
+* for the block-scaled FP4 (NVFP4) variant: the E4M3 bit-field definition and
+  the table in golden/e4m3_values.txt, brute-force nearest E4M3 encoding in
+  exact arithmetic (ties to the even code, saturation at 448), the row
+  encoding redone with numpy float32 steps and exact nearest searches,
+  single-element layout probes (two codes per byte, one scale factor per 16,
+  one row scale), the closed form of a constant row, the rounding bound, sign
+  symmetry, and a dense brute-force variant layer; the variant stays within a
+  loose distance of the exact layer.
 """
 from __future__ import annotations
 
@@ -498,6 +506,210 @@ def check_mixed_dense_bruteforce(o, rng):
     assert np.abs(y64 - ref).max() <= 1e-10 * np.abs(ref).max()
 
 
+# -- the NVFP4 variant -------------------------------------------------------------
+
+def e4m3_from_bits(b: int) -> float:
+    """E4M3 value from its bit fields (OCP OFP8 E4M3: bias 7, no infinities, S.1111.111 NaN)."""
+    s, e, m = (b >> 7) & 1, (b >> 3) & 15, b & 7
+    if e == 15 and m == 7:
+        return float("nan")
+    mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return -mag if s else mag
+
+
+E4M3_POS = [Fraction(e4m3_from_bits(c)) for c in range(0x7F)]   # the non-negative finite values
+
+
+def brute_e4m3(t) -> int:
+    """Nearest non-negative finite E4M3 code to t >= 0 in exact arithmetic, ties to the even
+    code, values above the largest (448) to 448."""
+    t = Fraction(float(t))
+    if t >= E4M3_POS[-1]:
+        return 0x7E
+    best, bd = 0, None
+    for c, v in enumerate(E4M3_POS):
+        d = abs(t - v)
+        if bd is None or d < bd or (d == bd and c % 2 == 0):
+            best, bd = c, d
+    return best
+
+
+def nvfp4_row_reference(v: np.ndarray):
+    """The NVFP4 row encoding, each rounding step done by numpy float32 and each nearest-value
+    choice by exact search: (codes [K/2], sf [K/16], g)."""
+    v = np.asarray(v, dtype=np.float32)
+    K = v.shape[0]
+    amax = np.float32(np.abs(v).max()) if K else np.float32(0)
+    g = np.float32(amax / np.float32(2688.0))
+    d6 = np.float32(np.float32(6.0) * g)
+    codes = np.zeros(K // 2, dtype=np.uint8)
+    sf = np.zeros(K // 16, dtype=np.uint8)
+    for b in range(K // 16):
+        blk = v[16 * b:16 * b + 16]
+        ab = np.float32(np.abs(blk).max())
+        sb = brute_e4m3(np.float32(ab / d6)) if d6 > 0 else 0
+        sf[b] = sb
+        dq = np.float32(np.float32(e4m3_from_bits(sb)) * g)
+        for kk in range(16):
+            k = 16 * b + kk
+            c = brute_force_code(float(np.float32(blk[kk] / dq))) if dq > 0 else 0
+            codes[k // 2] |= np.uint8(c << (4 * (k % 2)))
+    return codes, sf, g
+
+
+def nvfp4_decode_rows(codes: np.ndarray, sf: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """codes [R, K/2], sf [R, K/16], g [R] -> float64 [R, K]."""
+    R, K2 = codes.shape
+    vals = np.empty((R, 2 * K2))
+    vals[:, 0::2] = E2M1_TABLE[codes & 0x0F]
+    vals[:, 1::2] = E2M1_TABLE[codes >> 4]
+    s = np.repeat(np.array([[e4m3_from_bits(int(b)) for b in row] for row in sf]), 16, axis=1)
+    return vals * s * g.astype(np.float64)[:, None]
+
+
+def check_e4m3_table(o):
+    rows = [ln.split() for ln in open(os.path.join(GOLDEN, "e4m3_values.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    assert len(rows) >= 12
+    for b_s, v_s in rows:
+        b, v = int(b_s, 16), float(v_s)
+        got, ref = o.e4m3_decode(b), e4m3_from_bits(b)
+        if math.isnan(v):
+            assert math.isnan(got) and math.isnan(ref), f"byte {b:#x}"
+        else:
+            assert ref == v and got == v and math.copysign(1, got) == math.copysign(1, v), f"byte {b:#x}"
+    for b in range(256):
+        got, ref = o.e4m3_decode(b), e4m3_from_bits(b)
+        assert (math.isnan(got) and math.isnan(ref)) or got == ref, f"byte {b:#x}"
+    pos = [o.e4m3_decode(b) for b in range(0x7F)]
+    assert all(a < b for a, b in zip(pos, pos[1:]))
+
+
+def check_e4m3_encode(o, rng):
+    vals = [float(v) for v in E4M3_POS]
+    mids = [(a + b) / 2 for a, b in zip(E4M3_POS, E4M3_POS[1:])]
+    base = np.array(vals + [float(m) for m in mids] + [448.0, 464.0, 480.0, 1e6, 2.0 ** -10, 2.0 ** -11, 0.0],
+                    dtype=np.float32)
+    near = np.concatenate([np.nextafter(base, np.float32(np.inf)), np.nextafter(base, np.float32(0))])
+    rnd = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(600.0), 600)).astype(np.float32)
+    for t in np.concatenate([base, near, rnd]):
+        assert o.e4m3_encode(float(t)) == brute_e4m3(t), f"e4m3({float(t)!r})"
+
+
+def _nvfp4_probe_rows(rng) -> np.ndarray:
+    K = 64
+    rows = [rng.standard_normal(K) * 0.02, rng.standard_normal(K) * 30.0, rng.standard_normal(K) * 1e-5,
+            np.where(rng.random(K) < 0.3, rng.standard_normal(K), 0.0), np.zeros(K),
+            rng.standard_normal(K) * np.repeat(10.0 ** rng.uniform(-6, 2, K // 16), 16)]
+    # values on the E2M1 decision points of their block
+    r = rng.standard_normal(K) * 0.1
+    r[0] = 1.0
+    r[1:8] = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]) / 6.0
+    rows.append(r)
+    return np.array(rows, dtype=np.float32)
+
+
+def check_nvfp4_row_bruteforce(o, rng):
+    V = _nvfp4_probe_rows(rng)
+    codes, sf, g = o.nvfp4_quantize(V)
+    for r in range(V.shape[0]):
+        c_ref, s_ref, g_ref = nvfp4_row_reference(V[r])
+        assert g[r] == g_ref, f"row {r}: g {g[r]!r} vs {g_ref!r}"
+        assert np.array_equal(sf[r], s_ref), f"row {r}: scale factors"
+        assert np.array_equal(codes[r], c_ref), f"row {r}: codes"
+
+
+def check_nvfp4_layout(o):
+    K = 48
+    for (k, v) in [(0, 0.3), (17, -2.5), (47, 1e-3), (32, 7.0)]:
+        V = np.zeros((1, K), dtype=np.float32)
+        V[0, k] = v
+        codes, sf, g = o.nvfp4_quantize(V)
+        # the single value is its row's and its block's maximum: scale factor 448, code 6
+        assert g[0] == np.float32(np.float32(abs(v)) / np.float32(2688.0))
+        exp_sf = np.zeros(K // 16, dtype=np.uint8)
+        exp_sf[k // 16] = 0x7E
+        assert np.array_equal(sf[0], exp_sf), (k, sf[0])
+        exp_c = np.zeros(K // 2, dtype=np.uint8)
+        exp_c[k // 2] = (0xF if v < 0 else 0x7) << (4 * (k % 2))
+        assert np.array_equal(codes[0], exp_c), (k, codes[0])
+
+
+def check_nvfp4_closed_form_and_bounds(o, rng):
+    # a constant row decodes to itself exactly: g = c / 2688, scale factor 448, code 6
+    for c in [0.37, 1.0, 3e-4, 250.0]:
+        V = np.full((1, 32), c, dtype=np.float32)
+        codes, sf, g = o.nvfp4_quantize(V)
+        assert np.all(codes == 0x77) and np.all(sf == 0x7E)
+        assert np.allclose(nvfp4_decode_rows(codes, sf, g), np.float32(c), rtol=2e-7, atol=0)
+    V = _nvfp4_probe_rows(rng)
+    codes, sf, g = o.nvfp4_quantize(V)
+    dec = nvfp4_decode_rows(codes, sf, g)
+    for r in range(V.shape[0]):
+        for b in range(V.shape[1] // 16):
+            s = e4m3_from_bits(int(sf[r, b])) * float(g[r])
+            blk = V[r, 16 * b:16 * b + 16].astype(np.float64)
+            if s == 0.0:
+                assert np.all(dec[r, 16 * b:16 * b + 16] == 0.0)
+                continue
+            # the block maximum fits below 6 s up to the scale factor's rounding (3 mantissa bits)
+            assert np.abs(blk).max() <= 6.0 * s * (1.0 + 2.0 ** -4) * (1 + 1e-6)
+            # nearest-value rounding: within half of the widest E2M1 gap (2 s) unless saturated
+            err = np.abs(blk - dec[r, 16 * b:16 * b + 16])
+            assert np.all(err <= np.maximum(1.0 * s, np.abs(blk) - 6.0 * s) * (1 + 1e-6) + 1e-300)
+    # sign symmetry
+    c2, s2, g2 = o.nvfp4_quantize(-V)
+    assert np.array_equal(s2, sf) and np.array_equal(g2, g)
+    nz_lo, nz_hi = (codes & 0x07) != 0, (codes & 0x70) != 0
+    flip = (nz_lo * 0x08 + nz_hi * 0x80).astype(np.uint8)
+    assert np.array_equal(c2, codes ^ flip)
+
+
+def nvfp4_dense_layer_reference(o, x_bf16, logits, k, gu_c, gu_s, dn_c, dn_s):
+    """The NVFP4 variant, unpermuted: every operand encoded with the (pinned) row encoder,
+    every token through every expert as dense float64 matmuls, act rounded to bf16 by
+    enumeration of its neighbours, the routing mask applied at the end."""
+    T, H = x_bf16.shape
+    E = logits.shape[1]
+    I = dn_c.shape[1] * 2
+    xq = nvfp4_decode_rows(*o.nvfp4_quantize(bf16_to_f64(x_bf16).astype(np.float32)))
+    Wgu = dequant_dense(gu_c, gu_s)       # [E, H, 2I]
+    Wdn = dequant_dense(dn_c, dn_s)       # [E, I, H]
+    y = np.zeros((T, H))
+    for e in range(E):
+        wg = nvfp4_decode_rows(*o.nvfp4_quantize(Wgu[e].T.astype(np.float32))).T   # columns along K
+        wd = nvfp4_decode_rows(*o.nvfp4_quantize(Wdn[e].T.astype(np.float32))).T
+        for t in range(T):
+            order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))
+            sel = list(order[:k])
+            if e not in sel:
+                continue
+            ls = logits[t, order[:k]].astype(np.float64)
+            wsel = (np.exp(ls - ls[0]) / np.exp(ls - ls[0]).sum()).astype(np.float32).astype(np.float64)
+            h = xq[t] @ wg
+            a = h[:I] / (1.0 + np.exp(-h[:I])) * h[I:]
+            a16 = np.array([nearest_bf16_bits(np.float32(v)) if abs(v) < 3e38 else 0 for v in a], dtype=np.uint16)
+            aq = nvfp4_decode_rows(*o.nvfp4_quantize(bf16_to_f64(a16)[None, :].astype(np.float32)))[0]
+            y[t] += wsel[sel.index(e)] * (aq @ wd)
+    return y
+
+
+def check_nvfp4_dense_bruteforce(o, rng):
+    for (E, H, I, T, k) in [(4, 64, 32, 3, 2), (6, 32, 64, 2, 3)]:
+        gu_c, gu_s, dn_c, dn_s = _layer_inputs(rng, E, H, I, T, random_codes=True)
+        x = rng.standard_normal((T, H)).astype(np.float32)
+        x_bf16 = (x.view(np.uint32) >> 16).astype(np.uint16)
+        logits = rng.standard_normal((T, E)).astype(np.float32)
+        ew = _expert_weights(E, H, I, gu_c, gu_s, dn_c, dn_s)
+        y64, _ = o.moe_forward_nvfp4(ew, x_bf16, logits, k)
+        ref = nvfp4_dense_layer_reference(o, x_bf16, logits, k, gu_c, gu_s, dn_c, dn_s)
+        scale = np.abs(ref).max()
+        assert np.abs(y64 - ref).max() <= 1e-10 * scale, np.abs(y64 - ref).max() / scale
+        # the variant approximates the exact layer (a swapped operand or a lost scale would not)
+        exact, _ = o.moe_forward(ew, x_bf16, logits, k)
+        assert np.linalg.norm(y64 - exact) <= 0.3 * np.linalg.norm(exact)
+
+
 ALL_CHECKS = [
     ("e2m1_table", lambda o, rng: check_e2m1_table(o)),
     ("encode_bruteforce", check_encode_bruteforce),
@@ -518,4 +730,10 @@ ALL_CHECKS = [
     ("int2_quantize_layout", lambda o, rng: check_int2_quantize_layout(o)),
     ("int2_roundtrip", check_int2_roundtrip),
     ("mixed_dense_bruteforce", check_mixed_dense_bruteforce),
+    ("e4m3_table", lambda o, rng: check_e4m3_table(o)),
+    ("e4m3_encode", check_e4m3_encode),
+    ("nvfp4_row_bruteforce", check_nvfp4_row_bruteforce),
+    ("nvfp4_layout", lambda o, rng: check_nvfp4_layout(o)),
+    ("nvfp4_closed_form_and_bounds", check_nvfp4_closed_form_and_bounds),
+    ("nvfp4_dense_bruteforce", check_nvfp4_dense_bruteforce),
 ]

@@ -45,6 +45,14 @@ MUTANTS = [
     ("mixed_ignores_format", "const int f = fmt ? fmt[e] : 0;", "const int f = 0;"),
     ("down_scale_group", "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[(k / 32) * N + n]);",
      "return (float)orc_e2m1_decode(code) * orc_bf16_to_f32(scales[((k / 32) / 2) * N + n]);"),
+    ("e4m3_tie_odd", "if (d < bd || (d == bd && (c & 1) == 0)) {", "if (d < bd || (d == bd && (c & 1) == 1)) {"),
+    ("e4m3_bias", "ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
+    ("nvfp4_row_scale", "const float g = amax / 2688.0f;", "const float g = amax / 1344.0f;"),
+    ("nvfp4_block_max_of_first_block", "if (fabsf(v[b * 16 + kk]) > ab) ab = fabsf(v[b * 16 + kk]);",
+     "if (fabsf(v[kk]) > ab) ab = fabsf(v[kk]);"),
+    ("nvfp4_act_not_bf16", "af[i] = orc_bf16_to_f32(orc_f64_to_bf16_rne(gv / (1.0 + exp(-gv)) * uv));",
+     "af[i] = (float)(gv / (1.0 + exp(-gv)) * uv);"),
+    ("nvfp4_down_reads_unencoded_act", "acc += orc_nvfp4_value(ac, as, ga, kk) *", "acc += (double)af[kk] *"),
 ]
 
 
