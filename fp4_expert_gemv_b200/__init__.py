@@ -30,7 +30,7 @@ FE_DEVICE_EXCHANGE_TIMEOUT = 0x4
 FE_DEVICE_LOAD_TIMEOUT = 0x8
 FE_DEVICE_TC_TIMEOUT = 0x10
 
-PATH_AUTO, PATH_GEMV, PATH_TCGEN05, PATH_FUSED_DECODE = 0, 1, 2, 3
+PATH_AUTO, PATH_GEMV, PATH_TCGEN05, PATH_FUSED_DECODE, PATH_NVFP4 = 0, 1, 2, 3, 4
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is not built; run `python fp4_expert_gemv_b200/build.py`")
@@ -75,6 +75,8 @@ _SIGS = {
     "fe_moe_pack_int2_host": (_st, [_P, _i64, _i64, _i64, _P, _P]),
     "fe_moe_pack_int2_device": (_st, [_P, _i64, _i64, _i64, _P, _P, _P]),
     "fe_moe_forward_router": (_st, [_P, _P, _P, _i32, _i32, _P, _P, _P]),
+    "fe_moe_load_nvfp4": (_st, [_P, _P, _P, _P, _P, _i32, _P]),
+    "fe_moe_nvfp4_quantize_device": (_st, [_P, _i64, _i64, _P, _P, _P, _P]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -170,6 +172,22 @@ class MoELayer:
         else:
             check(fe_moe_load_int2(self.h, fmt.ctypes.data, _dptr(gu_codes), _dptr(gu_scales), _dptr(dn_codes),
                                    _dptr(dn_scales), 1, _stream_ptr(stream)), "fe_moe_load_int2")
+
+    def load_nvfp4(self, gu_codes, gu_scales, dn_codes, dn_scales, stream=None):
+        """The block-scaled FP4 re-encoding of the packed weights (the arrays of load_packed:
+        host numpy arrays or device torch tensors); then set_path(PATH_NVFP4) runs the variant."""
+        import numpy as np
+        if isinstance(gu_codes, np.ndarray):
+            arrs = [np.ascontiguousarray(a) for a in (gu_codes, gu_scales, dn_codes, dn_scales)]
+            check(fe_moe_load_nvfp4(self.h, *[a.ctypes.data for a in arrs], 0, _stream_ptr(stream)),
+                  "fe_moe_load_nvfp4")
+            import torch
+            torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+        else:
+            for t in (gu_codes, gu_scales, dn_codes, dn_scales):
+                assert t.is_cuda and t.is_contiguous()
+            check(fe_moe_load_nvfp4(self.h, _dptr(gu_codes), _dptr(gu_scales), _dptr(dn_codes), _dptr(dn_scales),
+                                    1, _stream_ptr(stream)), "fe_moe_load_nvfp4")
 
     def router(self, x_bf16, w_router_bf16, top_k: int, logits=None, idx=None, w=None, stream=None):
         """The router GEMM fused with the top-k: (logits [T, E] f32, idx [T, k] i32, w [T, k] f32)."""
@@ -345,6 +363,20 @@ def pack_int2_device(W, codes=None, scales=None, stream=None):
     check(fe_moe_pack_int2_device(_dptr(W), E, K, N, _dptr(codes), _dptr(scales), _stream_ptr(stream)),
           "fe_moe_pack_int2_device")
     return codes, scales
+
+
+def nvfp4_quantize_device(V, stream=None):
+    """torch float32 CUDA [R, K] -> NVFP4 (codes uint8 [R, K/2], E4M3 scale factors uint8 [R, K/16],
+    row scales float32 [R])."""
+    import torch
+    R, K = V.shape
+    assert V.is_cuda and V.is_contiguous() and V.dtype == torch.float32
+    codes = torch.empty((R, K // 2), dtype=torch.uint8, device=V.device)
+    sf = torch.empty((R, K // 16), dtype=torch.uint8, device=V.device)
+    g = torch.empty((R,), dtype=torch.float32, device=V.device)
+    check(fe_moe_nvfp4_quantize_device(_dptr(V), R, K, _dptr(codes), _dptr(sf), _dptr(g), _stream_ptr(stream)),
+          "fe_moe_nvfp4_quantize_device")
+    return codes, sf, g
 
 
 def pack_device(W, codes=None, scales=None, stream=None):

@@ -16,6 +16,7 @@
 #include "gemv.cuh"
 #include "gemv_canonical.cuh"
 #include "gmma.cuh"
+#include "nvfp4.cuh"
 #include "pack.cuh"
 #include "route.cuh"
 #include "route_large.cuh"
@@ -74,6 +75,14 @@ struct fe_moe_s {
     int32_t* tc_tiles = nullptr;            // [max tiles][3]
     int32_t* tc_ntiles = nullptr;           // [1]
     int32_t* grp_bh = nullptr;              // grouping for many tokens: [P / kGroupChunk + 1][E]
+    // block-scaled FP4 variant (nvfp4.cuh, fe_moe_load_nvfp4): weight tile images and
+    // row scales, built at load; token tile images per forward (workspace)
+    uint8_t* nv_gu = nullptr;               // [E][2I/128][H/256] x kNvAChunk bytes
+    uint8_t* nv_dn = nullptr;               // [E][H/128][I/256] x kNvAChunk bytes
+    float* nv_gug = nullptr;                // [E][2I]
+    float* nv_dng = nullptr;                // [E][H]
+    uint8_t* nv_b = nullptr;                // [tile slots][max(H, I)/256] x kNvBChunk bytes
+    float* nv_bg = nullptr;                 // [tile slots][256]
     float* rt_part = nullptr;               // router GEMM: K-split partials (router.cuh)
     unsigned* rt_ticket = nullptr;          // router GEMM: per 16-token tile, CTAs done
     uint32_t* status = nullptr;
@@ -151,7 +160,7 @@ void free_workspace(fe_moe_s* h)
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
                     h->dec_part, h->dec_epoch, h->sg_table, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
-                    h->tc_tiles, h->tc_ntiles, h->grp_bh, h->rt_part, h->rt_ticket};
+                    h->tc_tiles, h->tc_ntiles, h->grp_bh, h->rt_part, h->rt_ticket, h->nv_b, h->nv_bg};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
@@ -165,6 +174,8 @@ void free_workspace(fe_moe_s* h)
     h->grp_bh = nullptr;
     h->rt_part = nullptr;
     h->rt_ticket = nullptr;
+    h->nv_b = nullptr;
+    h->nv_bg = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -263,6 +274,10 @@ fe_status decode_path(fe_moe_s* h, const void* x, const float* logits, int T, in
 // rows) and 256 output columns per tile.
 bool tc_shape_ok(const fe_moe_s* h) { return h->I % 128 == 0 && h->H % 256 == 0; }
 
+// Shapes of the block-scaled FP4 variant: K stages of 256 for both projections
+// (so also 128-row weight tiles of 2I and H).
+bool nv_shape_ok(const fe_moe_s* h) { return h->I % 256 == 0 && h->H % 256 == 0; }
+
 // Token-expert pairs from which the automatic path choice takes the tensor
 // cores (below it the grouped mma.sync kernels keep the weights' single pass).
 constexpr int kTcAutoPairs = 4096;
@@ -338,6 +353,10 @@ cudaError_t configure_kernels(const fe_moe_s* h)
         e = cudaFuncSetAttribute(fe::tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fe::tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fe::nvfp4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fe::nvfp4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     // (the streaming kernels hold a little static shared state besides)
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fe::sg_kernel<true, kSgGateUpBlocks>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -535,6 +554,54 @@ fe_status tcgen05_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_
     return FE_OK;
 }
 
+// Token tile images of the block-scaled FP4 variant: slots x K stages.
+size_t nv_token_bytes(const fe_moe_s* h, size_t slots)
+{
+    return slots * (size_t)(std::max(h->H, h->I) / fe::kNvKc) * fe::kNvBChunk;
+}
+
+// Block-scaled FP4 variant (nvfp4.cuh): tile list, x rows gathered into NVFP4
+// token images, gate_up tiles (SwiGLU into act, bf16), act rows into token
+// images, down tiles (into o, bf16).  Routing and grouping ran before; the
+// ordered combine runs after.
+fe_status nvfp4_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t s)
+{
+    const int P = T * k;
+    const int max_tiles = (int)tc_max_tiles(h, (size_t)P);
+    fe::tc_tiles_kernel<<<1, 1024, 0, s>>>(h->counts, h->offsets, h->E, h->tc_tiles, h->tc_ntiles);
+    const unsigned row_blocks = (unsigned)(((size_t)max_tiles * fe::kNvN + 7) / 8);
+    fe::nvfp4_token_rows_kernel<<<row_blocks, 256, 0, s>>>(x, h->H, h->tc_tiles, h->tc_ntiles, h->sorted_pair, k, 1,
+                                                           h->nv_b, h->nv_bg);
+    fe::NvParams np{};
+    np.tiles = h->tc_tiles;
+    np.n_tiles = h->tc_ntiles;
+    np.status = h->status;
+    np.timeout_ns = 200ull * 1000 * 1000;
+    np.b_img = h->nv_b;
+    np.b_g = h->nv_bg;
+    np.a_img = h->nv_gu;
+    np.a_g = h->nv_gug;
+    np.MT = 2 * h->I / fe::kNvM;
+    np.KC = h->H / fe::kNvKc;
+    np.out = reinterpret_cast<uint16_t*>(h->act);
+    np.out_ld = h->I;
+    fe::nvfp4_gemm_kernel<true><<<dim3(np.MT, max_tiles), fe::kNvThreads, fe::nv_smem_bytes(), s>>>(np);
+    FE_CUDA_TRY(cudaGetLastError());
+    // act was left as bf16 rows by sorted position
+    fe::nvfp4_token_rows_kernel<<<row_blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(h->act), h->I,
+                                                           h->tc_tiles, h->tc_ntiles, h->sorted_pair, k, 0, h->nv_b,
+                                                           h->nv_bg);
+    np.a_img = h->nv_dn;
+    np.a_g = h->nv_dng;
+    np.MT = h->H / fe::kNvM;
+    np.KC = h->I / fe::kNvKc;
+    np.out = reinterpret_cast<uint16_t*>(h->o);
+    np.out_ld = h->H;
+    fe::nvfp4_gemm_kernel<false><<<dim3(np.MT, max_tiles), fe::kNvThreads, fe::nv_smem_bytes(), s>>>(np);
+    FE_CUDA_TRY(cudaGetLastError());
+    return FE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -645,6 +712,10 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
         if (e == cudaSuccess) e = dmalloc(&h->tc_tiles, 3 * tc_max_tiles(h, P), &acc);
         if (e == cudaSuccess) e = dmalloc(&h->tc_ntiles, 1, &acc);
     }
+    if (h->nv_gu) {
+        if (e == cudaSuccess) e = dmalloc(&h->nv_b, nv_token_bytes(h, tc_max_tiles(h, P)), &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->nv_bg, tc_max_tiles(h, P) * fe::kNvN, &acc);
+    }
     h->work_bytes = 0;
     for (auto& row : h->dec_planned)
         for (bool& b : row) b = false;
@@ -722,6 +793,79 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gu_codes, const uint16_t
     if (staging) FE_CUDA_TRY(cudaFreeAsync(staging, s));
     h->loaded = true;
     return FE_OK;
+}
+
+fe_status fe_moe_load_nvfp4(fe_moe_t h, const uint8_t* gu_codes, const uint16_t* gu_scales, const uint8_t* dn_codes,
+                            const uint16_t* dn_scales, int src_on_device, fe_stream_t stream)
+{
+    if (!h || !gu_codes || !gu_scales || !dn_codes || !dn_scales) return FE_ERR_INVALID_ARG;
+    if (!nv_shape_ok(h)) return FE_ERR_UNSUPPORTED;
+    DeviceGuard g(h->device);
+    if (!g.ok) return FE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t E = h->E, H = h->H, I = h->I;
+    const size_t gu_c = (size_t)E * (H / 2) * (2 * I), gu_s = (size_t)E * (H / 32) * (2 * I);
+    const size_t dn_c = (size_t)E * (I / 2) * H, dn_s = (size_t)E * (I / 32) * H;
+    const uint8_t* sgc = gu_codes;
+    const uint16_t* sgs = gu_scales;
+    const uint8_t* sdc = dn_codes;
+    const uint16_t* sds = dn_scales;
+    if (!h->nv_gu) {
+        cudaError_t e = cudaSuccess;
+        size_t acc = 0;
+        if (e == cudaSuccess) e = dmalloc(&h->nv_gu, (size_t)E * (2 * I / fe::kNvM) * (H / fe::kNvKc) * fe::kNvAChunk, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->nv_dn, (size_t)E * (H / fe::kNvM) * (I / fe::kNvKc) * fe::kNvAChunk, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->nv_gug, (size_t)E * 2 * I, &acc);
+        if (e == cudaSuccess) e = dmalloc(&h->nv_dng, (size_t)E * H, &acc);
+        if (e == cudaSuccess && h->max_T > 0) {
+            const size_t slots = tc_max_tiles(h, (size_t)h->max_T * h->max_k);
+            e = dmalloc(&h->nv_b, nv_token_bytes(h, slots), &h->work_bytes);
+            if (e == cudaSuccess) e = dmalloc(&h->nv_bg, slots * fe::kNvN, &h->work_bytes);
+        }
+        if (e != cudaSuccess) {
+            void* ptrs[] = {h->nv_gu, h->nv_dn, h->nv_gug, h->nv_dng, h->nv_b, h->nv_bg};
+            for (void* q : ptrs)
+                if (q) cudaFree(q);
+            h->nv_gu = h->nv_dn = h->nv_b = nullptr;
+            h->nv_gug = h->nv_dng = h->nv_bg = nullptr;
+            return record_cuda(e, "fe_moe_load_nvfp4 allocation");
+        }
+        h->weight_bytes += acc;
+    }
+    void* staging = nullptr;
+    if (!src_on_device) {
+        const size_t bytes = gu_c + 2 * gu_s + dn_c + 2 * dn_s;
+        FE_CUDA_TRY(cudaMallocAsync(&staging, bytes, s));
+        uint8_t* b = static_cast<uint8_t*>(staging);
+        FE_CUDA_TRY(cudaMemcpyAsync(b, gu_codes, gu_c, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c, gu_scales, 2 * gu_s, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c + 2 * gu_s, dn_codes, dn_c, cudaMemcpyHostToDevice, s));
+        FE_CUDA_TRY(cudaMemcpyAsync(b + gu_c + 2 * gu_s + dn_c, dn_scales, 2 * dn_s, cudaMemcpyHostToDevice, s));
+        sgc = b;
+        sgs = reinterpret_cast<const uint16_t*>(b + gu_c);
+        sdc = b + gu_c + 2 * gu_s;
+        sds = reinterpret_cast<const uint16_t*>(b + gu_c + 2 * gu_s + dn_c);
+    }
+    const long long n_gu = E * 2 * I, n_dn = E * H;
+    fe::nvfp4_weights_kernel<<<(unsigned)((n_gu + 255) / 256), 256, 0, s>>>(sgc, sgs, (int)E, (int)H, (int)(2 * I), 1,
+                                                                             (int)I, h->nv_gu, h->nv_gug);
+    fe::nvfp4_weights_kernel<<<(unsigned)((n_dn + 255) / 256), 256, 0, s>>>(sdc, sds, (int)E, (int)I, (int)H, 0,
+                                                                             (int)I, h->nv_dn, h->nv_dng);
+    FE_CUDA_TRY(cudaGetLastError());
+    if (staging) FE_CUDA_TRY(cudaFreeAsync(staging, s));
+    return FE_OK;
+}
+
+fe_status fe_moe_nvfp4_quantize_device(const float* src, int64_t rows, int64_t K, uint8_t* codes, uint8_t* sf,
+                                       float* row_scale, fe_stream_t stream)
+{
+    if (!src || !codes || !sf || !row_scale || rows < 0 || K < 16 || K % 16 || rows > (int64_t)1 << 26 ||
+        K > (int64_t)1 << 20)
+        return FE_ERR_INVALID_ARG;
+    if (rows == 0) return FE_OK;
+    fe::nvfp4_rows_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+        src, (int)rows, (int)K, codes, sf, row_scale);
+    return cudaGetLastError() == cudaSuccess ? FE_OK : FE_ERR_CUDA;
 }
 
 fe_status fe_moe_load_int2(fe_moe_t h, const uint8_t* formats, const uint8_t* gu_codes, const uint16_t* gu_scales,
@@ -820,6 +964,23 @@ fe_status forward_impl(fe_moe_t h, const void* x_bf16, const float* router_logit
     }
     // INT2 experts are read by the single-launch decode kernel only
     if (h->has_int2) return FE_ERR_UNSUPPORTED;
+    if (h->path == FE_PATH_NVFP4) {
+        if (!h->nv_gu || !h->nv_b || !h->tc_tiles) return FE_ERR_UNSUPPORTED;
+        const fe_status rs = route_and_group(h, router_logits, T, top_k, nullptr, s);
+        if (rs != FE_OK) return rs;
+        const fe_status st = nvfp4_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
+        if (st != FE_OK) return st;
+        dim3 cgrid((h->H / 8 + 255) / 256, T);
+        fe::combine_kernel<true><<<cgrid, 256, 0, s>>>(h->o, h->w, h->pair_row, h->H, top_k,
+                                                        static_cast<__nv_bfloat16*>(y_bf16));
+        FE_CUDA_TRY(cudaGetLastError());
+        h->last_T = T;
+        h->last_k = top_k;
+        h->last_path = FE_PATH_NVFP4;
+        const bool large_route = T >= kRouteLargeTokens && fe::route_large_ok(h->E, top_k);
+        h->last_kernels = (large_route ? 4 : 1) + 5 + 1;   // routing, tiles + 2 x (token images, tiles), combine
+        return FE_OK;
+    }
 
     const bool use_tc = tc_ok && (h->path == FE_PATH_TCGEN05 || (h->path == FE_PATH_AUTO && P >= kTcAutoPairs));
     SgSetup sg;
@@ -1227,7 +1388,7 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits)
 
 fe_status fe_moe_set_path(fe_moe_t h, int path)
 {
-    if (!h || path < FE_PATH_AUTO || path > FE_PATH_FUSED_DECODE) return FE_ERR_INVALID_ARG;
+    if (!h || path < FE_PATH_AUTO || path > FE_PATH_NVFP4) return FE_ERR_INVALID_ARG;
     h->path = path;
     return FE_OK;
 }
@@ -1262,7 +1423,8 @@ void fe_moe_destroy(fe_moe_t h)
         DeviceGuard g(h->device);
         cudaDeviceSynchronize();
         free_workspace(h);
-        void* ptrs[] = {h->gu_blocks, h->dn_blocks, h->dn_rows, h->fmt, h->gu2_blocks, h->dn2_rows};
+        void* ptrs[] = {h->gu_blocks, h->dn_blocks, h->dn_rows, h->fmt, h->gu2_blocks, h->dn2_rows,
+                        h->nv_gu, h->nv_dn, h->nv_gug, h->nv_dng};
         for (void* p : ptrs)
             if (p) cudaFree(p);
     }

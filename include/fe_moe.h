@@ -126,6 +126,37 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uin
  * only (T <= 8, T * top_k <= 16): fe_moe_forward returns FE_ERR_UNSUPPORTED
  * for larger T, and a stack of such layers makes one launch per layer.
  * H % 64 and I % 64 must be 0 (else FE_ERR_UNSUPPORTED). */
+/* Block-scaled FP4 variant of the projections ("FireEcho Engine", "The Goliath
+ * Kernel: Why It's Fast": FP4 codes at the matmul; the tensor cores' FP4 rate
+ * takes only E4M3 scale factors per 16 elements, which the bf16 group scales
+ * are not).  Re-encodes the layer's packed weights -- the same arrays, layout
+ * and src_on_device convention as fe_moe_load_packed -- into NVFP4, per output
+ * column along K:
+ *   g = amax / 2688 (fp32 row scale), s_b = E4M3(amax_b / (6 g)) per block of
+ *   16 (nearest, ties to even, at most 448), code = E2M1(w / (s_b g)) (nearest,
+ *   ties to even), every step in fp32,
+ * into tile images the kernels copy as they are (27 E I H / 16 bytes with
+ * their scale factors, plus the row scales; allocated by the first call).  With FE_PATH_NVFP4 set, fe_moe_forward then encodes x per token and
+ * act (bf16) per pair row the same way and runs both projections as
+ * kind::mxf4nvf4 MMAs with fp32 accumulation: an approximation of the layer,
+ * whose distance to it the caller measures (it is not within the layer's
+ * tolerance).  Needs H % 256 == 0 and I % 256 == 0 (else FE_ERR_UNSUPPORTED)
+ * and fe_moe_load_packed for the routing workspace's layer; token images are
+ * workspace of fe_moe_reserve (tile slots x max(H, I) / 256 x 36 KiB).  Work is
+ * enqueued on stream; host sources are staged through a stream-ordered buffer. */
+fe_status fe_moe_load_nvfp4(fe_moe_t h, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
+                            const uint8_t* down_codes, const uint16_t* down_scales, int src_on_device,
+                            fe_stream_t stream);
+
+/* The NVFP4 row encoding of fe_moe_load_nvfp4 on rows of fp32 values: src
+ * device float [rows][K] -> device codes uint8 [rows][K/2] (two per byte, the
+ * low nibble for the even k; bit 3 the sign), E4M3 scale factors uint8
+ * [rows][K/16], row scales float [rows].  A value decodes as E2M1(code) *
+ * E4M3(scale factor) * row scale.  K % 16 == 0, K >= 16 (else
+ * FE_ERR_INVALID_ARG).  Asynchronous on stream. */
+fe_status fe_moe_nvfp4_quantize_device(const float* src, int64_t rows, int64_t K, uint8_t* codes, uint8_t* sf,
+                                       float* row_scale, fe_stream_t stream);
+
 fe_status fe_moe_load_int2(fe_moe_t h, const uint8_t* formats, const uint8_t* gate_up_codes,
                            const uint16_t* gate_up_scales, const uint8_t* down_codes, const uint16_t* down_scales,
                            int src_on_device, fe_stream_t stream);
@@ -208,6 +239,9 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
                                    H % 256 == 0, scales in the exact-f16 range) */
 #define FE_PATH_FUSED_DECODE 3  /* one kernel for the whole layer (T <= 8, T * top_k <= 16), its CTAs all
                                    resident at once (checked from the occupancy; otherwise not taken) */
+#define FE_PATH_NVFP4 4         /* routing + block-scaled FP4 tensor-core tiles (tcgen05.mma kind::mxf4nvf4)
+                                   + combine: an approximation of the layer (fe_moe_load_nvfp4); any T;
+                                   never chosen by FE_PATH_AUTO */
 
 /* Force a compute path (FE_PATH_*); FE_ERR_UNSUPPORTED from forward if the
  * forced path cannot run the call.  For tests and measurements. */

@@ -2,7 +2,9 @@
 // library's own headers and run on the CPU (tests/test_host_plans.py): the unit
 // split of the decode kernels, the per-layer rotation of the persistent stack,
 // its per-buffer count targets, the shared-memory layouts against the per-block
-// limit, the router's K splits, and the B-fragment word order.  Prints "ok" or
+// limit, the router's K splits, the B-fragment word order, and the NVFP4 tile
+// images (every byte of a stage written once, a row's scale factors of one
+// k-block in one word, the gate/up row order).  Prints "ok" or
 // the first failed check, and exits nonzero on a failure.
 #include <cstdio>
 #include <cstdlib>
@@ -10,6 +12,7 @@
 
 #include "../fp4_expert_gemv_b200/csrc/router.cuh"
 #include "../fp4_expert_gemv_b200/csrc/stack_decode.cuh"
+#include "../fp4_expert_gemv_b200/csrc/nvfp4.cuh"
 #include "../fp4_expert_gemv_b200/csrc/tcgen05.cuh"
 
 static int failures = 0;
@@ -96,6 +99,43 @@ int main()
             if (w >= base && w < base + 32) ++seen[w - base];
         }
         for (int i = 0; i < 32; ++i) CHECK(seen[i] == 1, "block %u word %d", base, i);
+    }
+    // NVFP4 tile images: code bytes, A and B scale factors each a bijection onto their region
+    {
+        std::vector<int> seen(fe::kNvBChunk, 0);
+        for (int r = 0; r < fe::kNvN; ++r)
+            for (int kb = 0; kb < 128; ++kb) ++seen[fe::nv_code_off(r, kb)];
+        for (int n = 0; n < fe::kNvN; ++n)
+            for (int j = 0; j < 16; ++j) ++seen[fe::nv_sfb_off(n, j)];
+        for (uint32_t i = 0; i < fe::kNvBChunk; ++i) CHECK(seen[i] == 1, "B image byte %u seen %d", i, seen[i]);
+        std::vector<int> sa(fe::kNvAChunk, 0);
+        for (int r = 0; r < fe::kNvM; ++r) {
+            for (int kb = 0; kb < 128; ++kb) ++sa[fe::nv_code_off(r, kb)];
+            for (int j = 0; j < 16; ++j) ++sa[fe::nv_sfa_off(r, j)];
+        }
+        for (uint32_t i = 0; i < fe::kNvAChunk; ++i) CHECK(sa[i] == 1, "A image byte %u seen %d", i, sa[i]);
+        // a row's scale factors of one k-block are one 32-bit word (the tensor core reads them as one)
+        for (int r = 0; r < fe::kNvN; ++r)
+            for (int q = 0; q < 4; ++q) {
+                CHECK(fe::nv_sfb_off(r, 4 * q) % 4 == 0 && fe::nv_sfb_off(r, 4 * q + 3) == fe::nv_sfb_off(r, 4 * q) + 3,
+                      "B row %d k-block %d", r, q);
+                if (r < fe::kNvM)
+                    CHECK(fe::nv_sfa_off(r, 4 * q) % 4 == 0 && fe::nv_sfa_off(r, 4 * q + 3) == fe::nv_sfa_off(r, 4 * q) + 3,
+                          "A row %d k-block %d", r, q);
+            }
+        for (int I : {128, 256, 768}) {
+            std::vector<int> col(2 * I, 0);
+            for (int R = 0; R < 2 * I; ++R) ++col[fe::nv_gate_up_column(R, I)];
+            for (int n = 0; n < 2 * I; ++n) CHECK(col[n] == 1, "I=%d column %d", I, n);
+            // gate and up of act column i sit 16 rows apart in one 32-row group
+            for (int i = 0; i < I; ++i) {
+                const int Rg = 32 * (i / 16) + i % 16;
+                CHECK(fe::nv_gate_up_column(Rg, I) == i && fe::nv_gate_up_column(Rg + 16, I) == I + i, "I=%d i=%d", I, i);
+            }
+        }
+        CHECK(fe::nv_smem_bytes() <= kMaxSmem, "NVFP4 tiles %u", fe::nv_smem_bytes());
+        CHECK(256u + 4u * fe::kNvSfCols <= fe::kNvTmemCols, "TMEM columns");
+        CHECK(fe::nv_instr_desc(256) == ((1u << 7) | (1u << 10) | (32u << 17) | (8u << 24)), "instruction descriptor");
     }
     if (failures) {
         std::printf("%d checks failed\n", failures);
