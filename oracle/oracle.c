@@ -402,7 +402,8 @@ int orc_moe_forward(int E, int H, int I, int T, int k, const uint16_t* x_bf16, c
 /*     d6  = 6 * g                                                          */
 /*     s_b = E4M3(amax_b / d6) for each block b of 16 (nearest, ties to the */
 /*           even mantissa, above 448 -> 448; 0 when d6 = 0)               */
-/*     q   = E2M1(v / (s_b * g))       (orc_e2m1_encode; 0 when s_b g = 0)   */
+/*     q   = E2M1(v * r_b), r_b = 1 / (s_b * g)  (orc_e2m1_encode; 0 when   */
+/*           s_b g = 0): the block's fp32 reciprocal, then one product     */
 /*   decoded value: E2M1(q) * s_b * g (exact in fp64).                      */
 /*                                                                          */
 /*   The layer: x (bf16) is encoded per token row; the gate_up and down     */
@@ -455,9 +456,10 @@ static void orc_nvfp4_row(const float* v, int64_t K, uint8_t* codes, uint8_t* sf
         const int sb = (d6 > 0.0f) ? orc_e4m3_encode(ab / d6) : 0;
         sf[b] = (uint8_t)sb;
         const float dq = (float)orc_e4m3_decode(sb) * g;
+        const float rq = (dq > 0.0f) ? 1.0f / dq : 0.0f;
         for (int64_t kk = 0; kk < 16; ++kk) {
             const int64_t k = b * 16 + kk;
-            const int code = (dq > 0.0f) ? orc_e2m1_encode(v[k] / dq) : 0;
+            const int code = (dq > 0.0f) ? orc_e2m1_encode(v[k] * rq) : 0;
             if (k % 2 == 0) codes[k / 2] = (uint8_t)((codes[k / 2] & 0xF0) | code);
             else            codes[k / 2] = (uint8_t)((codes[k / 2] & 0x0F) | (code << 4));
         }

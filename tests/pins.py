@@ -550,9 +550,10 @@ def nvfp4_row_reference(v: np.ndarray):
         sb = brute_e4m3(np.float32(ab / d6)) if d6 > 0 else 0
         sf[b] = sb
         dq = np.float32(np.float32(e4m3_from_bits(sb)) * g)
+        rq = np.float32(np.float32(1.0) / dq) if dq > 0 else np.float32(0)
         for kk in range(16):
             k = 16 * b + kk
-            c = brute_force_code(float(np.float32(blk[kk] / dq))) if dq > 0 else 0
+            c = brute_force_code(float(np.float32(blk[kk] * rq))) if dq > 0 else 0
             codes[k // 2] |= np.uint8(c << (4 * (k % 2)))
     return codes, sf, g
 

@@ -50,6 +50,8 @@ MUTANTS = [
     ("nvfp4_row_scale", "const float g = amax / 2688.0f;", "const float g = amax / 1344.0f;"),
     ("nvfp4_block_max_of_first_block", "if (fabsf(v[b * 16 + kk]) > ab) ab = fabsf(v[b * 16 + kk]);",
      "if (fabsf(v[kk]) > ab) ab = fabsf(v[kk]);"),
+    ("nvfp4_divides_by_scale_factor_only", "const float rq = (dq > 0.0f) ? 1.0f / dq : 0.0f;",
+     "const float rq = (dq > 0.0f) ? 1.0f / (float)orc_e4m3_decode(sb) : 0.0f;"),
     ("nvfp4_act_not_bf16", "af[i] = orc_bf16_to_f32(orc_f64_to_bf16_rne(gv / (1.0 + exp(-gv)) * uv));",
      "af[i] = (float)(gv / (1.0 + exp(-gv)) * uv);"),
     ("nvfp4_down_reads_unencoded_act", "acc += orc_nvfp4_value(ac, as, ga, kk) *", "acc += (double)af[kk] *"),
