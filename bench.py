@@ -43,6 +43,7 @@ METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of B200 peak) at T=
 PREFILL_METRIC = "MoE-layer prefill tokens/s and tensor-core TFLOP/s at T=4096"
 HEADLINE = "decode_e128_t1"
 OTHERS = ["decode_e128_t64_zipf", "decode_e512_t1", "decode_e512_t4", "prefill_e128_t4096"]
+NVFP4_WORKLOAD = "nvfp4_prefill_e128_t4096"
 LAYERS = 48
 NOMINAL_HBM_GBS = 8000.0
 NOMINAL_FP4_TFLOPS = 9000.0
@@ -714,6 +715,93 @@ def run_int2(device, n_layers=16, steps=20):
             "status_bits": int(max(st_bits))}
 
 
+def run_nvfp4(device, n_layers=4, steps=8, warmup=3):
+    """The prefill layer (E 128, H 2048, I 768, top-8, T = 4096) on the block-scaled FP4
+    variant (fe_moe_load_nvfp4, FE_PATH_NVFP4): n_layers layers with their own seeded
+    weights, x and logits (each layer's weight images alone exceed L2), one CUDA graph of
+    the layers' forwards; the same layers on the exact tensor-core path beside it.  The
+    variant approximates the layer (its distance to the exact layer is measured by the
+    tests, not here)."""
+    import torch
+
+    import fp4_expert_gemv_b200 as fe
+    import synth
+    cfg = synth.WORKLOADS["prefill_e128_t4096"]
+    E, H, I, k, T = cfg["E"], cfg["H"], cfg["I"], cfg["top_k"], cfg["T"]
+    st = torch.cuda.current_stream().cuda_stream
+    handles = []
+    Wgu = torch.empty((E, H, 2 * I), dtype=torch.float32, device=device)
+    Wdn = torch.empty((E, I, H), dtype=torch.float32, device=device)
+    for layer in range(n_layers):
+        seed = synth.STACK_SEED0 + layer
+        synth.device_gate_up(Wgu.data_ptr(), seed, E, H, I, st)
+        synth.device_down(Wdn.data_ptr(), seed, E, I, H, st)
+        gc, gs = fe.pack_device(Wgu)
+        dc, ds = fe.pack_device(Wdn)
+        m = fe.MoELayer(E, H, I, max_T=T, max_top_k=k)
+        m.load_packed(gc, gs, dc, ds)
+        m.load_nvfp4(gc, gs, dc, ds)
+        handles.append(m)
+        del gc, gs, dc, ds
+    torch.cuda.synchronize()
+    del Wgu, Wdn
+    x, lg = stack_inputs(cfg, n_layers)
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    ld = torch.from_numpy(lg).to(device)
+    yd = torch.empty_like(xd)
+    peaks, src = measured_peaks()
+
+    def timed(path):
+        for m in handles:
+            m.set_path(path)
+        s = torch.cuda.Stream()
+
+        def calls():
+            for l, m in enumerate(handles):
+                fe.check(fe.fe_moe_forward(m.h, xd[l].data_ptr(), ld[l].data_ptr(), T, k, yd[l].data_ptr(),
+                                           s.cuda_stream), "fe_moe_forward")
+
+        with torch.cuda.stream(s):
+            calls()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            calls()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(steps):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / (steps * n_layers)
+
+    us_nv = timed(fe.PATH_NVFP4)
+    launches = handles[0].last_forward_info()[1]
+    us_tc = timed(fe.PATH_TCGEN05)
+    st_bits = [m.status()[1] for m in handles]
+    for m in handles:
+        m.close()
+    del xd, ld, yd
+    torch.cuda.empty_cache()
+    flops = 2.0 * T * k * (H * 2 * I + I * H)
+    tf = flops / (us_nv * 1e-6) / 1e12
+    fp4_peak = 4.0 * float(peaks["bf16_tflops_sustained"])   # measured bf16 (sustained) x the nominal fp4:bf16 ratio
+    return {"workload": "prefill_e128_t4096 on the block-scaled FP4 variant (NVFP4)", "layers": n_layers, "T": T,
+            "top_k": k, "us_per_layer": us_nv, "tokens_per_s": T / (us_nv * 1e-6), "launches_per_layer": launches,
+            "roofline": {"bound": "tensor", "achieved": tf, "unit": "TFLOP/s", "peak": fp4_peak,
+                         "frac": tf / fp4_peak, "frac_of_nominal_fp4_9pflops": tf / NOMINAL_FP4_TFLOPS,
+                         "peak_source": f"{src} bf16_tflops_sustained x 4 (nominal fp4 : bf16)"},
+            "exact_tcgen05_us_per_layer": us_tc, "speedup_vs_exact_path": us_tc / us_nv,
+            "accuracy": "an approximation of the layer: about 18 % l2 distance to the exact layer "
+                        "(tests/test_gpu_nvfp4.py prints it per case)",
+            "status_bits": int(max(st_bits))}
+
+
 def run_gpu(args):
     import torch
 
@@ -766,6 +854,7 @@ def run_gpu(args):
     if args.workload == "all":
         line["router_gemm"] = run_router(device)
         line["int2_mixed"] = run_int2(device)
+        line["nvfp4_prefill"] = run_nvfp4(device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
         reps = args.cpu_reps
@@ -790,13 +879,22 @@ def main(argv=None):
     ap.add_argument("--cpu-reps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true", help="skip the oracle check of the headline stack's output")
-    ap.add_argument("--workload", default="all", choices=["all", HEADLINE] + OTHERS,
-                    help="all: the headline workload plus the others under 'workloads'")
+    ap.add_argument("--workload", default="all", choices=["all", HEADLINE] + OTHERS + [NVFP4_WORKLOAD],
+                    help="all: the headline workload plus the others under 'workloads'; "
+                         f"{NVFP4_WORKLOAD}: only the block-scaled FP4 variant's record (--layers layers, "
+                         "--steps graph replays)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == NVFP4_WORKLOAD:
+        import torch
+        torch.cuda.set_device(0)
+        rec = run_nvfp4(torch.device("cuda", 0), n_layers=min(args.layers, 8), steps=args.steps,
+                        warmup=args.warmup)
+        print(json.dumps(rec), flush=True)
+        return 0
     return run_gpu(args)
 
 

@@ -83,6 +83,9 @@ struct fe_moe_s {
     float* nv_dng = nullptr;                // [E][H]
     uint8_t* nv_b = nullptr;                // [tile slots][max(H, I)/256] x kNvBChunk bytes
     float* nv_bg = nullptr;                 // [tile slots][256]
+    uint8_t* nv_xc = nullptr;               // x encoded per token: codes [max_T][H/2]
+    uint8_t* nv_xs = nullptr;               // scale factors [max_T][H/16]
+    float* nv_xg = nullptr;                 // row scales [max_T]
     float* rt_part = nullptr;               // router GEMM: K-split partials (router.cuh)
     unsigned* rt_ticket = nullptr;          // router GEMM: per 16-token tile, CTAs done
     uint32_t* status = nullptr;
@@ -160,7 +163,8 @@ void free_workspace(fe_moe_s* h)
     void* ptrs[] = {h->idx, h->w, h->counts, h->offsets, h->sorted_pair, h->pair_row, h->active, h->n_active,
                     h->max_count, h->act, h->o, h->status, h->x_stage, h->logits_stage, h->y_stage,
                     h->dec_part, h->dec_epoch, h->sg_table, h->tc_x, h->tc_xshift, h->tc_act, h->tc_ashift,
-                    h->tc_tiles, h->tc_ntiles, h->grp_bh, h->rt_part, h->rt_ticket, h->nv_b, h->nv_bg};
+                    h->tc_tiles, h->tc_ntiles, h->grp_bh, h->rt_part, h->rt_ticket, h->nv_b, h->nv_bg,
+                    h->nv_xc, h->nv_xs, h->nv_xg};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     h->idx = nullptr; h->w = nullptr; h->counts = nullptr; h->offsets = nullptr; h->sorted_pair = nullptr;
@@ -176,6 +180,8 @@ void free_workspace(fe_moe_s* h)
     h->rt_ticket = nullptr;
     h->nv_b = nullptr;
     h->nv_bg = nullptr;
+    h->nv_xc = h->nv_xs = nullptr;
+    h->nv_xg = nullptr;
     h->max_T = h->max_k = 0;
     h->work_bytes = 0;
 }
@@ -560,6 +566,19 @@ size_t nv_token_bytes(const fe_moe_s* h, size_t slots)
     return slots * (size_t)(std::max(h->H, h->I) / fe::kNvKc) * fe::kNvBChunk;
 }
 
+// Workspace of the block-scaled FP4 variant for max_T tokens and P pairs:
+// token images of every tile slot, and x encoded per token.
+cudaError_t nv_alloc_workspace(fe_moe_s* h, int max_T, size_t P, size_t* acc)
+{
+    const size_t slots = tc_max_tiles(h, P);
+    cudaError_t e = dmalloc(&h->nv_b, nv_token_bytes(h, slots), acc);
+    if (e == cudaSuccess) e = dmalloc(&h->nv_bg, slots * fe::kNvN, acc);
+    if (e == cudaSuccess) e = dmalloc(&h->nv_xc, (size_t)max_T * (h->H / 2), acc);
+    if (e == cudaSuccess) e = dmalloc(&h->nv_xs, (size_t)max_T * (h->H / 16), acc);
+    if (e == cudaSuccess) e = dmalloc(&h->nv_xg, (size_t)max_T, acc);
+    return e;
+}
+
 // Block-scaled FP4 variant (nvfp4.cuh): tile list, x rows gathered into NVFP4
 // token images, gate_up tiles (SwiGLU into act, bf16), act rows into token
 // images, down tiles (into o, bf16).  Routing and grouping ran before; the
@@ -569,9 +588,11 @@ fe_status nvfp4_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t 
     const int P = T * k;
     const int max_tiles = (int)tc_max_tiles(h, (size_t)P);
     fe::tc_tiles_kernel<<<1, 1024, 0, s>>>(h->counts, h->offsets, h->E, h->tc_tiles, h->tc_ntiles);
+    // x encoded once per token, then gathered into the tiles' images
+    fe::nvfp4_rows_kernel<true><<<(unsigned)((T + 7) / 8), 256, 0, s>>>(x, T, h->H, h->nv_xc, h->nv_xs, h->nv_xg);
     const unsigned row_blocks = (unsigned)(((size_t)max_tiles * fe::kNvN + 7) / 8);
-    fe::nvfp4_token_rows_kernel<<<row_blocks, 256, 0, s>>>(x, h->H, h->tc_tiles, h->tc_ntiles, h->sorted_pair, k, 1,
-                                                           h->nv_b, h->nv_bg);
+    fe::nvfp4_gather_rows_kernel<<<row_blocks, 256, 0, s>>>(h->nv_xc, h->nv_xs, h->nv_xg, h->H, h->tc_tiles,
+                                                            h->tc_ntiles, h->sorted_pair, k, h->nv_b, h->nv_bg);
     fe::NvParams np{};
     np.tiles = h->tc_tiles;
     np.n_tiles = h->tc_ntiles;
@@ -589,8 +610,7 @@ fe_status nvfp4_path(fe_moe_s* h, const uint16_t* x, int T, int k, cudaStream_t 
     FE_CUDA_TRY(cudaGetLastError());
     // act was left as bf16 rows by sorted position
     fe::nvfp4_token_rows_kernel<<<row_blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(h->act), h->I,
-                                                           h->tc_tiles, h->tc_ntiles, h->sorted_pair, k, 0, h->nv_b,
-                                                           h->nv_bg);
+                                                           h->tc_tiles, h->tc_ntiles, h->nv_b, h->nv_bg);
     np.a_img = h->nv_dn;
     np.a_g = h->nv_dng;
     np.MT = h->H / fe::kNvM;
@@ -712,10 +732,7 @@ fe_status fe_moe_reserve(fe_moe_t h, int max_T, int max_top_k)
         if (e == cudaSuccess) e = dmalloc(&h->tc_tiles, 3 * tc_max_tiles(h, P), &acc);
         if (e == cudaSuccess) e = dmalloc(&h->tc_ntiles, 1, &acc);
     }
-    if (h->nv_gu) {
-        if (e == cudaSuccess) e = dmalloc(&h->nv_b, nv_token_bytes(h, tc_max_tiles(h, P)), &acc);
-        if (e == cudaSuccess) e = dmalloc(&h->nv_bg, tc_max_tiles(h, P) * fe::kNvN, &acc);
-    }
+    if (h->nv_gu && e == cudaSuccess) e = nv_alloc_workspace(h, max_T, P, &acc);
     h->work_bytes = 0;
     for (auto& row : h->dec_planned)
         for (bool& b : row) b = false;
@@ -817,17 +834,14 @@ fe_status fe_moe_load_nvfp4(fe_moe_t h, const uint8_t* gu_codes, const uint16_t*
         if (e == cudaSuccess) e = dmalloc(&h->nv_dn, (size_t)E * (H / fe::kNvM) * (I / fe::kNvKc) * fe::kNvAChunk, &acc);
         if (e == cudaSuccess) e = dmalloc(&h->nv_gug, (size_t)E * 2 * I, &acc);
         if (e == cudaSuccess) e = dmalloc(&h->nv_dng, (size_t)E * H, &acc);
-        if (e == cudaSuccess && h->max_T > 0) {
-            const size_t slots = tc_max_tiles(h, (size_t)h->max_T * h->max_k);
-            e = dmalloc(&h->nv_b, nv_token_bytes(h, slots), &h->work_bytes);
-            if (e == cudaSuccess) e = dmalloc(&h->nv_bg, slots * fe::kNvN, &h->work_bytes);
-        }
+        if (e == cudaSuccess && h->max_T > 0)
+            e = nv_alloc_workspace(h, h->max_T, (size_t)h->max_T * h->max_k, &h->work_bytes);
         if (e != cudaSuccess) {
-            void* ptrs[] = {h->nv_gu, h->nv_dn, h->nv_gug, h->nv_dng, h->nv_b, h->nv_bg};
+            void* ptrs[] = {h->nv_gu, h->nv_dn, h->nv_gug, h->nv_dng, h->nv_b, h->nv_bg, h->nv_xc, h->nv_xs, h->nv_xg};
             for (void* q : ptrs)
                 if (q) cudaFree(q);
-            h->nv_gu = h->nv_dn = h->nv_b = nullptr;
-            h->nv_gug = h->nv_dng = h->nv_bg = nullptr;
+            h->nv_gu = h->nv_dn = h->nv_b = h->nv_xc = h->nv_xs = nullptr;
+            h->nv_gug = h->nv_dng = h->nv_bg = h->nv_xg = nullptr;
             return record_cuda(e, "fe_moe_load_nvfp4 allocation");
         }
         h->weight_bytes += acc;
@@ -860,10 +874,11 @@ fe_status fe_moe_nvfp4_quantize_device(const float* src, int64_t rows, int64_t K
                                        float* row_scale, fe_stream_t stream)
 {
     if (!src || !codes || !sf || !row_scale || rows < 0 || K < 16 || K % 16 || rows > (int64_t)1 << 26 ||
-        K > (int64_t)1 << 20)
+        K > (int64_t)1 << 20 || !aligned16(src) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
+        (reinterpret_cast<uintptr_t>(row_scale) & 3u))
         return FE_ERR_INVALID_ARG;
     if (rows == 0) return FE_OK;
-    fe::nvfp4_rows_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+    fe::nvfp4_rows_kernel<false><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
         src, (int)rows, (int)K, codes, sf, row_scale);
     return cudaGetLastError() == cudaSuccess ? FE_OK : FE_ERR_CUDA;
 }
@@ -966,6 +981,7 @@ fe_status forward_impl(fe_moe_t h, const void* x_bf16, const float* router_logit
     if (h->has_int2) return FE_ERR_UNSUPPORTED;
     if (h->path == FE_PATH_NVFP4) {
         if (!h->nv_gu || !h->nv_b || !h->tc_tiles) return FE_ERR_UNSUPPORTED;
+        if (!aligned16(x_bf16)) return FE_ERR_INVALID_ARG;   // the x rows are read in 16-byte pieces
         const fe_status rs = route_and_group(h, router_logits, T, top_k, nullptr, s);
         if (rs != FE_OK) return rs;
         const fe_status st = nvfp4_path(h, static_cast<const uint16_t*>(x_bf16), T, top_k, s);
@@ -978,7 +994,7 @@ fe_status forward_impl(fe_moe_t h, const void* x_bf16, const float* router_logit
         h->last_k = top_k;
         h->last_path = FE_PATH_NVFP4;
         const bool large_route = T >= kRouteLargeTokens && fe::route_large_ok(h->E, top_k);
-        h->last_kernels = (large_route ? 4 : 1) + 5 + 1;   // routing, tiles + 2 x (token images, tiles), combine
+        h->last_kernels = (large_route ? 4 : 1) + 6 + 1;   // routing, tile list, x rows, 2 x (images, tiles), combine
         return FE_OK;
     }
 

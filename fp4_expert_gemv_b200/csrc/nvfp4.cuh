@@ -12,10 +12,10 @@
 //
 //   g   = amax|v| / 2688               (6 * 448: the row's fp32 scale)
 //   s_b = E4M3(amax_b / (6 g))          per block b of 16, nearest, ties even, <= 448
-//   q   = E2M1(v / (s_b g))             nearest, ties even, |.| <= 6
+//   q   = E2M1(v * r_b), r_b = 1 / (s_b g)   nearest, ties even, |.| <= 6
 //
-// every step in fp32 (IEEE division and products, no contraction), so that
-// the codes are the same wherever they are computed.  The product of two
+// every step in fp32 (IEEE division, reciprocal and products, no
+// contraction), so that the codes are the same wherever they are computed.  The product of two
 // encoded rows is sum_b s_b^x s_b^w sum_k q^x q^w, times g^x g^w: the tensor
 // core forms the block-scaled sum, the epilogue multiplies by the row scales.
 //
@@ -29,7 +29,6 @@
 // per forward, one 256-row slot per tile of the tile list (tcgen05.cuh).
 #pragma once
 
-#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "bulk.cuh"
@@ -108,11 +107,23 @@ FE_DEV float e2m1_value(uint32_t q)
 // Nearest E4M3 (ties to even) of t >= 0, saturating at 448.
 FE_DEV uint32_t e4m3_rn(float t) { return (uint32_t)__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3) & 0x7Fu; }
 
-// Nearest E2M1 code (ties to even, |.| <= 6); a zero magnitude is code 0.
-FE_DEV uint32_t e2m1_rn(float r)
+// Eight values -> eight E2M1 codes (nearest, ties to even, |.| <= 6) in one
+// word, r[i] in bits 4i .. 4i+3.  cvt ... e2m1x2 puts its first source in the
+// high nibble.  A zero magnitude is written as code 0 (no negative zero).
+FE_DEV uint32_t e2m1x8_rn(const float* r)
 {
-    const uint32_t q = (uint32_t)__nv_cvt_float_to_fp4(r, __NV_E2M1, cudaRoundNearest) & 0xFu;
-    return (q & 7u) ? q : 0u;
+    uint32_t w;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(w)
+        : "f"(r[0]), "f"(r[1]), "f"(r[2]), "f"(r[3]), "f"(r[4]), "f"(r[5]), "f"(r[6]), "f"(r[7]));
+    const uint32_t m = w & 0x77777777u;                                  // magnitudes
+    const uint32_t nz = (m | (m >> 1) | (m >> 2)) & 0x11111111u;         // per nibble: magnitude != 0
+    return m | (w & (nz << 3));
 }
 
 // Row scale g and 6 g from the row's largest magnitude.
@@ -131,12 +142,12 @@ FE_DEV uint32_t nv_encode_block(const float (&v)[16], float g, float d6, uint32_
     for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(v[i]));
     const uint32_t sb = d6 > 0.0f ? e4m3_rn(__fdiv_rn(ab, d6)) : 0u;
     const float dq = __fmul_rn(e4m3_value(sb), g);
-    codes[0] = codes[1] = 0u;
+    const float rq = dq > 0.0f ? __frcp_rn(dq) : 0.0f;
+    float r[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const uint32_t q = dq > 0.0f ? e2m1_rn(__fdiv_rn(v[i], dq)) : 0u;
-        codes[i >> 3] |= q << (4 * (i & 7));
-    }
+    for (int i = 0; i < 16; ++i) r[i] = __fmul_rn(v[i], rq);
+    codes[0] = e2m1x8_rn(r);
+    codes[1] = e2m1x8_rn(r + 8);
     return sb;
 }
 
@@ -152,23 +163,45 @@ FE_DEV void bf16x16_to_f32(const uint16_t* src, float (&v)[16])
     }
 }
 
-// Rows of fp32 values -> NVFP4 in plain row order: codes [R][K/2], scale factors
-// [R][K/16], row scales [R].  One warp per row.
-__global__ void nvfp4_rows_kernel(const float* src, int R, int K, uint8_t* codes, uint8_t* sf, float* g_out)
+// 16 values of a row: bf16 (two 16-byte loads) or fp32 (four).
+template <bool BF16>
+FE_DEV void nv_load16(const void* row, int b, float (&v)[16])
+{
+    if (BF16) {
+        bf16x16_to_f32(static_cast<const uint16_t*>(row) + 16 * b, v);
+    } else {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(row) + 16 * b);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 q = p[i];
+            v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
+        }
+    }
+}
+
+// Rows of bf16 or fp32 values -> NVFP4 in plain row order: codes [R][K/2],
+// scale factors [R][K/16], row scales [R].  One warp per row.
+template <bool BF16>
+__global__ void nvfp4_rows_kernel(const void* src, int R, int K, uint8_t* codes, uint8_t* sf, float* g_out)
 {
     const int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
     if (r >= R) return;
-    const float* row = src + (size_t)r * K;
+    const void* row = BF16 ? (const void*)(static_cast<const uint16_t*>(src) + (size_t)r * K)
+                           : (const void*)(static_cast<const float*>(src) + (size_t)r * K);
     float amax = 0.0f;
-    for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(row[k]));
+    for (int b = lane; b < K / 16; b += 32) {
+        float v[16];
+        nv_load16<BF16>(row, b, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     float g, d6;
     nv_row_scale(amax, g, d6);
     for (int b = lane; b < K / 16; b += 32) {
         float v[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = row[16 * b + i];
+        nv_load16<BF16>(row, b, v);
         uint32_t c[2];
         sf[(size_t)r * (K / 16) + b] = (uint8_t)nv_encode_block(v, g, d6, c);
         *reinterpret_cast<uint2*>(codes + (size_t)r * (K / 2) + 8 * b) = make_uint2(c[0], c[1]);
@@ -214,12 +247,42 @@ __global__ void nvfp4_weights_kernel(const uint8_t* codes, const uint16_t* scale
 }
 
 // ---- token images (every forward) --------------------------------------------------
-// One warp per (tile slot, row n < 256): the row is x[token of sorted position
-// pos0 + n] (gather, gate_up) or act[pos0 + n] (down), bf16, K values; rows past
-// the tile's count, and slots past the tile count, are written as zeros.  Image
-// chunk (slot, stage) at (slot * KC + stage) * kNvBChunk; row scale gb[slot][n].
+// Rows past a tile's count are written as zeros; slots past the tile count are
+// left alone (no CTA reads them).  Image chunk (slot, stage) at (slot * KC +
+// stage) * kNvBChunk; row scale gb[slot][n].
+
+// gate_up: one warp per (tile slot, row n < 256) copies the encoded row of the
+// token of sorted position pos0 + n (codes [T][K/2], scale factors [T][K/16],
+// row scales [T], from nvfp4_rows_kernel) into the slot's image.
+__global__ void nvfp4_gather_rows_kernel(const uint8_t* codes, const uint8_t* sf, const float* g, int K,
+                                         const int32_t* tiles, const int32_t* n_tiles, const int32_t* sorted_pair,
+                                         int top_k, uint8_t* img, float* gb)
+{
+    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int slot = (int)(wid / kNvN), n = (int)(wid % kNvN);
+    if (slot >= *n_tiles) return;
+    const int pos0 = tiles[3 * slot + 1], rows = tiles[3 * slot + 2];
+    uint8_t* base = img + (size_t)slot * (K / kNvKc) * kNvBChunk;
+    const bool live = n < rows;
+    const int t = live ? sorted_pair[pos0 + n] / top_k : 0;
+    const uint4* src = reinterpret_cast<const uint4*>(codes + (size_t)t * (K / 2));
+    for (int c = lane; c < K / 32; c += 32) {   // 16-byte chunks: 8 per stage
+        const uint4 v = live ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(base + (size_t)(c >> 3) * kNvBChunk + nv_code_off(n, 16 * (c & 7))) = v;
+    }
+    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(sf + (size_t)t * (K / 16));
+    for (int w = lane; w < K / 64; w += 32) {   // one word per k-block: 4 per stage
+        const uint32_t v = live ? ssrc[w] : 0u;
+        *reinterpret_cast<uint32_t*>(base + (size_t)(w >> 2) * kNvBChunk + nv_sfb_off(n, 4 * (w & 3))) = v;
+    }
+    if (lane == 0) gb[(size_t)slot * kNvN + n] = live ? g[t] : 0.0f;
+}
+
+// down: one warp per (tile slot, row n < 256) encodes act row pos0 + n (bf16,
+// rows by sorted position) straight into the slot's image.
 __global__ void nvfp4_token_rows_kernel(const uint16_t* src, int K, const int32_t* tiles, const int32_t* n_tiles,
-                                        const int32_t* sorted_pair, int top_k, int gather, uint8_t* img, float* gb)
+                                        uint8_t* img, float* gb)
 {
     const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -237,8 +300,7 @@ __global__ void nvfp4_token_rows_kernel(const uint16_t* src, int K, const int32_
         if (lane == 0) gb[(size_t)slot * kNvN + n] = 0.0f;
         return;
     }
-    const int pos = pos0 + n;
-    const uint16_t* row = src + (size_t)(gather ? sorted_pair[pos] / top_k : pos) * K;
+    const uint16_t* row = src + (size_t)(pos0 + n) * K;
     float amax = 0.0f;
     for (int b = lane; b < K / 16; b += 32) {
         float v[16];

@@ -143,7 +143,9 @@ fe_status fe_moe_load_packed(fe_moe_t h, const uint8_t* gate_up_codes, const uin
  * tolerance).  Needs H % 256 == 0 and I % 256 == 0 (else FE_ERR_UNSUPPORTED)
  * and fe_moe_load_packed for the routing workspace's layer; token images are
  * workspace of fe_moe_reserve (tile slots x max(H, I) / 256 x 36 KiB).  Work is
- * enqueued on stream; host sources are staged through a stream-ordered buffer. */
+ * enqueued on stream; host sources are staged through a stream-ordered buffer.
+ * On this path fe_moe_forward also needs x 16-byte aligned (else
+ * FE_ERR_INVALID_ARG). */
 fe_status fe_moe_load_nvfp4(fe_moe_t h, const uint8_t* gate_up_codes, const uint16_t* gate_up_scales,
                             const uint8_t* down_codes, const uint16_t* down_scales, int src_on_device,
                             fe_stream_t stream);
@@ -152,8 +154,8 @@ fe_status fe_moe_load_nvfp4(fe_moe_t h, const uint8_t* gate_up_codes, const uint
  * device float [rows][K] -> device codes uint8 [rows][K/2] (two per byte, the
  * low nibble for the even k; bit 3 the sign), E4M3 scale factors uint8
  * [rows][K/16], row scales float [rows].  A value decodes as E2M1(code) *
- * E4M3(scale factor) * row scale.  K % 16 == 0, K >= 16 (else
- * FE_ERR_INVALID_ARG).  Asynchronous on stream. */
+ * E4M3(scale factor) * row scale.  K % 16 == 0, K >= 16, src 16-byte and
+ * codes 8-byte aligned (else FE_ERR_INVALID_ARG).  Asynchronous on stream. */
 fe_status fe_moe_nvfp4_quantize_device(const float* src, int64_t rows, int64_t K, uint8_t* codes, uint8_t* sf,
                                        float* row_scale, fe_stream_t stream);
 
