@@ -483,7 +483,8 @@ def test_argument_errors(torch_cuda):
         assert fe.fe_moe_forward(h, None, 16, 1, 2, 32, None) == fe.FE_ERR_INVALID_ARG
         assert fe.fe_moe_forward(h, 16, 16, 1, 2, 16, None) == fe.FE_ERR_INVALID_ARG   # y aliases x
         assert fe.fe_moe_forward(h, 16, 16, -1, 2, 32, None) == fe.FE_ERR_INVALID_ARG
-        assert fe.fe_moe_set_path(h, 4) == fe.FE_ERR_INVALID_ARG
+        assert fe.fe_moe_set_path(h, fe.PATH_NVFP4 + 1) == fe.FE_ERR_INVALID_ARG
+        assert fe.fe_moe_set_path(h, -1) == fe.FE_ERR_INVALID_ARG
         assert fe.fe_moe_set_path(h, fe.PATH_AUTO) == fe.FE_OK
         st, = [fe.fe_moe_get_status(h, None)]
         assert st == fe.FE_OK
