@@ -245,8 +245,10 @@ fe_status fe_moe_get_status(fe_moe_t h, uint32_t* bits);
                                    + combine: an approximation of the layer (fe_moe_load_nvfp4); any T;
                                    never chosen by FE_PATH_AUTO */
 
-/* Force a compute path (FE_PATH_*); FE_ERR_UNSUPPORTED from forward if the
- * forced path cannot run the call.  For tests and measurements. */
+/* Force a compute path (FE_PATH_*; any other value: FE_ERR_INVALID_ARG);
+ * FE_ERR_UNSUPPORTED from forward if the forced path cannot run the call.
+ * A stack whose layers have a forced path runs one layer at a time on it.
+ * For tests and measurements (and to choose the FE_PATH_NVFP4 variant). */
 fe_status fe_moe_set_path(fe_moe_t h, int path);
 
 /* Which path the last successful forward took and how many kernels it
