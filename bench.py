@@ -715,6 +715,18 @@ def run_int2(device, n_layers=16, steps=20):
             "status_bits": int(max(st_bits))}
 
 
+def nvfp4_roofline(us_per_layer, T, k, H, I, peaks, src):
+    """The block-scaled FP4 record's roofline: the layer's 2 T k (2 H I + I H) FLOPs per
+    us_per_layer, against the measured sustained bf16 rate times 4 (the nominal FP4 : bf16
+    ratio of the dense tensor peaks, 9 : 2.25 PFLOP/s)."""
+    flops = 2.0 * T * k * (H * 2 * I + I * H)
+    tf = flops / (us_per_layer * 1e-6) / 1e12
+    fp4_peak = 4.0 * float(peaks["bf16_tflops_sustained"])
+    return {"bound": "tensor", "achieved": tf, "unit": "TFLOP/s", "peak": fp4_peak, "frac": tf / fp4_peak,
+            "frac_of_nominal_fp4_9pflops": tf / NOMINAL_FP4_TFLOPS,
+            "peak_source": f"{src} bf16_tflops_sustained x 4 (nominal fp4 : bf16)"}
+
+
 def run_nvfp4(device, n_layers=4, steps=8, warmup=3):
     """The prefill layer (E 128, H 2048, I 768, top-8, T = 4096) on the block-scaled FP4
     variant (fe_moe_load_nvfp4, FE_PATH_NVFP4): n_layers layers with their own seeded
@@ -788,14 +800,9 @@ def run_nvfp4(device, n_layers=4, steps=8, warmup=3):
         m.close()
     del xd, ld, yd
     torch.cuda.empty_cache()
-    flops = 2.0 * T * k * (H * 2 * I + I * H)
-    tf = flops / (us_nv * 1e-6) / 1e12
-    fp4_peak = 4.0 * float(peaks["bf16_tflops_sustained"])   # measured bf16 (sustained) x the nominal fp4:bf16 ratio
     return {"workload": "prefill_e128_t4096 on the block-scaled FP4 variant (NVFP4)", "layers": n_layers, "T": T,
             "top_k": k, "us_per_layer": us_nv, "tokens_per_s": T / (us_nv * 1e-6), "launches_per_layer": launches,
-            "roofline": {"bound": "tensor", "achieved": tf, "unit": "TFLOP/s", "peak": fp4_peak,
-                         "frac": tf / fp4_peak, "frac_of_nominal_fp4_9pflops": tf / NOMINAL_FP4_TFLOPS,
-                         "peak_source": f"{src} bf16_tflops_sustained x 4 (nominal fp4 : bf16)"},
+            "roofline": nvfp4_roofline(us_nv, T, k, H, I, peaks, src),
             "exact_tcgen05_us_per_layer": us_tc, "speedup_vs_exact_path": us_tc / us_nv,
             "accuracy": "an approximation of the layer: about 18 % l2 distance to the exact layer "
                         "(tests/test_gpu_nvfp4.py prints it per case)",

@@ -133,6 +133,17 @@ int main()
                 CHECK(fe::nv_gate_up_column(Rg, I) == i && fe::nv_gate_up_column(Rg + 16, I) == I + i, "I=%d i=%d", I, i);
             }
         }
+        // the scale-factor layout of CUTLASS's sm100 block-scaled K-major atom: per 128 rows and
+        // 4 factors (one 64-wide k-block), shape ((32, 4), (16, 4)) with strides ((16, 4), (0, 1))
+        // over (row, k); further 128-row blocks 512 bytes apart, k-blocks after all rows' blocks
+        for (int n = 0; n < fe::kNvN; ++n)
+            for (int k = 0; k < fe::kNvKc; ++k) {
+                const int q = k / 64, kk = k % 64, nb = n / 128, m = n % 128;
+                const uint32_t atom = 16u * (m % 32) + 4u * (m / 32) + 0u * (kk % 16) + 1u * (kk / 16);
+                CHECK(fe::nv_sfb_off(n, k / 16) == fe::kNvBCodes + 1024u * q + 512u * nb + atom, "B n=%d k=%d", n, k);
+                if (n < fe::kNvM)
+                    CHECK(fe::nv_sfa_off(n, k / 16) == fe::kNvACodes + 512u * q + atom, "A n=%d k=%d", n, k);
+            }
         CHECK(fe::nv_smem_bytes() <= kMaxSmem, "NVFP4 tiles %u", fe::nv_smem_bytes());
         CHECK(256u + 4u * fe::kNvSfCols <= fe::kNvTmemCols, "TMEM columns");
         CHECK(fe::nv_instr_desc(256) == ((1u << 7) | (1u << 10) | (32u << 17) | (8u << 24)), "instruction descriptor");

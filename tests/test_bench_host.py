@@ -47,3 +47,17 @@ def test_kernel_label_follows_the_launch_count():
     assert "per token" in bench.kernel_label(3, 4, 4)
     assert "decode_kernel" in bench.kernel_label(3, 48, 1) and "stack" not in bench.kernel_label(3, 48, 1)
     assert "sg_kernel" in bench.kernel_label(1, 336, 64)
+
+
+def test_nvfp4_roofline_arithmetic():
+    """The block-scaled FP4 record: 309.24 GFLOP per prefill layer, the FP4 peak as 4 x the
+    measured sustained bf16 rate."""
+    import bench
+    peaks = {"bf16_tflops_sustained": 1400.0}
+    r = bench.nvfp4_roofline(1000.0, 4096, 8, 2048, 768, peaks, "measured")
+    flops = 2.0 * 4096 * 8 * 3 * 2048 * 768
+    assert abs(flops - 309.237645312e9) < 1.0
+    assert abs(r["achieved"] - flops / 1e-3 / 1e12) < 1e-9
+    assert r["peak"] == 5600.0 and abs(r["frac"] - r["achieved"] / 5600.0) < 1e-12
+    assert abs(r["frac_of_nominal_fp4_9pflops"] - r["achieved"] / 9000.0) < 1e-12
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
