@@ -98,3 +98,21 @@ def test_synth_device_library_is_built():
     lib = ctypes.CDLL(path)
     for n in ("fe_synth_gate_up", "fe_synth_down", "fe_synth_normal"):
         assert hasattr(lib, n)
+
+
+def test_nvfp4_entry_points_refuse_bad_arguments_on_the_host():
+    """The block-scaled FP4 entry points validate before touching the device (no GPU needed):
+    null or misaligned pointers, K not a multiple of 16, negative rows, a null handle."""
+    import fp4_expert_gemv_b200 as fe
+    q = fe.fe_moe_nvfp4_quantize_device
+    A = 1 << 20   # aligned fake addresses: never dereferenced, every call here is refused first
+    assert q(None, 1, 16, A, A, A, None) == fe.FE_ERR_INVALID_ARG
+    assert q(A, 1, 16, None, A, A, None) == fe.FE_ERR_INVALID_ARG
+    assert q(A, 1, 15, A, A, A, None) == fe.FE_ERR_INVALID_ARG
+    assert q(A, 1, 0, A, A, A, None) == fe.FE_ERR_INVALID_ARG
+    assert q(A, -1, 16, A, A, A, None) == fe.FE_ERR_INVALID_ARG
+    assert q(A + 8, 1, 16, A, A, A, None) == fe.FE_ERR_INVALID_ARG      # src not 16-byte aligned
+    assert q(A, 1, 16, A + 4, A, A, None) == fe.FE_ERR_INVALID_ARG      # codes not 8-byte aligned
+    assert q(A, 0, 16, A, A, A, None) == fe.FE_OK                        # nothing to do
+    assert fe.fe_moe_load_nvfp4(None, A, A, A, A, 1, None) == fe.FE_ERR_INVALID_ARG
+    assert fe.fe_moe_set_path(None, fe.PATH_NVFP4) == fe.FE_ERR_INVALID_ARG
